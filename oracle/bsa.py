@@ -1,0 +1,92 @@
+"""Oracle: query pruning and reconstruction of bidirectional sparse attention (fp64).
+
+Source: ``bsa_attn`` page (FastVideo API docs), ``BSAAttentionImpl.forward``: the tile-ordered
+sequence is viewed as blocks of ``block_size`` tokens (the length must be an exact multiple), the
+queries of each block are pruned, KV blocks are selected from the pruned queries, attention runs
+for the kept queries only, and the pruned positions are filled back in before the output is
+returned in tile order. ``BSAAttentionImpl.__init__`` fixes the contract: no grouped-query
+attention, no causal mask, softmax scale 1/sqrt(D).
+
+The pages name the pruning and reconstruction helpers but do not print their bodies. Readings
+taken here (the workload definition prunes by a cosine threshold):
+* a query row of a block is pruned iff its cosine similarity to the mean of all rows of the block
+  exceeds the threshold; a cosine with a zero-norm operand counts as 0;
+* if every row of a block would be pruned, the row with the lowest cosine (lowest index on ties)
+  is kept;
+* a pruned row takes the output of the kept row of the same block and head that it is most
+  cosine-similar to (lowest index on ties);
+* KV selection pools the queries over the kept rows of the block only.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+TILE_ELEMS = 64
+
+
+def _cos(a: np.ndarray, b: np.ndarray) -> float:
+    na = float(np.sqrt(np.dot(a, a)))
+    nb = float(np.sqrt(np.dot(b, b)))
+    if na == 0.0 or nb == 0.0:
+        return 0.0
+    return float(np.dot(a, b)) / (na * nb)
+
+
+def prune_block(rows: np.ndarray, thresh: float):
+    """One block ``[n, D]`` -> ``(keep bool[n], src int[n], cos_to_mean float[n])``.
+
+    ``src[i] == i`` for kept rows; for pruned rows it names the kept row whose output they copy."""
+    rows = rows.astype(np.float64)
+    n = rows.shape[0]
+    mu = rows.sum(axis=0) / n
+    cmean = np.array([_cos(rows[i], mu) for i in range(n)])
+    keep = ~(cmean > thresh)
+    if not keep.any():
+        keep[int(np.argmin(cmean))] = True
+    kept = np.nonzero(keep)[0]
+    src = np.arange(n)
+    for i in range(n):
+        if keep[i]:
+            continue
+        best_j, best_c = -1, -np.inf
+        for j in kept:
+            c = _cos(rows[i], rows[j])
+            if c > best_c:
+                best_j, best_c = int(j), c
+        src[i] = best_j
+    return keep, src, cmean
+
+
+def prune_queries(qt: np.ndarray, thresh: float):
+    """Tile-ordered queries ``[B, 64*nT, heads, D]`` (no pad rows) ->
+    ``keep [B, heads, nT, 64]`` bool, ``src [B, heads, nT, 64]`` int, ``cos [B, heads, nT, 64]``."""
+    B, Lp, nh, D = qt.shape
+    nT = Lp // TILE_ELEMS
+    keep = np.zeros((B, nh, nT, TILE_ELEMS), dtype=bool)
+    src = np.zeros((B, nh, nT, TILE_ELEMS), dtype=np.int64)
+    cosm = np.zeros((B, nh, nT, TILE_ELEMS), dtype=np.float64)
+    for b in range(B):
+        for h in range(nh):
+            for i in range(nT):
+                rows = qt[b, TILE_ELEMS * i:TILE_ELEMS * (i + 1), h, :]
+                keep[b, h, i], src[b, h, i], cosm[b, h, i] = prune_block(rows, thresh)
+    return keep, src, cosm
+
+
+def pooled_kept_queries(qt: np.ndarray, keep: np.ndarray) -> np.ndarray:
+    """Mean of each block's kept query rows: ``[B, heads, nT, D]`` fp64."""
+    B, Lp, nh, D = qt.shape
+    nT = Lp // TILE_ELEMS
+    out = np.zeros((B, nh, nT, D), dtype=np.float64)
+    for b in range(B):
+        for h in range(nh):
+            for i in range(nT):
+                rows = qt[b, TILE_ELEMS * i:TILE_ELEMS * (i + 1), h, :].astype(np.float64)
+                kk = keep[b, h, i]
+                out[b, h, i] = rows[kk].sum(axis=0) / int(kk.sum())
+    return out
+
+
+def reconstruct_pruned(o_block: np.ndarray, src: np.ndarray) -> np.ndarray:
+    """Fill pruned rows of one block's output ``[64, D]`` from their source rows."""
+    return o_block[src]

@@ -1,0 +1,34 @@
+"""Oracle: mean pooling of each 64-token tile (fp64).
+
+Source: ``fastvideo.attention.backends`` page, ``sla.mean_pool`` (one mean per block along the
+sequence) as used by ``sla.get_block_map`` for both queries and keys.
+
+Reading taken where the pages are silent: a partial tile is averaged over its valid tokens only
+(divide by the tile's valid count, not by 64); pad rows never enter the mean.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+TILE_ELEMS = 64
+
+
+def tile_mean_pool(y: np.ndarray, vc: np.ndarray) -> np.ndarray:
+    """Padded tile order ``[B, 64*nT, heads, D]`` -> pooled ``[B, heads, nT, D]`` (fp64)."""
+    B, Lp, nh, D = y.shape
+    nT = Lp // TILE_ELEMS
+    assert nT * TILE_ELEMS == Lp and len(vc) == nT
+    out = np.zeros((B, nh, nT, D), dtype=np.float64)
+    for i in range(nT):
+        n = int(vc[i])
+        rows = y[:, TILE_ELEMS * i:TILE_ELEMS * i + n].astype(np.float64)  # [B, n, heads, D]
+        out[:, :, i, :] = rows.sum(axis=1) / n
+    return out
+
+
+def block_mean_pool_rows(rows: np.ndarray, keep: np.ndarray) -> np.ndarray:
+    """Mean of the rows of one block selected by boolean ``keep`` (fp64). Empty selection -> 0."""
+    n = int(keep.sum())
+    if n == 0:
+        return np.zeros(rows.shape[-1], dtype=np.float64)
+    return rows[keep].astype(np.float64).sum(axis=0) / n
