@@ -1,0 +1,427 @@
+"""Benchmark of the tile-sparse attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config small] [--impl ours|reference]
+
+One step = the whole hot path over one batch of the workload: scatter Q, K, V into 4x4x4 tile
+order, coarse selection (pool Q and K, score tile pairs, keep the top-k key tiles per query tile;
+or the workload's own selection mode), block-sparse attention over the kept tile pairs, gather the
+output back to raster order. Inputs are resident in HBM when the timed region starts; the raster
+Q, K, V (264 MB at the small layer) exceed the 126 MB L2, so no flush is inserted.
+
+The metric is effective TFLOPS over kept blocks (4 * 64 * 64 * D FLOPs per kept query-tile /
+key-tile pair) per step, with ms per call, and the fraction of the roofline of the dominant kernel
+(the attention) measured live with CUDA events. ``e2e`` repeats the measurement through the public
+API with host buffers: every step copies Q, K, V from pinned host memory and the output back.
+
+With N > 1 (torchrun), every rank runs its own replica of the workload (independent batches, no
+data exchange); ``value`` is the kept-block FLOPs of all ranks over the max-over-ranks time.
+
+``--impl reference`` times the CPU oracle (fp64 numpy) on a bounded sample of the same workload
+on the host cores; it is the reported CPU baseline, not a target.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "ms/call and effective TFLOPS (kept blocks) at 28,672 tok×12 heads; % of roofline"
+FLOPS_PER_PAIR = lambda D: 4 * 64 * 64 * D  # noqa: E731
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def _describe(w) -> str:
+    sel = {"topk": f"top-{w.k} of {w.nT} tiles",
+           "bsa": f"BSA: prune cos>{w.cos_thresh}, mass {w.mass}",
+           "mask": f"fixed {w.mask} block mask"}[w.mode]
+    return (f"{w.name}: B={w.B}, heads={w.heads}, D={w.D}, grid {w.T}x{w.H}x{w.W} "
+            f"({w.L:,} tokens, {w.nT} tiles of 4x4x4), {sel}")
+
+
+# --------------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the measured window."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 100):
+        self.index = index
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", str(period_ms)],
+                stdout=self.file, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [[c.strip() for c in ln.split(",")] for ln in f if ln.strip()]
+        os.unlink(self.file.name)
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in rows for j in range(4) if r[5 + j] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------------- oracle arm
+
+def oracle_sample(w, q, k, v, heads, q_tiles_per_head=None):
+    """Run the CPU oracle's whole path for the given heads (tiling, pooling, scores, selection,
+    attention for the first ``q_tiles_per_head`` query tiles, or all). Returns (seconds, flops,
+    pairs) for the sample."""
+    import numpy as np
+    import torch
+
+    from oracle import attention, bsa, pool, select, tiling
+
+    D = w.D
+    t0 = time.perf_counter()
+    pairs = 0
+    vc = tiling.variable_block_sizes(w.T, w.H, w.W)
+    mask = None
+    if w.mode == "mask":
+        from block_sparse_video_tile3d_b200 import workloads
+        mask = workloads.block_mask(w).numpy()
+    for b in range(w.B):
+        for h in heads:
+            sl = lambda x: x[b:b + 1, :, h:h + 1].to(torch.float64).numpy()  # noqa: E731
+            qt, kt, vt = (tiling.tile_scatter(sl(x), w.T, w.H, w.W) for x in (q, k, v))
+            keep = src = None
+            if w.mode == "mask":
+                sets = select.map_to_sets(mask[b:b + 1, h:h + 1])
+            else:
+                pk = pool.tile_mean_pool(kt, vc)
+                if w.mode == "bsa":
+                    keep, src, _ = bsa.prune_queries(qt, w.cos_thresh)
+                    pq = bsa.pooled_kept_queries(qt, keep)
+                else:
+                    pq = pool.tile_mean_pool(qt, vc)
+                S = select.tile_scores(pq, pk)
+                sets = select.select_topk(S, w.k) if w.mode == "topk" else \
+                    select.select_mass(S, w.scale, w.mass, w.min_kv)
+            n = w.nT if q_tiles_per_head is None else min(q_tiles_per_head, w.nT)
+            tiles = [(0, 0, i) for i in range(n)]
+            attention.block_sparse_attention(qt, kt, vt, vc, sets, w.scale, keep=keep, src=src,
+                                             q_tiles=tiles)
+            pairs += sum(len(sets[0][0][i]) for i in range(n))
+    sec = time.perf_counter() - t0
+    return sec, pairs * FLOPS_PER_PAIR(D), pairs
+
+
+def _cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, q, k, v, budget_s: float = 20.0) -> dict:
+    """Oracle throughput on a bounded sample (about ``budget_s`` of CPU work), in TFLOPS over the
+    kept blocks it computed, with the full-call time extrapolated from it."""
+    # calibrate on a quarter of one head, then size the sample in whole heads
+    sec, fl, pairs = oracle_sample(w, q, k, v, [0], max(1, w.nT // 4))
+    per_head = sec * 4
+    nh = int(max(1, min(w.heads, budget_s // max(per_head, 1e-3))))
+    sec, fl, pairs = oracle_sample(w, q, k, v, list(range(nh)))
+    tflops = fl / sec / 1e12
+    scale_up = (w.B * w.heads) / (w.B * nh)
+    return {"value": tflops, "unit": "TFLOPS", "cores": _cores(), "kind": "oracle",
+            "ms_per_call_est": sec * scale_up * 1e3,
+            "sample": (f"fp64 numpy oracle, whole path (tile, pool, score, select, attend all "
+                       f"{w.nT} query tiles) for heads 0..{nh - 1} of {w.heads} x batch {w.B}: "
+                       f"{pairs:,} kept pairs in {sec:.1f} s; ms_per_call_est scales by "
+                       f"{scale_up:.1f}")}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from block_sparse_video_tile3d_b200 import workloads
+    q, k, v = workloads.make_qkv(w)
+    n = max(1, w.nT // 8)  # bounded sample per step: one head, an eighth of its query tiles
+
+    def step(h):
+        return oracle_sample(w, q, k, v, [h % w.heads], n)
+
+    for s in range(args.warmup):
+        step(s)
+    tot_s = tot_f = 0.0
+    tot_pairs = 0
+    for s in range(args.steps):
+        sec, fl, pairs = step(s)
+        tot_s += sec
+        tot_f += fl
+        tot_pairs += pairs
+    tflops = tot_f / tot_s / 1e12
+    sample = (f"fp64 numpy oracle, per step: one head's tiling, pooling, scores and selection plus "
+              f"attention for {n} of its {w.nT} query tiles ({tot_pairs // max(args.steps, 1):,} "
+              f"kept pairs)")
+    line = {"metric": METRIC, "value": tflops, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_s / max(args.steps, 1) * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": _describe(w), "l2": "n/a (host CPU)"},
+            "cpu_baseline": {"value": tflops, "unit": "TFLOPS", "cores": _cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": tflops, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------------- our arm
+
+def _stage_bytes(w, name, pairs, kmax):
+    """Algorithmic HBM bytes of one stage launch (each input read once, each output written once)."""
+    B, heads, D, L, Lp, nT = w.B, w.heads, w.D, w.L, 64 * w.nT, w.nT
+    row = heads * D * 2
+    if name.startswith("scatter"):
+        return B * L * row + B * Lp * row
+    if name == "gather":
+        return 2 * B * L * row
+    if name.startswith("pool"):
+        return B * L * row + B * heads * nT * D * 4
+    if name == "prune_q":
+        return B * L * row + B * heads * nT * (D * 4 + 128)
+    if name.startswith("select"):
+        return 2 * B * heads * nT * D * 4 + B * heads * nT * (kmax + 1) * 4
+    if name == "mask_to_index":
+        return B * heads * nT * nT + B * heads * nT * (kmax + 1) * 4
+    if name == "attention":
+        return 4 * B * Lp * row + B * heads * nT * (kmax + 1) * 4
+    return 0
+
+
+def _source_sha() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_video_tile3d_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        if n.startswith("attn") or n in ("common.cuh", "kernels.h"):
+            with open(os.path.join(csrc, n), "rb") as f:
+                h.update(n.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(workload: str):
+    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, if it was
+    taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d.get(workload)
+        if e and e.get("source_sha") == _source_sha():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+def run_ours(args, w):
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_video_tile3d_b200 import TileSparseAttention, workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    q, k, v = workloads.make_qkv(w)
+    mask = workloads.block_mask(w) if w.mode == "mask" else None
+    if w.mode == "bsa":
+        pass  # the benchmark runs the workload's own data; query pruning drops what it finds
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    od = torch.empty_like(qd)
+    model = TileSparseAttention(w.B, w.T, w.H, w.W, w.heads, w.D, mode=w.mode, topk=w.k or None,
+                                mass=w.mass, min_k=w.min_kv, cos_thresh=w.cos_thresh, mask=mask,
+                                device=dev)
+    stages = model.stages(qd, kd, vd, od)
+    names = [n for n, _ in stages]
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    for _ in range(max(args.warmup, 3)):
+        for _, launch in stages:
+            launch()
+    torch.cuda.synchronize()
+    pairs = int(model.kv_cnt.sum().item())
+    flops = pairs * FLOPS_PER_PAIR(w.D)
+
+    # ---- device-resident timed region, events between stages on the launching stream
+    nst = len(stages)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for s in range(args.steps):
+        ev[s][0].record()
+        for j, (_, launch) in enumerate(stages):
+            launch()
+            ev[s][j + 1].record()
+    torch.cuda.synchronize()
+    barrier()
+    total_ms = ev[0][0].elapsed_time(ev[-1][-1])
+    stage_ms = {n: sum(ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(args.steps)) / args.steps
+                for j, n in enumerate(names)}
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(total_ms)
+    ms_step = total_ms / args.steps
+    status = model.device_status()
+
+    # ---- end to end through the public API with pinned host buffers
+    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True)  # noqa: E702
+        vd.copy_(vh, non_blocking=True); model.forward(qd, kd, vd, od)  # noqa: E702
+        oh.copy_(od, non_blocking=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        model.forward(qd, kd, vd, od)
+        oh.copy_(od, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+
+    peaks = _peaks()
+    attn_ms = stage_ms["attention"]
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    kmax = model.kmax
+    stage_report = {}
+    for n in names:
+        byt = _stage_bytes(w, n, pairs, kmax)
+        stage_report[n] = {"ms": round(stage_ms[n], 4),
+                           "gbs": round(byt / (stage_ms[n] * 1e-3) / 1e9, 1) if byt else None,
+                           "bytes": byt}
+    coarse_ms = sum(stage_ms[n] for n in names if n != "attention")
+    coarse_bytes = sum(_stage_bytes(w, n, pairs, kmax) for n in names if n != "attention")
+    line = {
+        "metric": METRIC,
+        "value": world * flops / (ms_step * 1e-3) / 1e12,
+        "unit": "TFLOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "ms_per_call": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": _describe(w), "kept_pairs": pairs,
+                   "kept_block_gflop": flops / 1e9,
+                   "density": pairs / (w.B * w.heads * w.nT * w.nT),
+                   "l2": "no flush: raster Q/K/V inputs of "
+                         f"{3 * w.B * w.L * w.heads * w.D * 2 / 1e6:.0f} MB exceed the 126 MB L2",
+                   "parallelism": f"{world} independent replica(s), one per GPU"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": _ncu_traffic(w.name), "kernel": "block_sparse_attn_fwd",
+                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                     "ms_per_launch": attn_ms},
+        "coarse_and_tiling": {"ms": coarse_ms, "bytes": coarse_bytes,
+                              "gbs": coarse_bytes / (coarse_ms * 1e-3) / 1e9,
+                              "frac_hbm": coarse_bytes / (coarse_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "hbm_peak_gbs": peaks["hbm_gbs"]},
+        "stages": stage_report,
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                "d2h_bytes_per_step": od.numel() * od.element_size()},
+        "gpu_launches": args.steps * nst,
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, q, k, v, budget_s=args.cpu_budget)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="small",
+                    help="workload: tiny, small, large, bsa, ragged_sliding, ragged_random")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=20.0,
+                    help="seconds of oracle work for the cpu_baseline sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from block_sparse_video_tile3d_b200.workloads import WORKLOADS
+    w = WORKLOADS[args.config]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

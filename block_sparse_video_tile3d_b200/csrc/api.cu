@@ -1,0 +1,228 @@
+// C ABI of libtile3d: argument validation, then one asynchronous launch per call.
+// Declarations and the contract of each call are in include/tile3d.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+t3d_status fail(t3d_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+t3d_status ok() {
+  g_err[0] = '\0';
+  return T3D_OK;
+}
+
+t3d_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(T3D_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+t3d_status check_geom(const t3d_geom* g, t3d::Geo* out) {
+  if (g == nullptr) return fail(T3D_ERR_INVALID, "geometry pointer is NULL");
+  if (g->B < 1 || g->T < 1 || g->H < 1 || g->W < 1 || g->heads < 1)
+    return fail(T3D_ERR_INVALID, "B, T, H, W and heads must be >= 1 (got %d, %d, %d, %d, %d)", g->B,
+                g->T, g->H, g->W, g->heads);
+  if (g->D != 64 && g->D != 128)
+    return fail(T3D_ERR_UNSUPPORTED, "head dimension D=%d is not supported (64 or 128)", g->D);
+  const t3d::Geo geo = t3d::make_geo(*g);
+  if (geo.nT > t3d::kMaxTiles)
+    return fail(T3D_ERR_UNSUPPORTED, "%d tiles exceed the supported maximum %d", geo.nT,
+                t3d::kMaxTiles);
+  if ((long long)g->B * geo.Lp * g->heads > (1LL << 31))
+    return fail(T3D_ERR_UNSUPPORTED, "B * Lp * heads = %lld token-head rows exceeds 2^31",
+                (long long)g->B * geo.Lp * g->heads);
+  *out = geo;
+  return T3D_OK;
+}
+
+#define T3D_CHECK(expr)            \
+  do {                             \
+    t3d_status _st = (expr);       \
+    if (_st != T3D_OK) return _st; \
+  } while (0)
+
+t3d_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(T3D_ERR_INVALID, "%s is NULL", name);
+  if (!aligned16(p)) return fail(T3D_ERR_INVALID, "%s is not 16-byte aligned", name);
+  return T3D_OK;
+}
+
+t3d_status check_ptr4(const void* p, const char* name) {
+  if (p == nullptr) return fail(T3D_ERR_INVALID, "%s is NULL", name);
+  if ((reinterpret_cast<uintptr_t>(p) & 3u) != 0)
+    return fail(T3D_ERR_INVALID, "%s is not 4-byte aligned", name);
+  return T3D_OK;
+}
+
+cudaStream_t as_stream(t3d_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace
+
+extern "C" {
+
+const char* t3d_last_error_string(void) { return g_err; }
+
+const char* t3d_version(void) { return "0.1.0"; }
+
+t3d_status tile3d_geometry(const t3d_geom* g, int* nT, int* Lp, int32_t* vc_host) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  if (nT) *nT = geo.nT;
+  if (Lp) *Lp = geo.Lp;
+  if (vc_host)
+    for (int i = 0; i < geo.nT; ++i) vc_host[i] = t3d::tile_valid_count(geo, i);
+  return ok();
+}
+
+t3d_status tile3d_scatter(const t3d_geom* g, const void* x, void* y, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(x, "x"));
+  T3D_CHECK(check_ptr(y, "y"));
+  return cuda_status(t3d::launch_scatter(geo, x, y, as_stream(stream)), "tile3d_scatter");
+}
+
+t3d_status tile3d_gather(const t3d_geom* g, const void* y, void* x, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(y, "y"));
+  T3D_CHECK(check_ptr(x, "x"));
+  return cuda_status(t3d::launch_gather(geo, y, x, as_stream(stream)), "tile3d_gather");
+}
+
+t3d_status tile_pool(const t3d_geom* g, const void* y, float* pooled, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(y, "y"));
+  T3D_CHECK(check_ptr(pooled, "pooled"));
+  return cuda_status(t3d::launch_pool(geo, y, pooled, as_stream(stream)), "tile_pool");
+}
+
+t3d_status tile_select_topk(const t3d_geom* g, const float* pq, const float* pk, int k,
+                            int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
+                            t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(pq, "pq"));
+  T3D_CHECK(check_ptr(pk, "pk"));
+  T3D_CHECK(check_ptr4(kv_idx, "kv_idx"));
+  T3D_CHECK(check_ptr4(kv_cnt, "kv_cnt"));
+  if (k < 1) return fail(T3D_ERR_INVALID, "k=%d must be >= 1", k);
+  return cuda_status(
+      t3d::launch_select_topk(geo, pq, pk, k, kv_idx, kv_cnt, dev_status, as_stream(stream)),
+      "tile_select_topk");
+}
+
+t3d_status tile_select_mass(const t3d_geom* g, const float* pq, const float* pk, float scale,
+                            float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
+                            int32_t* dev_status, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(pq, "pq"));
+  T3D_CHECK(check_ptr(pk, "pk"));
+  T3D_CHECK(check_ptr4(kv_idx, "kv_idx"));
+  T3D_CHECK(check_ptr4(kv_cnt, "kv_cnt"));
+  if (!(scale > 0.f) || !isfinite(scale))
+    return fail(T3D_ERR_INVALID, "scale=%g must be finite and > 0", (double)scale);
+  if (!(mass > 0.f) || mass > 1.f)
+    return fail(T3D_ERR_INVALID, "mass=%g must lie in (0, 1]", (double)mass);
+  if (min_k < 1) return fail(T3D_ERR_INVALID, "min_k=%d must be >= 1", min_k);
+  if (kmax < 1 || kmax > geo.nT)
+    return fail(T3D_ERR_INVALID, "kmax=%d must lie in [1, nT=%d]", kmax, geo.nT);
+  return cuda_status(t3d::launch_select_mass(geo, pq, pk, scale, mass, min_k, kmax, kv_idx, kv_cnt,
+                                             dev_status, as_stream(stream)),
+                     "tile_select_mass");
+}
+
+t3d_status tile_prune_queries(const t3d_geom* g, const void* q, float cos_thresh, uint8_t* keep,
+                              uint8_t* src_row, float* pq_kept, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(q, "q"));
+  T3D_CHECK(check_ptr(keep, "keep"));
+  T3D_CHECK(check_ptr(src_row, "src_row"));
+  T3D_CHECK(check_ptr(pq_kept, "pq_kept"));
+  if (geo.L != geo.Lp)
+    return fail(T3D_ERR_INVALID,
+                "query pruning needs every tile full (L=%d must equal 64 * nT = %d)", geo.L, geo.Lp);
+  if (isnan(cos_thresh)) return fail(T3D_ERR_INVALID, "cos_thresh is NaN");
+  return cuda_status(
+      t3d::launch_prune(geo, q, cos_thresh, keep, src_row, pq_kept, as_stream(stream)),
+      "tile_prune_queries");
+}
+
+t3d_status block_mask_to_index(const t3d_geom* g, const uint8_t* mask, int kmax, int32_t* kv_idx,
+                               int32_t* kv_cnt, int32_t* dev_status, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  if (mask == nullptr) return fail(T3D_ERR_INVALID, "mask is NULL");
+  T3D_CHECK(check_ptr4(kv_idx, "kv_idx"));
+  T3D_CHECK(check_ptr4(kv_cnt, "kv_cnt"));
+  if (kmax < 1 || kmax > geo.nT)
+    return fail(T3D_ERR_INVALID, "kmax=%d must lie in [1, nT=%d]", kmax, geo.nT);
+  return cuda_status(
+      t3d::launch_mask_to_index(geo, mask, kmax, kv_idx, kv_cnt, dev_status, as_stream(stream)),
+      "block_mask_to_index");
+}
+
+size_t block_sparse_attn_workspace_size(const t3d_geom* g, int kmax) {
+  t3d::Geo geo;
+  if (check_geom(g, &geo) != T3D_OK) return 0;
+  return t3d::attn_workspace_bytes(geo, kmax);
+}
+
+t3d_status block_sparse_attn_fwd(const t3d_geom* g, const void* q, const void* k, const void* v,
+                                 void* o, const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                 const uint8_t* keep, const uint8_t* src_row, float softmax_scale,
+                                 int causal, int num_kv_heads, void* workspace, size_t ws_bytes,
+                                 int32_t* dev_status, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  if (causal != 0)
+    return fail(T3D_ERR_UNSUPPORTED, "the attention is bidirectional; causal=1 is unsupported");
+  if (num_kv_heads != g->heads)
+    return fail(T3D_ERR_UNSUPPORTED,
+                "grouped-query attention is unsupported (num_kv_heads=%d, heads=%d)", num_kv_heads,
+                g->heads);
+  const double expected = 1.0 / sqrt((double)g->D);
+  const double diff = fabs((double)softmax_scale - expected);
+  if (!(diff <= fmax(1e-4 * fmax(fabs((double)softmax_scale), expected), 1e-5)))
+    return fail(T3D_ERR_INVALID, "softmax_scale=%.8g must be 1/sqrt(D)=%.8g", (double)softmax_scale,
+                expected);
+  T3D_CHECK(check_ptr(q, "q"));
+  T3D_CHECK(check_ptr(k, "k"));
+  T3D_CHECK(check_ptr(v, "v"));
+  T3D_CHECK(check_ptr(o, "o"));
+  T3D_CHECK(check_ptr4(kv_idx, "kv_idx"));
+  T3D_CHECK(check_ptr4(kv_cnt, "kv_cnt"));
+  if (kmax < 1 || kmax > geo.nT)
+    return fail(T3D_ERR_INVALID, "kmax=%d must lie in [1, nT=%d]", kmax, geo.nT);
+  if ((keep == nullptr) != (src_row == nullptr))
+    return fail(T3D_ERR_INVALID, "keep and src_row must both be given or both be NULL");
+  if (keep != nullptr && geo.L != geo.Lp)
+    return fail(T3D_ERR_INVALID, "pruned-query attention needs every tile full (L=%d, Lp=%d)",
+                geo.L, geo.Lp);
+  const size_t need = t3d::attn_workspace_bytes(geo, kmax);
+  if (ws_bytes < need)
+    return fail(T3D_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
+                ws_bytes, need);
+  if (need > 0) T3D_CHECK(check_ptr(workspace, "workspace"));
+  t3d::AttnArgs a{q, k, v, o, kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale,
+                  workspace, ws_bytes, dev_status};
+  return cuda_status(t3d::launch_attn(geo, a, as_stream(stream)), "block_sparse_attn_fwd");
+}
+
+}  // extern "C"

@@ -1,0 +1,47 @@
+// Internal launchers of libtile3d (host side). Arguments are validated by the C ABI layer in
+// api.cu before any of these is called; each returns the CUDA launch error.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace t3d {
+
+cudaError_t launch_scatter(const Geo& g, const void* x, void* y, cudaStream_t s);
+cudaError_t launch_gather(const Geo& g, const void* y, void* x, cudaStream_t s);
+cudaError_t launch_pool(const Geo& g, const void* y, float* pooled, cudaStream_t s);
+
+cudaError_t launch_select_topk(const Geo& g, const float* pq, const float* pk, int k,
+                               int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
+                               cudaStream_t s);
+cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, float scale,
+                               float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
+                               int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_mask_to_index(const Geo& g, const uint8_t* mask, int kmax, int32_t* kv_idx,
+                                 int32_t* kv_cnt, int32_t* dev_status, cudaStream_t s);
+cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, uint8_t* keep,
+                         uint8_t* src_row, float* pq_kept, cudaStream_t s);
+
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  const int32_t* kv_idx;
+  const int32_t* kv_cnt;
+  int kmax;
+  const uint8_t* keep;
+  const uint8_t* src_row;
+  float scale;
+  void* workspace;
+  size_t ws_bytes;
+  int32_t* dev_status;
+};
+
+size_t attn_workspace_bytes(const Geo& g, int kmax);
+cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s);
+
+}  // namespace t3d

@@ -11,6 +11,10 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long-running CPU test")
+    # The C ABI library is built in-tree; build it once if this checkout has not yet.
+    from block_sparse_video_tile3d_b200 import build as _build
+    if not os.path.exists(_build.LIB):
+        _build.build()
 
 
 @pytest.fixture(scope="session")

@@ -1,0 +1,173 @@
+"""GPU parity: KV tile selection (top-k, cumulative mass), block map -> index lists, BSA pruning."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_video_tile3d_b200 import (block_mask_to_index, tile3d_scatter, tile_pool,
+                                            tile_prune_queries, tile_select_mass, tile_select_topk,
+                                            workloads)
+from block_sparse_video_tile3d_b200._lib import T3D_DEV_OVERFLOW
+from oracle import bsa, pool, select, tiling
+from tests.helpers import check_topk_sets, f64, gpu_sets
+
+pytestmark = pytest.mark.gpu
+
+
+def _pooled(B, heads, nT, D, seed, ties=False):
+    g = torch.Generator().manual_seed(seed)
+    pq = torch.randn((B, heads, nT, D), generator=g)
+    pk = torch.randn((B, heads, nT, D), generator=g) + 0.3 * torch.randn((B, heads, 1, D), generator=g)
+    if ties:  # duplicate some key tiles exactly: equal scores in any precision
+        pk[:, :, 1::3] = pk[:, :, 0:-1:3][:, :, :pk[:, :, 1::3].shape[2]]
+    return pq.contiguous(), pk.contiguous()
+
+
+@pytest.mark.parametrize("grid,D,k,ties", [
+    ((9, 10, 13), 64, 1, False), ((9, 10, 13), 128, 5, False), ((9, 10, 13), 64, 36, False),
+    ((9, 10, 13), 64, 50, False), ((9, 10, 13), 128, 7, True), ((4, 8, 8), 64, 2, False),
+    ((1, 1, 1), 64, 3, False), ((40, 40, 40), 128, 100, False),
+])
+def test_topk_matches_oracle(grid, D, k, ties):
+    T, H, W = grid
+    nT = len(tiling.variable_block_sizes(T, H, W))
+    B, heads = 2, 3
+    pq, pk = _pooled(B, heads, nT, D, seed=nT + k, ties=ties)
+    kv_idx, kv_cnt = tile_select_topk(pq.cuda(), pk.cuda(), T, H, W, k)
+    S = select.tile_scores(f64(pq), f64(pk))
+    want = select.select_topk(S, k)
+    got = gpu_sets(kv_idx, kv_cnt)
+    stats = check_topk_sets(got, want, S, min(k, nT))
+    if ties:  # exact ties must resolve to the lower index, exactly like the oracle
+        for b in range(B):
+            for h in range(heads):
+                for i in range(nT):
+                    np.testing.assert_array_equal(got[b][h][i], want[b][h][i])
+    assert stats["exact"] >= 0.9 * B * heads * nT
+
+
+def _check_mass(got, S, scale, tau, min_k):
+    B, heads, nT = S.shape[:3]
+    n_exact = 0
+    for b in range(B):
+        for h in range(heads):
+            for i in range(nT):
+                row = S[b, h, i]
+                want = select.select_mass_row(row, scale, tau, min_k)
+                mm = select.mass_margins(row, scale, tau, min_k)
+                g = got[b][h][i]
+                assert np.all(np.diff(g) > 0)
+                if mm["cut_gap"] > 1e-3 and mm["sum_margin"] > 1e-4:
+                    np.testing.assert_array_equal(g, want, err_msg=f"row {(b, h, i)}")
+                    n_exact += 1
+                else:  # near a decision boundary: a valid prefix of the ranking, mass ~ tau
+                    p = select.softmax_row(scale * row)
+                    dropped = np.setdiff1d(np.arange(nT), g)
+                    if dropped.size:
+                        assert p[dropped].max() <= p[g].min() * (1 + 1e-3) + 1e-7
+                    assert abs(len(g) - len(want)) <= 2
+                    if len(g) > max(min_k, 1):
+                        assert p[g].sum() - p[g].min() < tau + 1e-4
+                    assert p[g].sum() >= min(tau, 1.0) - 1e-4 or len(g) >= min(min_k, nT)
+    return n_exact
+
+
+@pytest.mark.parametrize("grid,D,scale,tau,min_k", [
+    ((9, 10, 13), 64, 0.125, 0.9, 1), ((9, 10, 13), 128, 1.0, 0.5, 1),
+    ((9, 10, 13), 128, 0.088388, 0.9, 4), ((4, 8, 8), 64, 0.5, 0.3, 1),
+    ((9, 10, 13), 64, 3.0, 0.99, 2), ((9, 10, 13), 64, 0.2, 1.0, 1),
+])
+def test_mass_matches_oracle(grid, D, scale, tau, min_k):
+    T, H, W = grid
+    nT = len(tiling.variable_block_sizes(T, H, W))
+    B, heads = 2, 3
+    pq, pk = _pooled(B, heads, nT, D, seed=int(scale * 100) + min_k)
+    kv_idx, kv_cnt = tile_select_mass(pq.cuda(), pk.cuda(), T, H, W, scale, tau, min_k)
+    S = select.tile_scores(f64(pq), f64(pk))
+    n = _check_mass(gpu_sets(kv_idx, kv_cnt), S, scale, tau, min_k)
+    assert n >= 0.8 * B * heads * nT
+
+
+def test_mass_overflow_truncates_to_most_probable():
+    T, H, W, D = 9, 10, 13, 64
+    nT = 36
+    pq, pk = _pooled(1, 2, nT, D, seed=11)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kv_idx, kv_cnt = tile_select_mass(pq.cuda(), pk.cuda(), T, H, W, 0.01, 0.99, 1, kmax=5,
+                                      dev_status=status)
+    assert int(status.item()) & T3D_DEV_OVERFLOW
+    S = select.tile_scores(f64(pq), f64(pk))
+    got = gpu_sets(kv_idx, kv_cnt)
+    for h in range(2):
+        for i in range(nT):
+            if select.topk_gap(S[0, h, i][None], 5)[0] > 1e-3:
+                np.testing.assert_array_equal(got[0][h][i], select.select_topk_row(S[0, h, i], 5))
+
+
+@pytest.mark.parametrize("kmax", [None, 4])
+def test_mask_to_index_bit_exact(kmax):
+    T, H, W, D = 21, 30, 52, 128
+    nT = 624
+    g = torch.Generator().manual_seed(5)
+    mask = (torch.rand((2, 3, nT, nT), generator=g) < 0.05).to(torch.uint8)
+    mask[:, :, 7] = 0  # an empty row
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kv_idx, kv_cnt = block_mask_to_index(mask.cuda(), T, H, W, D, kmax, dev_status=status)
+    want = select.map_to_sets(mask.numpy())
+    got = gpu_sets(kv_idx, kv_cnt)
+    cap = nT if kmax is None else kmax
+    for b in range(2):
+        for h in range(3):
+            for i in range(nT):
+                np.testing.assert_array_equal(got[b][h][i], want[b][h][i][:cap])
+    overflow = any(len(want[b][h][i]) > cap for b in range(2) for h in range(3) for i in range(nT))
+    assert bool(int(status.item()) & T3D_DEV_OVERFLOW) == overflow
+
+
+def test_workload_selection_small_full():
+    """Independent pipelines: GPU scatter -> pool -> top-k versus the oracle's, on the small
+    video-DiT workload (12 heads, 448 tiles, k = 56)."""
+    w = workloads.WORKLOADS["small"]
+    q, k, _ = workloads.make_qkv(w)
+    qt = tile3d_scatter(q.cuda(), w.T, w.H, w.W)
+    kt = tile3d_scatter(k.cuda(), w.T, w.H, w.W)
+    pq = tile_pool(qt, w.T, w.H, w.W)
+    pk = tile_pool(kt, w.T, w.H, w.W)
+    kv_idx, kv_cnt = tile_select_topk(pq, pk, w.T, w.H, w.W, w.k)
+    vc = tiling.variable_block_sizes(w.T, w.H, w.W)
+    opq = pool.tile_mean_pool(tiling.tile_scatter(f64(q), w.T, w.H, w.W), vc)
+    opk = pool.tile_mean_pool(tiling.tile_scatter(f64(k), w.T, w.H, w.W), vc)
+    S = select.tile_scores(opq, opk)
+    stats = check_topk_sets(gpu_sets(kv_idx, kv_cnt), select.select_topk(S, w.k), S, w.k)
+    assert stats["exact"] >= 0.95 * w.heads * w.nT
+
+
+def test_prune_matches_oracle_structured():
+    w = workloads.WORKLOADS["bsa"].with_(T=8, H=8, W=12, heads=3)
+    q, _, _ = workloads.make_qkv(w)
+    q = workloads.make_structured_queries(w, q)
+    qt = tile3d_scatter(q.cuda(), w.T, w.H, w.W)
+    keep, src, pqk = tile_prune_queries(qt, w.T, w.H, w.W, w.cos_thresh)
+    oqt = tiling.tile_scatter(f64(q), w.T, w.H, w.W)
+    okeep, osrc, ocos = bsa.prune_queries(oqt, w.cos_thresh)
+    keep, src = keep.cpu().numpy().astype(bool), src.cpu().numpy()
+    assert (~okeep).sum() > 100  # the structured variant does prune
+    decided = np.abs(ocos - w.cos_thresh) > 1e-4
+    np.testing.assert_array_equal(keep[decided], okeep[decided])
+    nT = w.nT
+    for h in range(w.heads):
+        for i in range(nT):
+            if not np.array_equal(keep[0, h, i], okeep[0, h, i]):
+                continue
+            rows = oqt[0, 64 * i:64 * i + 64, h]
+            kept = np.nonzero(okeep[0, h, i])[0]
+            nrm = np.linalg.norm(rows, axis=1)
+            for r in np.nonzero(~okeep[0, h, i])[0]:
+                c = rows[kept] @ rows[r] / (nrm[kept] * nrm[r])
+                top = np.sort(c)[::-1]
+                if len(top) < 2 or top[0] - top[1] > 1e-4:
+                    assert src[0, h, i, r] == osrc[0, h, i, r]
+                else:
+                    assert keep[0, h, i, src[0, h, i, r]]
+            np.testing.assert_array_equal(src[0, h, i][okeep[0, h, i]], kept)
+            np.testing.assert_allclose(f64(pqk)[0, h, i], rows[kept].mean(axis=0), rtol=1e-5,
+                                       atol=2e-6)
