@@ -304,9 +304,14 @@ size_t attn_workspace_bytes(const Geo& g, int kmax) {
   return 0;
 }
 
-cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s) {
+cudaError_t launch_attn_mma(const Geo& g, const AttnArgs& a, cudaStream_t s) {
   if (g.D == 128) return launch_attn_d<128>(g, a, s);
   return launch_attn_d<64>(g, a, s);
+}
+
+cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s) {
+  if (g.D == 128) return launch_attn_sm100(g, a, s);
+  return launch_attn_mma(g, a, s);
 }
 
 }  // namespace t3d

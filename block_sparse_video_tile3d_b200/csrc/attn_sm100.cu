@@ -1,0 +1,543 @@
+// Fine stage on the sm_100a tensor cores: block-sparse softmax attention over the kept
+// (query tile, key tile) pairs with tcgen05 MMAs accumulating in tensor memory (TMEM) and the kept
+// key/value tiles fetched by TMA.
+//
+// FastVideo API docs, bsa_attn page, BSAAttentionImpl.__init__ / forward: bidirectional attention,
+// one KV head per query head, softmax scale 1/sqrt(D), tile-ordered [B, L, heads, D] bf16 tensors,
+// sparse attention per kept block pair, pruned query rows reconstructed afterwards.
+//
+// Shape of the computation. A query tile has 64 rows, and a tcgen05 MMA with M = 64 costs as much
+// as one with M = 128, so the kernel puts KEYS on the M dimension: each step takes a PAIR of kept key
+// tiles (128 keys) and computes
+//     S^T[128 keys, 64 queries]  = K_pair . Q^T          (A = K pair, K-major; B = Q, K-major)
+//     O^T[D, 64 queries]        += V_pair^T . P^T        (A = V pair, MN-major; B = P^T, MN-major)
+// both with M = 128, N = 64, accumulating in fp32 in TMEM. An odd last tile is paired with a copy of
+// itself whose keys are all masked.
+//
+// Roles (one persistent CTA per SM, work units = (batch, head, query tile), static round robin):
+//   warp 0      TMA producer for Q (once per unit) and the K pairs (3-stage ring)
+//   warp 1      TMEM allocation; one thread issues every tcgen05.mma and tcgen05.commit
+//   warps 2..5  softmax and epilogue; thread t owns TMEM lane t (a key of S^T, a column d of O^T)
+//   warp 6      TMA producer for the V pairs (2-stage ring)
+//
+// Softmax. Each softmax thread holds one key's 64 logits. The shift subtracted before exp2 is a
+// per-query value m[q] shared through shared memory; it is only raised (a "slow step": per-query
+// maxima by warp reductions, then a rescale of O^T and of the running sums) when some logit exceeds
+// m[q] by more than kShiftSlack (log2 units). Any shift gives the same softmax; the bound keeps P
+// within [0, 2^kShiftSlack] so nothing overflows. The first step of a unit is always slow. Each
+// thread keeps running sums of P for its own key over all steps; they are reduced across the 128
+// threads once per unit.
+//
+// Every mbarrier wait is bounded; on a timeout the CTA records T3D_DEV_TIMEOUT, stops issuing work,
+// waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
+#include "kernels.h"
+#include "sm100.cuh"
+
+namespace t3d {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 128;             // head dimension handled by this kernel
+constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a row
+constexpr int kKStages = 3;         // K-pair ring depth
+constexpr int kVStages = 2;         // V-pair ring depth
+constexpr int kThreads = 224;       // 7 warps
+constexpr int kSoftmaxThreads = 128;
+constexpr int kSoftmaxBar = 1;      // named barrier id of the softmax warps
+constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColS = 0;       // S^T buffers: columns [0, 64) and [64, 128)
+constexpr uint32_t kColO = 128;     // O^T: columns [128, 192)
+
+constexpr uint32_t kTileBytes = 64 * 128;                  // 64 rows x 128 B (one half of a tile)
+constexpr uint32_t kQBytes = kHalves * kTileBytes;         // 16 KB
+constexpr uint32_t kPairBytes = kHalves * 2 * kTileBytes;  // 32 KB: two tiles, both halves
+constexpr uint32_t kPBytes = 128 * 128;                    // P^T: 128 keys x 64 queries bf16
+
+struct alignas(1024) SmemLayout {
+  uint8_t q[kQBytes];
+  uint8_t k[kKStages][kPairBytes];
+  uint8_t v[kVStages][kPairBytes];
+  uint8_t p[2][kPBytes];
+  uint64_t q_full, q_empty, o_full, o_empty;
+  uint64_t k_full[kKStages], k_empty[kKStages];
+  uint64_t v_full[kVStages], v_empty[kVStages];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t drain;
+  float shift[64];    // current per-query shift (log2 units)
+  float red[4][64];   // per-warp partial results
+  float alpha[64];    // rescale factors of a slow step
+  float lsum[64];     // per-query softmax denominators
+  uint32_t tmem_base;
+  int abort;
+};
+
+constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
+constexpr uint32_t idesc_o = idesc_bf16(128, 64, true, true);
+
+struct UnitInfo {
+  int b, h, i, cnt, npairs;
+  const int32_t* list;
+};
+
+__device__ __forceinline__ UnitInfo unit_info(const Geo& g, const AttnArgs& a, int u) {
+  UnitInfo r;
+  r.i = u % g.nT;
+  const int bh = u / g.nT;
+  r.h = bh % g.heads;
+  r.b = bh / g.heads;
+  int c = a.kv_cnt[(long)bh * g.nT + r.i];
+  c = c < 0 ? 0 : (c > a.kmax ? a.kmax : c);
+  r.cnt = c;
+  r.npairs = (c + 1) >> 1;
+  r.list = a.kv_idx + ((long)bh * g.nT + r.i) * a.kmax;
+  return r;
+}
+
+// Key tile of entry e of the list, or -1 if absent / out of range.
+__device__ __forceinline__ int list_tile(const Geo& g, const UnitInfo& u, int e) {
+  if (e >= u.cnt) return -1;
+  const int j = u.list[e];
+  return (j >= 0 && j < g.nT) ? j : -1;
+}
+
+__device__ __forceinline__ void fail(SmemLayout& s, int32_t* status) {
+  s.abort = 1;
+  report(status, T3D_DEV_TIMEOUT);
+}
+
+struct Maps {
+  CUtensorMap q, k, v;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_sm100_kernel(const __grid_constant__ Maps maps, Geo g, AttnArgs a, float sl2) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemLayout& s = *reinterpret_cast<SmemLayout*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int total_units = g.B * g.heads * g.nT;
+  volatile int* abort_flag = &s.abort;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&s.q_full, 1);
+    mbar_init(&s.q_empty, 1);
+    mbar_init(&s.o_full, 1);
+    mbar_init(&s.o_empty, kSoftmaxThreads);
+    for (int t = 0; t < kKStages; ++t) { mbar_init(&s.k_full[t], 1); mbar_init(&s.k_empty[t], 1); }
+    for (int t = 0; t < kVStages; ++t) { mbar_init(&s.v_full[t], 1); mbar_init(&s.v_empty[t], 1); }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.s_empty[t], kSoftmaxThreads);
+      mbar_init(&s.p_full[t], kSoftmaxThreads);
+      mbar_init(&s.p_empty[t], 1);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch(&maps.q);
+    tma_prefetch(&maps.k);
+    tma_prefetch(&maps.v);
+  }
+  if (warp == 1) {
+    tmem_alloc(&s.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- Q and K producer
+    if (lane == 0) {
+      int active = 0;
+      long gp0 = 0;
+      long issued = 0;  // K pairs issued
+      for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
+        const UnitInfo ui = unit_info(g, a, u);
+        if (ui.npairs == 0) continue;
+        if (!mbar_wait(&s.q_empty, (active & 1) ^ 1, abort_flag)) { fail(s, a.dev_status); break; }
+        const int row0 = ui.b * g.Lp + ui.i * kTileElems;
+        mbar_expect_tx(&s.q_full, kQBytes);
+        for (int hh = 0; hh < kHalves; ++hh)
+          tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
+        bool ok = true;
+        for (int n = 0; n < ui.npairs; ++n) {
+          const long gp = gp0 + n;
+          const int ks = (int)(gp % kKStages);
+          if (!mbar_wait(&s.k_empty[ks], ((gp / kKStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
+          if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
+          if (jb < 0) jb = ja;
+          mbar_expect_tx(&s.k_full[ks], kPairBytes);
+          for (int hh = 0; hh < kHalves; ++hh) {
+            uint8_t* dst = s.k[ks] + hh * 2 * kTileBytes;
+            tma_load_3d(dst, &maps.k, &s.k_full[ks], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
+            tma_load_3d(dst + kTileBytes, &maps.k, &s.k_full[ks], 64 * hh, ui.h,
+                        ui.b * g.Lp + jb * kTileElems);
+          }
+          ++issued;
+        }
+        if (!ok) { fail(s, a.dev_status); break; }
+        gp0 += ui.npairs;
+        ++active;
+      }
+      // Drain: the last loads issued must land before the CTA can exit.
+      for (long gp = issued - kKStages; gp < issued; ++gp)
+        if (gp >= 0) mbar_wait(&s.k_full[gp % kKStages], (gp / kKStages) & 1, nullptr);
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------- V producer
+    if (lane == 0) {
+      long gp0 = 0, issued = 0;
+      for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
+        const UnitInfo ui = unit_info(g, a, u);
+        if (ui.npairs == 0) continue;
+        bool ok = true;
+        for (int n = 0; n < ui.npairs; ++n) {
+          const long gp = gp0 + n;
+          const int vs = (int)(gp & 1);
+          if (!mbar_wait(&s.v_empty[vs], ((gp >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
+          if (ja < 0) ja = 0;
+          if (jb < 0) jb = ja;
+          mbar_expect_tx(&s.v_full[vs], kPairBytes);
+          for (int hh = 0; hh < kHalves; ++hh) {
+            uint8_t* dst = s.v[vs] + hh * 2 * kTileBytes;
+            tma_load_3d(dst, &maps.v, &s.v_full[vs], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
+            tma_load_3d(dst + kTileBytes, &maps.v, &s.v_full[vs], 64 * hh, ui.h,
+                        ui.b * g.Lp + jb * kTileElems);
+          }
+          ++issued;
+        }
+        if (!ok) { fail(s, a.dev_status); break; }
+        gp0 += ui.npairs;
+      }
+      for (long gp = issued - kVStages; gp < issued; ++gp)
+        if (gp >= 0) mbar_wait(&s.v_full[gp & 1], (gp >> 1) & 1, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      int active = 0;
+      long gp0 = 0;
+      bool ok = true;
+      const uint32_t q_addr = smem_u32(s.q);
+      auto issue_pv = [&](long gp, bool first) -> bool {
+        if (first && !mbar_wait(&s.o_empty, (active & 1) ^ 1, abort_flag)) return false;
+        const int vs = (int)(gp & 1);
+        const uint32_t ph = (uint32_t)((gp >> 1) & 1);
+        if (!mbar_wait(&s.v_full[vs], ph, abort_flag)) return false;
+        if (!mbar_wait(&s.p_full[vs], ph, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(s.v[vs]);
+        const uint32_t p_addr = smem_u32(s.p[vs]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {  // 16 keys per MMA
+          const uint64_t da = sdesc_sw128(v_addr + kk * 2048, 2 * kTileBytes, 1024);
+          const uint64_t db = sdesc_sw128(p_addr + kk * 2048, kPBytes, 1024);
+          mma_bf16(tmem + kColO, da, db, idesc_o, (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(&s.p_empty[vs]);
+        mma_commit(&s.v_empty[vs]);
+        return true;
+      };
+      for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
+        const UnitInfo ui = unit_info(g, a, u);
+        if (ui.npairs == 0) continue;
+        if (!mbar_wait(&s.q_full, active & 1, abort_flag)) { ok = false; break; }
+        for (int n = 0; n < ui.npairs && ok; ++n) {
+          const long gp = gp0 + n;
+          const int ks = (int)(gp % kKStages);
+          const int sb = (int)(gp & 1);
+          if (!mbar_wait(&s.k_full[ks], (gp / kKStages) & 1, abort_flag) ||
+              !mbar_wait(&s.s_empty[sb], ((gp >> 1) & 1) ^ 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(s.k[ks]);
+#pragma unroll
+          for (int hh = 0; hh < kHalves; ++hh) {
+#pragma unroll
+            for (int st = 0; st < 4; ++st) {  // 16 elements of D per MMA
+              const uint64_t da = sdesc_sw128(k_addr + hh * 2 * kTileBytes + st * 32, 16, 1024);
+              const uint64_t db = sdesc_sw128(q_addr + hh * kTileBytes + st * 32, 16, 1024);
+              mma_bf16(tmem + kColS + sb * 64, da, db, idesc_s, (hh | st) ? 1u : 0u);
+            }
+          }
+          mma_commit(&s.s_full[sb]);
+          mma_commit(&s.k_empty[ks]);
+          if (n == ui.npairs - 1) mma_commit(&s.q_empty);
+          if (n >= 1) ok = issue_pv(gp - 1, n == 1);
+        }
+        if (ok) ok = issue_pv(gp0 + ui.npairs - 1, ui.npairs == 1);
+        if (!ok) break;
+        mma_commit(&s.o_full);
+        gp0 += ui.npairs;
+        ++active;
+      }
+      if (!ok) fail(s, a.dev_status);
+      // Every MMA issued must complete before TMEM is released.
+      mma_commit(&s.drain);
+      mbar_wait(&s.drain, 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------- softmax + epilogue (warps 2..5)
+    const int sp = warp & 3;            // TMEM sub-partition of this warp
+    const int r = sp * 32 + lane;       // TMEM lane: key row of S^T, column d of O^T
+    const int wq = warp - 2;            // 0..3 within the group
+    const int gt = threadIdx.x - 64;    // 0..127 within the group
+    const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
+    int active = 0;
+    long gp0 = 0;
+    bool reported = false;
+    float lpart[64];
+    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+      const UnitInfo ui = unit_info(g, a, u);
+      const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
+      const int vci = tile_valid_count(g, ui.i);
+      if (ui.npairs == 0) {
+        // No kept key tile: the output rows are zero.
+        const long ld = (long)g.heads * kD;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
+        for (int e = gt; e < kTileElems * kD / 8; e += kSoftmaxThreads) {
+          const int rr = e / (kD / 8), c = e - rr * (kD / 8);
+          *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+      if (gt < 64) s.shift[gt] = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 64; ++q) lpart[q] = 0.f;
+      named_bar(kSoftmaxBar, kSoftmaxThreads);
+      bool failed = false;
+      for (int n = 0; n < ui.npairs; ++n) {
+        const long gp = gp0 + n;
+        const int sb = (int)(gp & 1);
+        const uint32_t ph = (uint32_t)((gp >> 1) & 1);
+        bool ok = mbar_wait(&s.s_full[sb], ph, abort_flag);
+        ok = ok && mbar_wait(&s.p_empty[sb], ph ^ 1, abort_flag);
+        tc_fence_after();
+        float x[64];
+        {
+          uint32_t v[32];
+          tmem_ld32(lane_base + kColS + sb * 64, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(v[q]);
+          tmem_ld32(lane_base + kColS + sb * 64 + 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 32; ++q) x[32 + q] = __uint_as_float(v[q]);
+        }
+        tc_fence_before();
+        mbar_arrive(&s.s_empty[sb]);
+        // Validity of this thread's key: tile a holds rows 0..63, tile b rows 64..127.
+        const int jt = list_tile(g, ui, 2 * n + (r >> 6));
+        const bool valid = jt >= 0 && (r & 63) < tile_valid_count(g, jt);
+        if (!reported && wq == 0 && lane == 0) {
+          for (int e = 2 * n; e < 2 * n + 2 && e < ui.cnt; ++e)
+            if (ui.list[e] < 0 || ui.list[e] >= g.nT) {
+              report(a.dev_status, T3D_DEV_INDEX_RANGE);
+              reported = true;
+            }
+        }
+        bool over = false;
+#pragma unroll
+        for (int q = 0; q < 64; ++q) {
+          x[q] = valid ? x[q] * sl2 : -INFINITY;
+          over |= (x[q] - s.shift[q]) > kShiftSlack;
+        }
+        if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, !ok || *abort_flag)) { failed = true; break; }
+        if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, over)) {
+          // Slow step: raise the shifts to the running maxima and rescale what was accumulated.
+#pragma unroll
+          for (int q = 0; q < 64; ++q) {
+            const float mq = redux_max(x[q]);
+            if (lane == (q & 31)) s.red[wq][q] = mq;
+          }
+          named_bar(kSoftmaxBar, kSoftmaxThreads);
+          if (gt < 64) {
+            const float old = s.shift[gt];
+            float mx = fmaxf(fmaxf(s.red[0][gt], s.red[1][gt]), fmaxf(s.red[2][gt], s.red[3][gt]));
+            mx = fmaxf(mx, old);
+            s.alpha[gt] = (old == -INFINITY) ? (mx == -INFINITY ? 1.f : 0.f) : ex2(old - mx);
+            s.shift[gt] = mx;
+          }
+          named_bar(kSoftmaxBar, kSoftmaxThreads);
+          bool wok = true;
+          if (n > 0) {
+            // O^T holds the contributions of earlier steps: rescale column q by alpha[q] once the
+            // last PV MMA has landed.
+            wok = mbar_wait(&s.p_empty[(gp - 1) & 1], ((gp - 1) >> 1) & 1, abort_flag);
+            tc_fence_after();
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+              uint32_t v[32];
+              tmem_ld32(lane_base + kColO + half * 32, v);
+              tmem_wait_ld();
+#pragma unroll
+              for (int q = 0; q < 32; ++q)
+                v[q] = __float_as_uint(__uint_as_float(v[q]) * s.alpha[half * 32 + q]);
+              tmem_st32(lane_base + kColO + half * 32, v);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+          }
+#pragma unroll
+          for (int q = 0; q < 64; ++q) lpart[q] *= s.alpha[q];
+          if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, !wok)) { failed = true; break; }
+        }
+        // P = exp2(x - shift), running sums, bf16 row of P^T into shared memory (MN-major, 128B
+        // swizzle: 16-byte chunk c of row r lives at chunk c ^ (r & 7)).
+        uint8_t* prow = s.p[sb] + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int q = c * 8 + 2 * e;
+            const float b0 = s.shift[q] == -INFINITY ? 0.f : s.shift[q];
+            const float b1 = s.shift[q + 1] == -INFINITY ? 0.f : s.shift[q + 1];
+            const float p0 = ex2(x[q] - b0), p1 = ex2(x[q + 1] - b1);
+            lpart[q] += p0;
+            lpart[q + 1] += p1;
+            __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
+            w[e] = *reinterpret_cast<uint32_t*>(&pk);
+          }
+          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        fence_proxy_async();
+        mbar_arrive(&s.p_full[sb]);
+      }
+      if (failed) break;
+      // ---- epilogue: denominators (reduce the 128 per-key partial sums per query)
+#pragma unroll
+      for (int o = 16, c = 64; o >= 1; o >>= 1, c >>= 1) {
+        const bool hi = (lane & o) != 0;
+#pragma unroll
+        for (int j = 0; j < c / 2; ++j) {
+          const float send = hi ? lpart[j] : lpart[j + c / 2];
+          const float keep = hi ? lpart[j + c / 2] : lpart[j];
+          lpart[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      s.red[wq][2 * lane] = lpart[0];
+      s.red[wq][2 * lane + 1] = lpart[1];
+      const bool ook = mbar_wait(&s.o_full, active & 1, abort_flag);
+      named_bar(kSoftmaxBar, kSoftmaxThreads);
+      if (gt < 64) s.lsum[gt] = s.red[0][gt] + s.red[1][gt] + s.red[2][gt] + s.red[3][gt];
+      if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, !ook || *abort_flag)) break;
+      tc_fence_after();
+      // O^T row r (= column d of O): divide by the denominators, stage O as [64 q][128 d] bf16.
+      __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(s.p[0]);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t v[32];
+        tmem_ld32(lane_base + kColO + half * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+          const int qq = half * 32 + q;
+          const float l = s.lsum[qq];
+          const float val = l > 0.f ? __uint_as_float(v[q]) / l : 0.f;
+          stage[qq * kD + r] = __float2bfloat16_rn(val);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&s.o_empty);
+      named_bar(kSoftmaxBar, kSoftmaxThreads);
+      const long ld = (long)g.heads * kD;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
+      const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
+      const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
+      const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
+      for (int e = gt; e < kTileElems * kD / 8; e += kSoftmaxThreads) {
+        const int rr = e / (kD / 8), c = e - rr * (kD / 8);
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (rr < vci) {
+          int sr = rr;
+          if (keep != nullptr && !keep[rr]) {
+            sr = srcr[rr];
+            if (sr >= kTileElems) sr = rr;
+          }
+          val = *reinterpret_cast<const uint4*>(stage + sr * kD + c * 8);
+        }
+        *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = val;
+      }
+      named_bar(kSoftmaxBar, kSoftmaxThreads);
+      gp0 += ui.npairs;
+      ++active;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------------- host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 3D map over a [B * Lp, heads, D] bf16 tensor; box = 64 rows x 1 head x 64 elements, 128B swizzle.
+bool make_map(CUtensorMap* m, const void* base, const Geo& g) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.heads, (cuuint64_t)g.B * g.Lp};
+  const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.heads * g.D * 2};
+  const cuuint32_t box[3] = {64, 1, 64};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+}  // namespace
+
+cudaError_t launch_attn_sm100(const Geo& g, const AttnArgs& a, cudaStream_t s) {
+  Maps maps;
+  if (!make_map(&maps.q, a.q, g) || !make_map(&maps.k, a.k, g) || !make_map(&maps.v, a.v, g))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(SmemLayout) + 1024;
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int units = g.B * g.heads * g.nT;
+  const int grid = units < sm_count() ? units : sm_count();
+  const float sl2 = a.scale * 1.4426950408889634f;
+  attn_sm100_kernel<<<grid, kThreads, smem, s>>>(maps, g, a, sl2);
+  return cudaGetLastError();
+}
+
+}  // namespace t3d

@@ -42,6 +42,9 @@ struct AttnArgs {
 };
 
 size_t attn_workspace_bytes(const Geo& g, int kmax);
+// D = 128: tcgen05/TMEM/TMA kernel (attn_sm100.cu). D = 64: warp-MMA kernel (attn_mma.cu).
 cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attn_sm100(const Geo& g, const AttnArgs& a, cudaStream_t s);
+cudaError_t launch_attn_mma(const Geo& g, const AttnArgs& a, cudaStream_t s);
 
 }  // namespace t3d
