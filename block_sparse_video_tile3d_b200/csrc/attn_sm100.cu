@@ -17,10 +17,11 @@
 // Roles (one persistent CTA per SM, work units = (batch, head, query tile), static round robin):
 //   warp 0      TMA producer for Q (once per unit) and the K pairs (3-stage ring)
 //   warp 1      TMEM allocation; one thread issues every tcgen05.mma and tcgen05.commit
-//   warps 2..5  softmax and epilogue; thread t owns TMEM lane t (a key of S^T, a column d of O^T)
-//   warp 6      TMA producer for the V pairs (2-stage ring)
+//   warps 2..9  softmax and epilogue, two warpgroups splitting the 64 query columns; a thread owns
+//               TMEM lane t (a key of S^T, a column d of O^T) for its warpgroup's 32 queries
+//   warp 10     TMA producer for the V pairs (2-stage ring)
 //
-// Softmax. Each softmax thread holds one key's 64 logits. The shift subtracted before exp2 is a
+// Softmax. Each softmax thread holds one key's 32 logits (its warpgroup's half of the queries). The shift subtracted before exp2 is a
 // per-query value m[q] shared through shared memory; it is only raised (a "slow step": per-query
 // maxima by warp reductions, then a rescale of O^T and of the running sums) when some logit exceeds
 // m[q] by more than kShiftSlack (log2 units). Any shift gives the same softmax; the bound keeps P
@@ -42,9 +43,10 @@ constexpr int kD = 128;             // head dimension handled by this kernel
 constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a row
 constexpr int kKStages = 3;         // K-pair ring depth
 constexpr int kVStages = 2;         // V-pair ring depth
-constexpr int kThreads = 224;       // 7 warps
+constexpr int kThreads = 352;       // 11 warps
 constexpr int kSoftmaxThreads = 128;
-constexpr int kSoftmaxBar = 1;      // named barrier id of the softmax warps
+constexpr int kSoftmaxBar = 1;      // named barrier ids 1, 2: one per softmax warpgroup
+constexpr int kSoftmaxWarps = 8;
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0;       // S^T buffers: columns [0, 64) and [64, 128)
@@ -66,13 +68,18 @@ struct alignas(1024) SmemLayout {
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full[2], p_empty[2];
   uint64_t drain;
-  float shift[64];    // current per-query shift (log2 units)
-  float red[4][64];   // per-warp partial results
-  float alpha[64];    // rescale factors of a slow step
-  float lsum[64];     // per-query softmax denominators
+  uint64_t wg_sync;  // rendezvous of both softmax warpgroups (bounded, unlike bar.sync)
+  alignas(16) float shift[64];   // current per-query shift (log2 units)
+  alignas(16) float red[4][64];  // per-warp partial results
+  alignas(16) float alpha[64];   // rescale factors of a slow step
+  alignas(16) float lsum[64];    // per-query softmax denominators
+  uint8_t vc[kMaxTiles];         // valid token count of every tile
   uint32_t tmem_base;
   int abort;
 };
+
+static_assert(sizeof(SmemLayout) + 1024 <= 232448, "shared memory per CTA");
+constexpr int kAbsent = -0x7fffffff - 1;  // list entry beyond kv_cnt
 
 constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
 constexpr uint32_t idesc_o = idesc_bf16(128, 64, true, true);
@@ -125,19 +132,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.q_full, 1);
     mbar_init(&s.q_empty, 1);
     mbar_init(&s.o_full, 1);
-    mbar_init(&s.o_empty, kSoftmaxThreads);
+    mbar_init(&s.o_empty, 2 * kSoftmaxThreads);
     for (int t = 0; t < kKStages; ++t) { mbar_init(&s.k_full[t], 1); mbar_init(&s.k_empty[t], 1); }
     for (int t = 0; t < kVStages; ++t) { mbar_init(&s.v_full[t], 1); mbar_init(&s.v_empty[t], 1); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.s_empty[t], kSoftmaxThreads);
-      mbar_init(&s.p_full[t], kSoftmaxThreads);
+      mbar_init(&s.s_empty[t], 2 * kSoftmaxThreads);
+      mbar_init(&s.p_full[t], 2 * kSoftmaxThreads);
       mbar_init(&s.p_empty[t], 1);
     }
     mbar_init(&s.drain, 1);
+    mbar_init(&s.wg_sync, 2 * kSoftmaxThreads);
     s.abort = 0;
     fence_mbar_init();
   }
+  for (int t = threadIdx.x; t < g.nT; t += kThreads) s.vc[t] = (uint8_t)tile_valid_count(g, t);
   if (warp == 0 && lane == 0) {
     tma_prefetch(&maps.q);
     tma_prefetch(&maps.k);
@@ -191,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (long gp = issued - kKStages; gp < issued; ++gp)
         if (gp >= 0) mbar_wait(&s.k_full[gp % kKStages], (gp / kKStages) & 1, nullptr);
     }
-  } else if (warp == 6) {
+  } else if (warp == 2 + kSoftmaxWarps) {
     // ------------------------------------------------------------- V producer
     if (lane == 0) {
       long gp0 = 0, issued = 0;
@@ -288,138 +297,159 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&s.drain, 0, nullptr);
     }
   } else {
-    // ------------------------------------------------------------- softmax + epilogue (warps 2..5)
-    const int sp = warp & 3;            // TMEM sub-partition of this warp
+    // ------------------------------------------------------------- softmax + epilogue (warps 2..9)
+    // Two warpgroups split the 64 query columns: warpgroup wg owns columns [32 wg, 32 wg + 32).
+    // Within a warpgroup, warp sub-partition sp covers TMEM lanes [32 sp, 32 sp + 32).
+    const int wg = (warp - 2) >> 2;
+    const int sp = warp & 3;
     const int r = sp * 32 + lane;       // TMEM lane: key row of S^T, column d of O^T
-    const int wq = warp - 2;            // 0..3 within the group
-    const int gt = threadIdx.x - 64;    // 0..127 within the group
+    const int gt = ((warp - 2) & 3) * 32 + lane;  // 0..127 within the warpgroup
+    const int bar_id = kSoftmaxBar + wg;
+    const int q0 = wg * 32;
     const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
     int active = 0;
     long gp0 = 0;
     bool reported = false;
-    float lpart[64];
+    uint32_t sync_phase = 0;
+    // Both warpgroups meet here; false if the other one never arrives (timeout / abort).
+    auto rendezvous = [&]() -> bool {
+      mbar_arrive(&s.wg_sync);
+      const bool r_ok = mbar_wait(&s.wg_sync, sync_phase, abort_flag);
+      sync_phase ^= 1u;
+      return r_ok;
+    };
+    float lpart[32];
     for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
       const UnitInfo ui = unit_info(g, a, u);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
-      const int vci = tile_valid_count(g, ui.i);
+      const int vci = s.vc[ui.i];
+      const long ld = (long)g.heads * kD;
+      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
       if (ui.npairs == 0) {
-        // No kept key tile: the output rows are zero.
-        const long ld = (long)g.heads * kD;
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
-        for (int e = gt; e < kTileElems * kD / 8; e += kSoftmaxThreads) {
-          const int rr = e / (kD / 8), c = e - rr * (kD / 8);
+        // No kept key tile: this warpgroup's 32 output rows are zero.
+        for (int e = gt; e < 32 * kD / 8; e += kSoftmaxThreads) {
+          const int rr = q0 + e / (kD / 8), c = e % (kD / 8);
           *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = make_uint4(0u, 0u, 0u, 0u);
         }
         continue;
       }
-      if (gt < 64) s.shift[gt] = -INFINITY;
+      if (gt < 32) s.shift[q0 + gt] = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < 64; ++q) lpart[q] = 0.f;
-      named_bar(kSoftmaxBar, kSoftmaxThreads);
+      for (int q = 0; q < 32; ++q) lpart[q] = 0.f;
+      named_bar(bar_id, kSoftmaxThreads);
+      // Key tile of this thread's row for the first step (list entries are prefetched a step ahead).
+      int raw_next = ((r >> 6) < ui.cnt) ? ui.list[r >> 6] : kAbsent;
       bool failed = false;
       for (int n = 0; n < ui.npairs; ++n) {
         const long gp = gp0 + n;
         const int sb = (int)(gp & 1);
         const uint32_t ph = (uint32_t)((gp >> 1) & 1);
+        const int raw = raw_next;
+        const int e_next = 2 * (n + 1) + (r >> 6);
+        raw_next = (e_next < ui.cnt) ? ui.list[e_next] : kAbsent;
         bool ok = mbar_wait(&s.s_full[sb], ph, abort_flag);
         ok = ok && mbar_wait(&s.p_empty[sb], ph ^ 1, abort_flag);
         tc_fence_after();
-        float x[64];
+        float x[32];
         {
           uint32_t v[32];
-          tmem_ld32(lane_base + kColS + sb * 64, v);
+          tmem_ld32(lane_base + kColS + sb * 64 + q0, v);
           tmem_wait_ld();
 #pragma unroll
           for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(v[q]);
-          tmem_ld32(lane_base + kColS + sb * 64 + 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < 32; ++q) x[32 + q] = __uint_as_float(v[q]);
         }
         tc_fence_before();
         mbar_arrive(&s.s_empty[sb]);
-        // Validity of this thread's key: tile a holds rows 0..63, tile b rows 64..127.
-        const int jt = list_tile(g, ui, 2 * n + (r >> 6));
-        const bool valid = jt >= 0 && (r & 63) < tile_valid_count(g, jt);
-        if (!reported && wq == 0 && lane == 0) {
-          for (int e = 2 * n; e < 2 * n + 2 && e < ui.cnt; ++e)
-            if (ui.list[e] < 0 || ui.list[e] >= g.nT) {
-              report(a.dev_status, T3D_DEV_INDEX_RANGE);
-              reported = true;
-            }
+        const bool in_range = raw >= 0 && raw < g.nT;
+        const bool valid = in_range && (r & 63) < s.vc[in_range ? raw : 0];
+        if (!reported && raw != kAbsent && !in_range) {
+          report(a.dev_status, T3D_DEV_INDEX_RANGE);
+          reported = true;
+        }
+        float sh[32];
+#pragma unroll
+        for (int q = 0; q < 32; q += 4) {
+          const float4 v4 = *reinterpret_cast<const float4*>(&s.shift[q0 + q]);
+          sh[q] = v4.x; sh[q + 1] = v4.y; sh[q + 2] = v4.z; sh[q + 3] = v4.w;
         }
         bool over = false;
 #pragma unroll
-        for (int q = 0; q < 64; ++q) {
+        for (int q = 0; q < 32; ++q) {
           x[q] = valid ? x[q] * sl2 : -INFINITY;
-          over |= (x[q] - s.shift[q]) > kShiftSlack;
+          over |= (x[q] - sh[q]) > kShiftSlack;
         }
-        if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, !ok || *abort_flag)) { failed = true; break; }
-        if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, over)) {
+        const bool bad = !ok || *abort_flag;
+        if (named_bar_or(bar_id, kSoftmaxThreads, over || bad)) {
+          if (named_bar_or(bar_id, kSoftmaxThreads, bad)) { failed = true; break; }
           // Slow step: raise the shifts to the running maxima and rescale what was accumulated.
 #pragma unroll
-          for (int q = 0; q < 64; ++q) {
+          for (int q = 0; q < 32; ++q) {
             const float mq = redux_max(x[q]);
-            if (lane == (q & 31)) s.red[wq][q] = mq;
+            if (lane == q) s.red[sp][q0 + q] = mq;
           }
-          named_bar(kSoftmaxBar, kSoftmaxThreads);
-          if (gt < 64) {
-            const float old = s.shift[gt];
-            float mx = fmaxf(fmaxf(s.red[0][gt], s.red[1][gt]), fmaxf(s.red[2][gt], s.red[3][gt]));
+          named_bar(bar_id, kSoftmaxThreads);
+          if (gt < 32) {
+            const int qq = q0 + gt;
+            const float old = s.shift[qq];
+            float mx = fmaxf(fmaxf(s.red[0][qq], s.red[1][qq]), fmaxf(s.red[2][qq], s.red[3][qq]));
             mx = fmaxf(mx, old);
-            s.alpha[gt] = (old == -INFINITY) ? (mx == -INFINITY ? 1.f : 0.f) : ex2(old - mx);
-            s.shift[gt] = mx;
+            s.alpha[qq] = (old == -INFINITY) ? (mx == -INFINITY ? 1.f : 0.f) : ex2(old - mx);
+            s.shift[qq] = mx;
           }
-          named_bar(kSoftmaxBar, kSoftmaxThreads);
+          named_bar(bar_id, kSoftmaxThreads);
           bool wok = true;
           if (n > 0) {
             // O^T holds the contributions of earlier steps: rescale column q by alpha[q] once the
             // last PV MMA has landed.
             wok = mbar_wait(&s.p_empty[(gp - 1) & 1], ((gp - 1) >> 1) & 1, abort_flag);
             tc_fence_after();
+            uint32_t v[32];
+            tmem_ld32(lane_base + kColO + q0, v);
+            tmem_wait_ld();
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-              uint32_t v[32];
-              tmem_ld32(lane_base + kColO + half * 32, v);
-              tmem_wait_ld();
-#pragma unroll
-              for (int q = 0; q < 32; ++q)
-                v[q] = __float_as_uint(__uint_as_float(v[q]) * s.alpha[half * 32 + q]);
-              tmem_st32(lane_base + kColO + half * 32, v);
-            }
+            for (int q = 0; q < 32; ++q)
+              v[q] = __float_as_uint(__uint_as_float(v[q]) * s.alpha[q0 + q]);
+            tmem_st32(lane_base + kColO + q0, v);
             tmem_wait_st();
             tc_fence_before();
           }
 #pragma unroll
-          for (int q = 0; q < 64; ++q) lpart[q] *= s.alpha[q];
-          if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, !wok)) { failed = true; break; }
+          for (int q = 0; q < 32; q += 4) {
+            const float4 a4 = *reinterpret_cast<const float4*>(&s.alpha[q0 + q]);
+            lpart[q] *= a4.x; lpart[q + 1] *= a4.y; lpart[q + 2] *= a4.z; lpart[q + 3] *= a4.w;
+            const float4 v4 = *reinterpret_cast<const float4*>(&s.shift[q0 + q]);
+            sh[q] = v4.x; sh[q + 1] = v4.y; sh[q + 2] = v4.z; sh[q + 3] = v4.w;
+          }
+          if (named_bar_or(bar_id, kSoftmaxThreads, !wok)) { failed = true; break; }
         }
-        // P = exp2(x - shift), running sums, bf16 row of P^T into shared memory (MN-major, 128B
-        // swizzle: 16-byte chunk c of row r lives at chunk c ^ (r & 7)).
+        // P = exp2(x - shift), running sums, bf16 into this row of P^T (MN-major, 128B swizzle:
+        // 16-byte chunk c of row r lives at chunk c ^ (r & 7); this warpgroup owns chunks 4wg..4wg+3).
         uint8_t* prow = s.p[sb] + r * 128;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t w[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int q = c * 8 + 2 * e;
-            const float b0 = s.shift[q] == -INFINITY ? 0.f : s.shift[q];
-            const float b1 = s.shift[q + 1] == -INFINITY ? 0.f : s.shift[q + 1];
+            const float b0 = sh[q] == -INFINITY ? 0.f : sh[q];
+            const float b1 = sh[q + 1] == -INFINITY ? 0.f : sh[q + 1];
             const float p0 = ex2(x[q] - b0), p1 = ex2(x[q + 1] - b1);
             lpart[q] += p0;
             lpart[q + 1] += p1;
             __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
             w[e] = *reinterpret_cast<uint32_t*>(&pk);
           }
-          *reinterpret_cast<uint4*>(prow + ((c ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+          const int chunk = 4 * wg + c;
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async();
         mbar_arrive(&s.p_full[sb]);
       }
       if (failed) break;
-      // ---- epilogue: denominators (reduce the 128 per-key partial sums per query)
+      // ---- epilogue: denominators (reduce the 128 per-key partial sums of each query)
 #pragma unroll
-      for (int o = 16, c = 64; o >= 1; o >>= 1, c >>= 1) {
+      for (int o = 16, c = 32; o >= 1; o >>= 1, c >>= 1) {
         const bool hi = (lane & o) != 0;
 #pragma unroll
         for (int j = 0; j < c / 2; ++j) {
@@ -428,23 +458,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           lpart[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
         }
       }
-      s.red[wq][2 * lane] = lpart[0];
-      s.red[wq][2 * lane + 1] = lpart[1];
+      s.red[sp][q0 + lane] = lpart[0];  // after the halving, lane l holds query q0 + l
       const bool ook = mbar_wait(&s.o_full, active & 1, abort_flag);
-      named_bar(kSoftmaxBar, kSoftmaxThreads);
-      if (gt < 64) s.lsum[gt] = s.red[0][gt] + s.red[1][gt] + s.red[2][gt] + s.red[3][gt];
-      if (named_bar_or(kSoftmaxBar, kSoftmaxThreads, !ook || *abort_flag)) break;
+      named_bar(bar_id, kSoftmaxThreads);
+      if (gt < 32) {
+        const int qq = q0 + gt;
+        s.lsum[qq] = s.red[0][qq] + s.red[1][qq] + s.red[2][qq] + s.red[3][qq];
+      }
+      if (named_bar_or(bar_id, kSoftmaxThreads, !ook || *abort_flag)) break;
       tc_fence_after();
-      // O^T row r (= column d of O): divide by the denominators, stage O as [64 q][128 d] bf16.
+      // O^T row r (= column d of O) for this warpgroup's queries: divide by the denominators and
+      // stage O as [64 q][128 d] bf16 in the P^T buffer 0 (idle here: every PV MMA of the unit is
+      // complete and the next unit's first P^T write waits for the closing barrier below).
       __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(s.p[0]);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
+      {
         uint32_t v[32];
-        tmem_ld32(lane_base + kColO + half * 32, v);
+        tmem_ld32(lane_base + kColO + q0, v);
         tmem_wait_ld();
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-          const int qq = half * 32 + q;
+          const int qq = q0 + q;
           const float l = s.lsum[qq];
           const float val = l > 0.f ? __uint_as_float(v[q]) / l : 0.f;
           stage[qq * kD + r] = __float2bfloat16_rn(val);
@@ -452,14 +485,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&s.o_empty);
-      named_bar(kSoftmaxBar, kSoftmaxThreads);
-      const long ld = (long)g.heads * kD;
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
+      named_bar(bar_id, kSoftmaxThreads);
       const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
       const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
       const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
-      for (int e = gt; e < kTileElems * kD / 8; e += kSoftmaxThreads) {
-        const int rr = e / (kD / 8), c = e - rr * (kD / 8);
+      if (keep != nullptr) {  // source rows span both halves
+        if (named_bar_or(bar_id, kSoftmaxThreads, !rendezvous())) break;
+      }
+      for (int e = gt; e < 32 * kD / 8; e += kSoftmaxThreads) {
+        const int rr = q0 + e / (kD / 8), c = e % (kD / 8);
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
         if (rr < vci) {
           int sr = rr;
@@ -471,7 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = val;
       }
-      named_bar(kSoftmaxBar, kSoftmaxThreads);
+      // The staging buffer is free for the next unit once both warpgroups are done with it.
+      if (named_bar_or(bar_id, kSoftmaxThreads, !rendezvous())) break;
       gp0 += ui.npairs;
       ++active;
     }
