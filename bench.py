@@ -216,6 +216,8 @@ def _stage_bytes(w, name, pairs, kmax):
     """Algorithmic HBM bytes of one stage launch (each input read once, each output written once)."""
     B, heads, D, L, Lp, nT = w.B, w.heads, w.D, w.L, 64 * w.nT, w.nT
     row = heads * D * 2
+    if name.startswith("scatter_pool"):
+        return B * L * row + B * Lp * row + B * heads * nT * D * 4
     if name.startswith("scatter"):
         return B * L * row + B * Lp * row
     if name == "gather":

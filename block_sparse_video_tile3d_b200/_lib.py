@@ -39,6 +39,7 @@ SIGNATURES = {
     "tile3d_scatter": (_I, [_G, _P, _P, _P]),
     "tile3d_gather": (_I, [_G, _P, _P, _P]),
     "tile_pool": (_I, [_G, _P, _P, _P]),
+    "tile3d_scatter_pool": (_I, [_G, _P, _P, _P, _P]),
     "tile_select_topk": (_I, [_G, _P, _P, _I, _P, _P, _P, _P]),
     "tile_select_mass": (_I, [_G, _P, _P, _F, _F, _I, _I, _P, _P, _P, _P]),
     "tile_prune_queries": (_I, [_G, _P, _F, _P, _P, _P, _P]),

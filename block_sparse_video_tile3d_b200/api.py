@@ -17,6 +17,7 @@ from ._lib import Geom, Tile3dError, check, lib
 
 __all__ = [
     "Geom", "Tile3dError", "geometry", "tile3d_scatter", "tile3d_gather", "tile_pool",
+    "tile3d_scatter_pool",
     "tile_select_topk", "tile_select_mass", "tile_prune_queries", "block_mask_to_index",
     "block_sparse_attn_fwd", "block_sparse_attn_workspace_size", "TileSparseAttention",
 ]
@@ -100,6 +101,24 @@ def tile_pool(y: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None 
     g = _geom(B, T, H, W, nh, D)
     check(lib.tile_pool(ctypes.byref(g), _ptr(y), _ptr(out), _stream()))
     return out
+
+
+def tile3d_scatter_pool(x: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None,
+                        pooled: torch.Tensor | None = None):
+    """Scatter and pool in one pass: returns ``(y [B, Lp, heads, D] bf16, pooled [B, heads, nT, D]
+    fp32)``, the same as :func:`tile3d_scatter` then :func:`tile_pool`."""
+    B, L, nh, D = x.shape
+    _need(x, "x", torch.bfloat16, (B, T * H * W, nh, D))
+    nT, Lp, _ = _geometry(int(T), int(H), int(W), B, nh, D)
+    if out is None:
+        out = torch.empty((B, Lp, nh, D), dtype=torch.bfloat16, device=x.device)
+    if pooled is None:
+        pooled = torch.empty((B, nh, nT, D), dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.bfloat16, (B, Lp, nh, D))
+    _need(pooled, "pooled", torch.float32, (B, nh, nT, D))
+    g = _geom(B, T, H, W, nh, D)
+    check(lib.tile3d_scatter_pool(ctypes.byref(g), _ptr(x), _ptr(out), _ptr(pooled), _stream()))
+    return out, pooled
 
 
 def _sel_out(B, nh, nT, kcap, device, kv_idx, kv_cnt):
@@ -270,21 +289,28 @@ class TileSparseAttention:
             out = torch.empty((self.B, T * H * W, self.heads, self.D), dtype=torch.bfloat16,
                               device=q.device)
         self._out = out
-        st = [
-            ("scatter_q", lambda: tile3d_scatter(q, T, H, W, self.qt)),
-            ("scatter_k", lambda: tile3d_scatter(k, T, H, W, self.kt)),
-            ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt)),
-        ]
         if self.mode == "mask":
-            st.append(("mask_to_index", lambda: block_mask_to_index(
-                self.mask, T, H, W, self.D, self.kmax, self.kv_idx, self.kv_cnt, self.status)))
+            st = [
+                ("scatter_q", lambda: tile3d_scatter(q, T, H, W, self.qt)),
+                ("scatter_k", lambda: tile3d_scatter(k, T, H, W, self.kt)),
+                ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt)),
+                ("mask_to_index", lambda: block_mask_to_index(
+                    self.mask, T, H, W, self.D, self.kmax, self.kv_idx, self.kv_cnt,
+                    self.status)),
+            ]
         else:
+            if self.mode == "bsa":  # queries are pooled over kept rows, by the pruning kernel
+                st = [("scatter_q", lambda: tile3d_scatter(q, T, H, W, self.qt))]
+            else:
+                st = [("scatter_pool_q",
+                       lambda: tile3d_scatter_pool(q, T, H, W, self.qt, self.pq))]
+            st += [
+                ("scatter_pool_k", lambda: tile3d_scatter_pool(k, T, H, W, self.kt, self.pk)),
+                ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt)),
+            ]
             if self.mode == "bsa":
                 st.append(("prune_q", lambda: tile_prune_queries(
                     self.qt, T, H, W, self.cos_thresh, self.keep, self.src_row, self.pq)))
-            else:
-                st.append(("pool_q", lambda: tile_pool(self.qt, T, H, W, self.pq)))
-            st.append(("pool_k", lambda: tile_pool(self.kt, T, H, W, self.pk)))
             if self.mode == "topk":
                 st.append(("select_topk", lambda: tile_select_topk(
                     self.pq, self.pk, T, H, W, self.topk, self.kv_idx, self.kv_cnt, self.status)))

@@ -111,6 +111,17 @@ t3d_status tile_pool(const t3d_geom* g, const void* y, float* pooled, t3d_stream
   return cuda_status(t3d::launch_pool(geo, y, pooled, as_stream(stream)), "tile_pool");
 }
 
+t3d_status tile3d_scatter_pool(const t3d_geom* g, const void* x, void* y, float* pooled,
+                               t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(x, "x"));
+  T3D_CHECK(check_ptr(y, "y"));
+  T3D_CHECK(check_ptr(pooled, "pooled"));
+  return cuda_status(t3d::launch_scatter_pool(geo, x, y, pooled, as_stream(stream)),
+                     "tile3d_scatter_pool");
+}
+
 t3d_status tile_select_topk(const t3d_geom* g, const float* pq, const float* pk, int k,
                             int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
                             t3d_stream stream) {

@@ -11,7 +11,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/tile3d.h"
+#include "tile3d.h"
 
 namespace t3d {
 

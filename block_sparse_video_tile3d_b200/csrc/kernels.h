@@ -13,6 +13,8 @@ namespace t3d {
 cudaError_t launch_scatter(const Geo& g, const void* x, void* y, cudaStream_t s);
 cudaError_t launch_gather(const Geo& g, const void* y, void* x, cudaStream_t s);
 cudaError_t launch_pool(const Geo& g, const void* y, float* pooled, cudaStream_t s);
+cudaError_t launch_scatter_pool(const Geo& g, const void* x, void* y, float* pooled,
+                                cudaStream_t s);
 
 cudaError_t launch_select_topk(const Geo& g, const float* pq, const float* pk, int k,
                                int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,

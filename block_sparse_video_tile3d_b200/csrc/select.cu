@@ -4,67 +4,166 @@
 // K transposed, top-k per row, block map and LUT forms); bsa_attn page, BSAAttentionImpl.forward
 // (query pruning per block, KV blocks by cumulative threshold with a floor).
 //
-// Selection is exact on the fp32 scores: the k-th largest value of a row is found by a 32-step
-// bitwise search over an order-preserving uint32 image of the floats (no sort), ties at the
-// boundary go to the lower index, and kept indices are emitted in ascending order with warp ballots.
+// Selection is exact on the fp32 scores: the k-th largest value of a row is found by a radix
+// select (four 8-bit passes) over an order-preserving uint32 image of the floats (no sort), ties at
+// the boundary go to the lower index, and kept indices are emitted in ascending order with warp
+// ballots.
 #include "kernels.h"
 
 namespace t3d {
 namespace {
 
-constexpr int kSelRows = 8;  // query tiles per CTA, one warp each
-constexpr int kSelThreads = 32 * kSelRows;
-constexpr int kKeyChunk = 32;  // pooled key rows staged in shared memory at a time
+constexpr int kSelThreads = 256;  // 8 warps
+constexpr int kKeyChunk = 64;     // pooled key rows staged in shared memory at a time
+constexpr int kPad = 4;           // row padding (floats): rows 16 B apart modulo 128 B
 
-// Shared-memory layout of the score kernels (floats): pq rows, a key chunk padded to D+1 columns
-// (conflict-free column reads), then one nT-long row of values per warp.
-__host__ __device__ inline size_t sel_smem_floats(int D, int nT) {
-  return (size_t)kSelRows * D + (size_t)kKeyChunk * (D + 1) + (size_t)kSelRows * nT;
+// Query tiles per CTA: 16 (two per warp, enough CTAs to fill the GPU), or 8 when 16 score rows
+// would not fit next to the staged operands (~200 KB of shared memory).
+__host__ __device__ inline int sel_rows(int D, int nT) {
+  return ((size_t)(16 + kKeyChunk) * (D + kPad) * 4 + (size_t)16 * nT * 4 + 8 * 1024 <= 200 * 1024)
+             ? 16 : 8;
 }
 
-// Scores S[i, j] = pq_i . pk_j (fp32, sequential over d) for the CTA's kSelRows rows; row w of the
-// CTA lands in vals[w * nT + j].
+// Shared memory (floats): pq rows [R][D+4], a key chunk [64][D+4], the R score rows [R][nT], then
+// one 256-bin histogram per warp.
+__host__ __device__ inline size_t sel_smem_floats(int D, int nT, int R) {
+  return (size_t)(R + kKeyChunk) * (D + kPad) + (size_t)R * nT + 8 * 256;
+}
+
+// Scores S[i, j] = pq_i . pk_j in fp32 (accumulated over d in order, four at a time) for the CTA's
+// R query tiles i0 .. i0 + R - 1; row r lands in vals[r * nT + j]. Register blocking: thread
+// (row group, key group) computes RT rows x 4 keys of each 64-key chunk, keys kg + 16 j so that
+// the lanes of a quarter warp read consecutive padded rows (no bank conflicts).
+template <int RT>
 __device__ void compute_scores(const Geo& g, const float* __restrict__ pq,
-                               const float* __restrict__ pk, long bh, int i0, float* sm) {
-  const int D = g.D, nT = g.nT;
+                               const float* __restrict__ pk, long bh, int i0, int R, float* sm) {
+  const int D = g.D, nT = g.nT, ldp = D + kPad;
   float* pq_s = sm;
-  float* pk_s = pq_s + kSelRows * D;
-  float* vals = pk_s + kKeyChunk * (D + 1);
-  const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  for (int e = tid; e < kSelRows * D; e += kSelThreads) {
-    const int r = e / D, d = e - r * D;
+  float* pk_s = pq_s + R * ldp;
+  float* vals = pk_s + kKeyChunk * ldp;
+  const int tid = threadIdx.x;
+  const int d4 = D / 4;
+  for (int e = tid; e < R * d4; e += kSelThreads) {
+    const int r = e / d4, c = e - r * d4;
     const int i = i0 + r;
-    pq_s[e] = (i < nT) ? pq[(bh * nT + i) * D + d] : 0.f;
+    const float4 v = (i < nT) ? reinterpret_cast<const float4*>(pq + (bh * nT + i) * D)[c]
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(pq_s + r * ldp + 4 * c) = v;
   }
   const float* pkh = pk + bh * nT * D;
+  const int rg = tid >> 4, kg = tid & 15;
+  const bool active = rg * RT < R;
   for (int j0 = 0; j0 < nT; j0 += kKeyChunk) {
     __syncthreads();
     const int rows = imin(kKeyChunk, nT - j0);
-    for (int e = tid; e < kKeyChunk * D; e += kSelThreads) {
-      const int r = e / D, d = e - r * D;
-      pk_s[r * (D + 1) + d] = (r < rows) ? pkh[(long)(j0 + r) * D + d] : 0.f;
+    for (int e = tid; e < kKeyChunk * d4; e += kSelThreads) {
+      const int r = e / d4, c = e - r * d4;
+      const float4 v = (r < rows) ? reinterpret_cast<const float4*>(pkh + (long)(j0 + r) * D)[c]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+      *reinterpret_cast<float4*>(pk_s + r * ldp + 4 * c) = v;
     }
     __syncthreads();
-    if (lane < rows) {
-      const float* a = pq_s + w * D;
-      const float* kr = pk_s + lane * (D + 1);
-      float acc = 0.f;
-      for (int d = 0; d < D; ++d) acc = fmaf(a[d], kr[d], acc);
-      vals[w * nT + j0 + lane] = acc;
+    if (active) {
+      float acc[RT][4];
+#pragma unroll
+      for (int a = 0; a < RT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
+      for (int d = 0; d < D; d += 4) {
+        float4 qa[RT], kb[4];
+#pragma unroll
+        for (int a = 0; a < RT; ++a)
+          qa[a] = *reinterpret_cast<const float4*>(pq_s + (rg * RT + a) * ldp + d);
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+          kb[b] = *reinterpret_cast<const float4*>(pk_s + (kg + 16 * b) * ldp + d);
+#pragma unroll
+        for (int a = 0; a < RT; ++a)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            acc[a][b] = fmaf(qa[a].x, kb[b].x, acc[a][b]);
+            acc[a][b] = fmaf(qa[a].y, kb[b].y, acc[a][b]);
+            acc[a][b] = fmaf(qa[a].z, kb[b].z, acc[a][b]);
+            acc[a][b] = fmaf(qa[a].w, kb[b].w, acc[a][b]);
+          }
+      }
+#pragma unroll
+      for (int a = 0; a < RT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int j = kg + 16 * b;
+          if (j < rows) vals[(rg * RT + a) * nT + j0 + j] = acc[a][b];
+        }
     }
   }
   __syncthreads();
 }
 
-// Key of the k-th largest value of row[0..n) (1 <= k <= n), by bitwise search from the top bit.
-__device__ uint32_t kth_largest_key(const float* row, int n, int k) {
+__device__ void compute_scores_any(const Geo& g, const float* pq, const float* pk, long bh, int i0,
+                                   int R, float* sm) {
+  if (R >= 64) compute_scores<4>(g, pq, pk, bh, i0, R, sm);
+  else if (R == 32) compute_scores<2>(g, pq, pk, bh, i0, R, sm);
+  else compute_scores<1>(g, pq, pk, bh, i0, R, sm);
+}
+
+// Key of the k-th largest value of row[0..n) (1 <= k <= n): radix select on the order-preserving
+// uint32 keys, 8 bits per pass from the top, with a 256-bin histogram per warp (`hist`, shared
+// memory) filled by warp-aggregated atomics.
+__device__ uint32_t kth_largest_key(const float* row, int n, int k, int* hist) {
   const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = prefix | (1u << bit);
-    int c = 0;
-    for (int j = lane; j < n; j += 32) c += (float_key(row[j]) >= cand) ? 1 : 0;
-    if (warp_sum_int(c) >= k) prefix = cand;
+  uint32_t prefix = 0, mask = 0;
+  int krem = k;  // rank still to find among the keys matching the prefix
+  for (int shift = 24; shift >= 0; shift -= 8) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) hist[lane * 8 + t] = 0;
+    __syncwarp();
+    for (int j0 = 0; j0 < n; j0 += 32) {
+      const int j = j0 + lane;
+      const uint32_t key = j < n ? float_key(row[j]) : 0u;
+      const bool in = j < n && (key & mask) == prefix;
+      const unsigned act = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const int bin = (key >> shift) & 255;
+        const unsigned peers = __match_any_sync(act, bin);
+        if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
+      }
+    }
+    __syncwarp();
+    // Lane l owns bins 255 - 8 l .. 248 - 8 l (descending); find the bin holding rank krem.
+    int c[8], tot = 0;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      c[t] = hist[255 - (lane * 8 + t)];
+      tot += c[t];
+    }
+    int incl = tot;  // inclusive prefix over lanes (bins above and including this lane's)
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - tot;
+    const unsigned hit = __ballot_sync(0xffffffffu, excl < krem && incl >= krem);
+    const int owner = __ffs(hit) - 1;
+    int digit = 0, above = 0;
+    if (lane == owner) {
+      int run = excl;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (run + c[t] >= krem) {
+          digit = 255 - (lane * 8 + t);
+          above = run;
+          break;
+        }
+        run += c[t];
+      }
+    }
+    digit = __shfl_sync(0xffffffffu, digit, owner);
+    above = __shfl_sync(0xffffffffu, above, owner);
+    prefix |= (uint32_t)digit << shift;
+    mask |= 255u << shift;
+    krem -= above;
+    __syncwarp();
   }
   return prefix;
 }
@@ -94,10 +193,10 @@ __device__ int emit_threshold(const float* row, int n, uint32_t thr, int need_eq
 }
 
 // Top-k of row[0..n) into out (ascending indices). Returns k (clamped to n).
-__device__ int select_topk_row(const float* row, int n, int k, int32_t* out) {
+__device__ int select_topk_row(const float* row, int n, int k, int32_t* out, int* hist) {
   k = imin(k, n);
   if (k <= 0) return 0;
-  const uint32_t thr = kth_largest_key(row, n, k);
+  const uint32_t thr = kth_largest_key(row, n, k, hist);
   const int lane = threadIdx.x & 31;
   int gt = 0;
   for (int j = lane; j < n; j += 32) gt += (float_key(row[j]) > thr) ? 1 : 0;
@@ -108,41 +207,34 @@ __device__ int select_topk_row(const float* row, int n, int k, int32_t* out) {
 
 __global__ void __launch_bounds__(kSelThreads) topk_kernel(Geo g, const float* __restrict__ pq,
                                                            const float* __restrict__ pk, int k,
-                                                           int32_t* __restrict__ kv_idx,
+                                                           int R, int32_t* __restrict__ kv_idx,
                                                            int32_t* __restrict__ kv_cnt) {
-  extern __shared__ float sm[];
+  extern __shared__ float4 sm4[];
+  float* sm = reinterpret_cast<float*>(sm4);
   const int nT = g.nT;
-  const int blocks_per_head = (nT + kSelRows - 1) / kSelRows;
+  const int blocks_per_head = (nT + R - 1) / R;
   const long bh = blockIdx.x / blocks_per_head;
-  const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * kSelRows;
-  compute_scores(g, pq, pk, bh, i0, sm);
+  const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * R;
+  compute_scores_any(g, pq, pk, bh, i0, R, sm);
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = i0 + w;
-  if (i >= nT) return;
-  const float* row = sm + kSelRows * g.D + kKeyChunk * (g.D + 1) + w * nT;
+  const float* vals = sm + (R + kKeyChunk) * (g.D + kPad);
+  int* hist = reinterpret_cast<int*>(sm + (R + kKeyChunk) * (g.D + kPad) + R * nT) + w * 256;
   const int kk = imin(k, nT);
-  const int n = select_topk_row(row, nT, kk, kv_idx + (bh * nT + i) * kk);
-  if (lane == 0) kv_cnt[bh * nT + i] = n;
+  for (int r = w; r < R; r += kSelThreads / 32) {
+    const int i = i0 + r;
+    if (i >= nT) break;
+    const int n = select_topk_row(vals + r * nT, nT, kk, kv_idx + (bh * nT + i) * kk, hist);
+    if (lane == 0) kv_cnt[bh * nT + i] = n;
+  }
 }
 
-// Cumulative-mass selection. Values are replaced by e_j = exp(scale * (S_j - max S)); tiles are
-// ranked by e (ties: lower index) and the smallest prefix whose sum reaches mass * sum(e) is kept.
-__global__ void __launch_bounds__(kSelThreads) mass_kernel(Geo g, const float* __restrict__ pq,
-                                                           const float* __restrict__ pk,
-                                                           float scale, float mass, int min_k,
-                                                           int kmax, int32_t* __restrict__ kv_idx,
-                                                           int32_t* __restrict__ kv_cnt,
-                                                           int32_t* dev_status) {
-  extern __shared__ float sm[];
-  const int nT = g.nT;
-  const int blocks_per_head = (nT + kSelRows - 1) / kSelRows;
-  const long bh = blockIdx.x / blocks_per_head;
-  const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * kSelRows;
-  compute_scores(g, pq, pk, bh, i0, sm);
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int i = i0 + w;
-  if (i >= nT) return;
-  float* row = sm + kSelRows * g.D + kKeyChunk * (g.D + 1) + w * nT;
+// Cumulative-mass selection of one row (one warp). The scores in row[0..nT) are replaced by
+// e_j = exp(scale * (S_j - max S)); tiles are ranked by e (ties: lower index) and the smallest
+// prefix whose sum reaches mass * sum(e) is kept (at least min_k, at most kmax tiles, the most
+// probable ones; T3D_DEV_OVERFLOW when truncated). Writes ascending indices to out, returns the count.
+__device__ int select_mass_row(float* row, int nT, float scale, float mass, int min_k, int kmax,
+                               int32_t* out, int32_t* dev_status, int* hist) {
+  const int lane = threadIdx.x & 31;
   float mx = -INFINITY;
   for (int j = lane; j < nT; j += 32) mx = fmaxf(mx, row[j]);
   mx = warp_max(mx);
@@ -196,16 +288,41 @@ __global__ void __launch_bounds__(kSelThreads) mass_kernel(Geo g, const float* _
     }
   }
   int count = n_above + need_eq;
-  int32_t* out = kv_idx + (bh * nT + i) * kmax;
   const int floor_k = imin(min_k, nT);
   if (count < floor_k || count > kmax) {
     const int kk = count < floor_k ? floor_k : kmax;
     if (count > kmax && lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
-    count = select_topk_row(row, nT, imin(kk, kmax), out);
+    count = select_topk_row(row, nT, imin(kk, kmax), out, hist);
   } else {
     emit_threshold(row, nT, prefix, need_eq, out, kmax);
   }
-  if (lane == 0) kv_cnt[bh * nT + i] = count;
+  return count;
+}
+
+__global__ void __launch_bounds__(kSelThreads) mass_kernel(Geo g, const float* __restrict__ pq,
+                                                           const float* __restrict__ pk,
+                                                           float scale, float mass, int min_k,
+                                                           int kmax, int R,
+                                                           int32_t* __restrict__ kv_idx,
+                                                           int32_t* __restrict__ kv_cnt,
+                                                           int32_t* dev_status) {
+  extern __shared__ float4 sm4[];
+  float* sm = reinterpret_cast<float*>(sm4);
+  const int nT = g.nT;
+  const int blocks_per_head = (nT + R - 1) / R;
+  const long bh = blockIdx.x / blocks_per_head;
+  const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * R;
+  compute_scores_any(g, pq, pk, bh, i0, R, sm);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float* vals = sm + (R + kKeyChunk) * (g.D + kPad);
+  int* hist = reinterpret_cast<int*>(vals + R * nT) + w * 256;
+  for (int r = w; r < R; r += kSelThreads / 32) {
+    const int i = i0 + r;
+    if (i >= nT) break;
+    const int count = select_mass_row(vals + r * nT, nT, scale, mass, min_k, kmax,
+                                      kv_idx + (bh * nT + i) * kmax, dev_status, hist);
+    if (lane == 0) kv_cnt[bh * nT + i] = count;
+  }
 }
 
 // One warp per row of the block map.
@@ -368,24 +485,26 @@ cudaError_t launch_select_topk(const Geo& g, const float* pq, const float* pk, i
                                int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
                                cudaStream_t s) {
   (void)dev_status;
-  const size_t smem = sel_smem_floats(g.D, g.nT) * sizeof(float);
+  const int R = sel_rows(g.D, g.nT);
+  const size_t smem = sel_smem_floats(g.D, g.nT, R) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const long blocks = (long)g.B * g.heads * ((g.nT + kSelRows - 1) / kSelRows);
-  topk_kernel<<<(unsigned)blocks, kSelThreads, smem, s>>>(g, pq, pk, k, kv_idx, kv_cnt);
+  const long blocks = (long)g.B * g.heads * ((g.nT + R - 1) / R);
+  topk_kernel<<<(unsigned)blocks, kSelThreads, smem, s>>>(g, pq, pk, k, R, kv_idx, kv_cnt);
   return cudaGetLastError();
 }
 
 cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, float scale,
                                float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
                                int32_t* dev_status, cudaStream_t s) {
-  const size_t smem = sel_smem_floats(g.D, g.nT) * sizeof(float);
+  const int R = sel_rows(g.D, g.nT);
+  const size_t smem = sel_smem_floats(g.D, g.nT, R) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(mass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const long blocks = (long)g.B * g.heads * ((g.nT + kSelRows - 1) / kSelRows);
-  mass_kernel<<<(unsigned)blocks, kSelThreads, smem, s>>>(g, pq, pk, scale, mass, min_k, kmax,
+  const long blocks = (long)g.B * g.heads * ((g.nT + R - 1) / R);
+  mass_kernel<<<(unsigned)blocks, kSelThreads, smem, s>>>(g, pq, pk, scale, mass, min_k, kmax, R,
                                                           kv_idx, kv_cnt, dev_status);
   return cudaGetLastError();
 }

@@ -1,4 +1,4 @@
-// Tile scatter, untile (gather) and per-tile mean pooling.
+// Tile scatter, untile (gather), per-tile mean pooling, and scatter fused with pooling.
 //
 // FastVideo API docs: bsa_attn page (get_tile_partition_indices, preprocess_qkv,
 // postprocess_output), video_sparse_attn_h3 page (tile(): padded tile buffer, zero pads) and the
@@ -125,6 +125,64 @@ __global__ void __launch_bounds__(32 * kPoolRows) pool_kernel(Geo g, const uint4
   }
 }
 
+// Fused scatter + pool: grid (ceil(row_chunks / 32), nT, B), block (32, 8). The CTA moves one
+// 512-byte column slab of one tile: thread (lane, ry) copies chunk column `lane` of the tile's
+// padded rows ry, ry + 8, ... from their raster rows (zeros for pad slots) and sums the valid ones;
+// the 8 partial sums are combined in shared memory and divided by the valid count.
+__global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_kernel(Geo g,
+                                                                      const uint4* __restrict__ x,
+                                                                      uint4* __restrict__ y,
+                                                                      float* __restrict__ pooled) {
+  __shared__ float part[kPoolRows][32 * 8 + 4];
+  __shared__ int src_row[kTileElems];
+  const int lane = threadIdx.x;
+  const int ry = threadIdx.y;
+  const int i = blockIdx.y;
+  const int b = blockIdx.z;
+  const int c = blockIdx.x * 32 + lane;
+  const int t = ry * 32 + lane;
+  if (t < kTileElems) src_row[t] = padded_to_raster(g, i * kTileElems + t);
+  __syncthreads();
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  if (c < g.row_chunks) {
+    const long dst0 = ((long)b * g.Lp + (long)i * kTileElems) * g.row_chunks + c;
+    const long src_b = (long)b * g.L;
+#pragma unroll 4
+    for (int r = ry; r < kTileElems; r += kPoolRows) {
+      const int sr = src_row[r];
+      uint4 u = make_uint4(0u, 0u, 0u, 0u);
+      if (sr >= 0) {
+        u = ld_nc(x + (src_b + sr) * g.row_chunks + c);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          acc[2 * e] += f.x;
+          acc[2 * e + 1] += f.y;
+        }
+      }
+      y[dst0 + (long)r * g.row_chunks] = u;
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[ry][lane * 8 + e] = acc[e];
+  __syncthreads();
+  const int cc = t >> 3;
+  const int e = t & 7;
+  const int col_chunk = blockIdx.x * 32 + cc;
+  if (col_chunk < g.row_chunks) {
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < kPoolRows; ++q) sum += part[q][cc * 8 + e];
+    const int col = col_chunk * 8 + e;
+    const int h = col / g.D;
+    const int d = col - h * g.D;
+    pooled[(((long)b * g.heads + h) * g.nT + i) * g.D + d] = sum / (float)tile_valid_count(g, i);
+  }
+}
+
 int copy_grid(long rows) {
   long blocks = (rows + (kCopyThreads / 32) - 1) / (kCopyThreads / 32);
   const long cap = 148L * 16;
@@ -144,6 +202,15 @@ cudaError_t launch_gather(const Geo& g, const void* y, void* x, cudaStream_t s) 
   const long rows = (long)g.B * g.L;
   gather_kernel<<<copy_grid(rows), kCopyThreads, 0, s>>>(g, static_cast<const uint4*>(y),
                                                          static_cast<uint4*>(x));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_pool(const Geo& g, const void* x, void* y, float* pooled,
+                                cudaStream_t s) {
+  dim3 grid((g.row_chunks + 31) / 32, g.nT, g.B);
+  dim3 block(32, kPoolRows);
+  scatter_pool_kernel<<<grid, block, 0, s>>>(g, static_cast<const uint4*>(x), static_cast<uint4*>(y),
+                                             pooled);
   return cudaGetLastError();
 }
 

@@ -108,6 +108,17 @@ t3d_status tile3d_gather(const t3d_geom* g, const void* y, void* x, t3d_stream s
 t3d_status tile_pool(const t3d_geom* g, const void* y, float* pooled, t3d_stream stream);
 
 /*
+ * tile3d_scatter_pool — tile3d_scatter and tile_pool in one pass over the raster rows.
+ * Same contracts as the two calls above (bsa_attn page, get_tile_partition_indices; sla page,
+ * mean_pool); y and pooled are exactly what tile3d_scatter followed by tile_pool would write, up
+ * to the order of the fp32 additions. Saves re-reading y.
+ *   x: in, bf16 [B, L, heads, D] raster.  y: out, bf16 [B, Lp, heads, D].  pooled: out, fp32
+ *   [B, heads, nT, D].
+ */
+t3d_status tile3d_scatter_pool(const t3d_geom* g, const void* x, void* y, float* pooled,
+                               t3d_stream stream);
+
+/*
  * tile_select_topk — keep the k key tiles with the largest pooled scores per query tile.
  * FastVideo API docs, fastvideo.attention.backends page, sla.get_block_map:
  * S = pooled_q @ pooled_k^T (no softmax scale), top-k per row, recorded as an index list (LUT).

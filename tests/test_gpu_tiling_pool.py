@@ -65,3 +65,19 @@ def test_pool_workload_offsets_small():
     vc = tiling.variable_block_sizes(w.T, w.H, w.W)
     want = pool.tile_mean_pool(tiling.tile_scatter(f64(q[:, :, 5:6]), w.T, w.H, w.W), vc)
     np.testing.assert_allclose(got[:, 5:6], want, rtol=1e-5, atol=2e-6)
+
+
+@pytest.mark.parametrize("B,T,H,W,heads,D", GRIDS)
+def test_scatter_pool_fused_matches(B, T, H, W, heads, D):
+    from block_sparse_video_tile3d_b200 import tile3d_scatter_pool
+    x = _rand_bf16((B, T * H * W, heads, D), seed=T * 5 + W)
+    xd = x.cuda()
+    y, pooled = tile3d_scatter_pool(xd, T, H, W)
+    want = tiling.tile_scatter(x.view(torch.int16).numpy(), T, H, W)
+    np.testing.assert_array_equal(y.cpu().view(torch.int16).numpy(), want)
+    vc = tiling.variable_block_sizes(T, H, W)
+    got = f64(pooled)
+    hs = range(heads) if heads <= 3 else [0, heads - 1]
+    for h in hs:
+        ref = pool.tile_mean_pool(tiling.tile_scatter(f64(x[:, :, h:h + 1]), T, H, W), vc)
+        np.testing.assert_allclose(got[:, h:h + 1], ref, rtol=1e-5, atol=2e-6)
