@@ -236,7 +236,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int active = 0;
       long gp0 = 0;
       bool ok = true;
-      const uint32_t q_addr = smem_u32(s.q);
+      // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4 and
+      // every buffer lies below 256 KB), so each MMA's operands are a base descriptor plus a
+      // constant: the issuing thread builds none of them in the loop.
+      const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
+      const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
+      const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
+      const uint64_t dp = sdesc_sw128(smem_u32(s.p[0]), kPBytes, 1024);
       auto issue_pv = [&](long gp, bool first) -> bool {
         if (first && !mbar_wait(&s.o_empty, (active & 1) ^ 1, abort_flag)) return false;
         const int vs = (int)(gp & 1);
@@ -244,14 +250,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&s.v_full[vs], ph, abort_flag)) return false;
         if (!mbar_wait(&s.p_full[vs], ph, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(s.v[vs]);
-        const uint32_t p_addr = smem_u32(s.p[vs]);
+        const uint64_t da0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
+        const uint64_t db0 = dp + (uint64_t)(vs * (kPBytes >> 4));
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {  // 16 keys per MMA
-          const uint64_t da = sdesc_sw128(v_addr + kk * 2048, 2 * kTileBytes, 1024);
-          const uint64_t db = sdesc_sw128(p_addr + kk * 2048, kPBytes, 1024);
-          mma_bf16(tmem + kColO, da, db, idesc_o, (first && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V^T and of P^T) per MMA
+          mma_bf16(tmem + kColO, da0 + kk * (2048 >> 4), db0 + kk * (2048 >> 4), idesc_o,
+                   (first && kk == 0) ? 0u : 1u);
         mma_commit(&s.p_empty[vs]);
         mma_commit(&s.v_empty[vs]);
         return true;
@@ -270,15 +274,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(s.k[ks]);
+          const uint64_t da0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
+          const uint32_t d_s = tmem + kColS + sb * 64;
 #pragma unroll
           for (int hh = 0; hh < kHalves; ++hh) {
 #pragma unroll
-            for (int st = 0; st < 4; ++st) {  // 16 elements of D per MMA
-              const uint64_t da = sdesc_sw128(k_addr + hh * 2 * kTileBytes + st * 32, 16, 1024);
-              const uint64_t db = sdesc_sw128(q_addr + hh * kTileBytes + st * 32, 16, 1024);
-              mma_bf16(tmem + kColS + sb * 64, da, db, idesc_s, (hh | st) ? 1u : 0u);
-            }
+            for (int st = 0; st < 4; ++st)  // 16 elements of D (32 bytes) per MMA
+              mma_bf16(d_s, da0 + ((hh * 2 * kTileBytes + st * 32) >> 4),
+                       dq + ((hh * kTileBytes + st * 32) >> 4), idesc_s, (hh | st) ? 1u : 0u);
           }
           mma_commit(&s.s_full[sb]);
           mma_commit(&s.k_empty[ks]);
