@@ -43,10 +43,12 @@ constexpr int kD = 128;             // head dimension handled by this kernel
 constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a row
 constexpr int kKStages = 3;         // K-pair ring depth
 constexpr int kVStages = 2;         // V-pair ring depth
-constexpr int kThreads = 352;       // 11 warps
+constexpr int kQW = 16;             // query columns per softmax warpgroup
+constexpr int kWGs = 64 / kQW;      // softmax warpgroups
 constexpr int kSoftmaxThreads = 128;
-constexpr int kSoftmaxBar = 1;      // named barrier ids 1, 2: one per softmax warpgroup
-constexpr int kSoftmaxWarps = 8;
+constexpr int kSoftmaxBar = 1;      // named barrier ids 1 .. kWGs: one per softmax warpgroup
+constexpr int kSoftmaxWarps = 4 * kWGs;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 4);  // + Q/K producer, two MMA issuers, V producer
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
 constexpr uint32_t kTmemCols = 256;
 constexpr uint32_t kColS = 0;       // S^T buffers: columns [0, 64) and [64, 128)
@@ -70,6 +72,8 @@ struct alignas(1024) SmemLayout {
   uint64_t drain;
   uint64_t wg_sync;  // rendezvous of both softmax warpgroups (bounded, unlike bar.sync)
   alignas(16) float shift[64];   // current per-query shift (log2 units)
+  alignas(16) float thr[64];     // raw logit above which a step is slow: (shift + slack) / scale
+  alignas(16) float nsh[64];     // -shift, or 0 while the shift is -inf
   alignas(16) float red[4][64];  // per-warp partial results
   alignas(16) float alpha[64];   // rescale factors of a slow step
   alignas(16) float lsum[64];    // per-query softmax denominators
@@ -132,17 +136,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.q_full, 1);
     mbar_init(&s.q_empty, 1);
     mbar_init(&s.o_full, 1);
-    mbar_init(&s.o_empty, 2 * kSoftmaxThreads);
+    mbar_init(&s.o_empty, kWGs * kSoftmaxThreads);
     for (int t = 0; t < kKStages; ++t) { mbar_init(&s.k_full[t], 1); mbar_init(&s.k_empty[t], 1); }
     for (int t = 0; t < kVStages; ++t) { mbar_init(&s.v_full[t], 1); mbar_init(&s.v_empty[t], 1); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.s_empty[t], 2 * kSoftmaxThreads);
-      mbar_init(&s.p_full[t], 2 * kSoftmaxThreads);
+      mbar_init(&s.s_empty[t], kWGs * kSoftmaxThreads);
+      mbar_init(&s.p_full[t], kWGs * kSoftmaxThreads);
       mbar_init(&s.p_empty[t], 1);
     }
-    mbar_init(&s.drain, 1);
-    mbar_init(&s.wg_sync, 2 * kSoftmaxThreads);
+    mbar_init(&s.drain, 2);  // one commit from each MMA-issuing thread
+    mbar_init(&s.wg_sync, kWGs * kSoftmaxThreads);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -230,8 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (long gp = issued - kVStages; gp < issued; ++gp)
         if (gp >= 0) mbar_wait(&s.v_full[gp & 1], (gp >> 1) & 1, nullptr);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 3 + kSoftmaxWarps) {
+    // ------------------------------------------------------------- MMA issuers
+    // Two threads issue the MMAs: warp 1 the S^T chains, warp 11 the PV chains. Each waits only on
+    // what its own chains read, so a late P^T never holds back the next scores (and vice versa);
+    // each commit tracks the MMAs of the thread that issues it.
     if (lane == 0) {
       int active = 0;
       long gp0 = 0;
@@ -243,54 +250,60 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
       const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
       const uint64_t dp = sdesc_sw128(smem_u32(s.p[0]), kPBytes, 1024);
-      auto issue_pv = [&](long gp, bool first) -> bool {
-        if (first && !mbar_wait(&s.o_empty, (active & 1) ^ 1, abort_flag)) return false;
-        const int vs = (int)(gp & 1);
-        const uint32_t ph = (uint32_t)((gp >> 1) & 1);
-        if (!mbar_wait(&s.v_full[vs], ph, abort_flag)) return false;
-        if (!mbar_wait(&s.p_full[vs], ph, abort_flag)) return false;
-        tc_fence_after();
-        const uint64_t da0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
-        const uint64_t db0 = dp + (uint64_t)(vs * (kPBytes >> 4));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V^T and of P^T) per MMA
-          mma_bf16(tmem + kColO, da0 + kk * (2048 >> 4), db0 + kk * (2048 >> 4), idesc_o,
-                   (first && kk == 0) ? 0u : 1u);
-        mma_commit(&s.p_empty[vs]);
-        mma_commit(&s.v_empty[vs]);
-        return true;
-      };
+      const bool s_issuer = warp == 1;
       for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
         const UnitInfo ui = unit_info(g, a, u);
         if (ui.npairs == 0) continue;
-        if (!mbar_wait(&s.q_full, active & 1, abort_flag)) { ok = false; break; }
-        for (int n = 0; n < ui.npairs && ok; ++n) {
-          const long gp = gp0 + n;
-          const int ks = (int)(gp % kKStages);
-          const int sb = (int)(gp & 1);
-          if (!mbar_wait(&s.k_full[ks], (gp / kKStages) & 1, abort_flag) ||
-              !mbar_wait(&s.s_empty[sb], ((gp >> 1) & 1) ^ 1, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t da0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
-          const uint32_t d_s = tmem + kColS + sb * 64;
+        if (s_issuer) {
+          if (!mbar_wait(&s.q_full, active & 1, abort_flag)) { ok = false; break; }
+          for (int n = 0; n < ui.npairs && ok; ++n) {
+            const long gp = gp0 + n;
+            const int ks = (int)(gp % kKStages);
+            const int sb = (int)(gp & 1);
+            if (!mbar_wait(&s.k_full[ks], (gp / kKStages) & 1, abort_flag) ||
+                !mbar_wait(&s.s_empty[sb], ((gp >> 1) & 1) ^ 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t da0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
+            const uint32_t d_s = tmem + kColS + sb * 64;
 #pragma unroll
-          for (int hh = 0; hh < kHalves; ++hh) {
+            for (int hh = 0; hh < kHalves; ++hh) {
 #pragma unroll
-            for (int st = 0; st < 4; ++st)  // 16 elements of D (32 bytes) per MMA
-              mma_bf16(d_s, da0 + ((hh * 2 * kTileBytes + st * 32) >> 4),
-                       dq + ((hh * kTileBytes + st * 32) >> 4), idesc_s, (hh | st) ? 1u : 0u);
+              for (int st = 0; st < 4; ++st)  // 16 elements of D (32 bytes) per MMA
+                mma_bf16(d_s, da0 + ((hh * 2 * kTileBytes + st * 32) >> 4),
+                         dq + ((hh * kTileBytes + st * 32) >> 4), idesc_s, (hh | st) ? 1u : 0u);
+            }
+            mma_commit(&s.s_full[sb]);
+            mma_commit(&s.k_empty[ks]);
+            if (n == ui.npairs - 1) mma_commit(&s.q_empty);
           }
-          mma_commit(&s.s_full[sb]);
-          mma_commit(&s.k_empty[ks]);
-          if (n == ui.npairs - 1) mma_commit(&s.q_empty);
-          if (n >= 1) ok = issue_pv(gp - 1, n == 1);
+        } else {
+          for (int n = 0; n < ui.npairs && ok; ++n) {
+            const long gp = gp0 + n;
+            const bool first = n == 0;
+            const int vs = (int)(gp & 1);
+            const uint32_t ph = (uint32_t)((gp >> 1) & 1);
+            if ((first && !mbar_wait(&s.o_empty, (active & 1) ^ 1, abort_flag)) ||
+                !mbar_wait(&s.v_full[vs], ph, abort_flag) ||
+                !mbar_wait(&s.p_full[vs], ph, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t da0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
+            const uint64_t db0 = dp + (uint64_t)(vs * (kPBytes >> 4));
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V^T and of P^T) per MMA
+              mma_bf16(tmem + kColO, da0 + kk * (2048 >> 4), db0 + kk * (2048 >> 4), idesc_o,
+                       (first && kk == 0) ? 0u : 1u);
+            mma_commit(&s.p_empty[vs]);
+            mma_commit(&s.v_empty[vs]);
+          }
+          if (ok) mma_commit(&s.o_full);
         }
-        if (ok) ok = issue_pv(gp0 + ui.npairs - 1, ui.npairs == 1);
         if (!ok) break;
-        mma_commit(&s.o_full);
         gp0 += ui.npairs;
         ++active;
       }
@@ -300,28 +313,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&s.drain, 0, nullptr);
     }
   } else {
-    // ------------------------------------------------------------- softmax + epilogue (warps 2..9)
-    // Two warpgroups split the 64 query columns: warpgroup wg owns columns [32 wg, 32 wg + 32).
+    // ------------------------------------------------------------- softmax + epilogue
+    // kWGs warpgroups split the 64 query columns: warpgroup wg owns columns [kQW wg, kQW wg + kQW).
     // Within a warpgroup, warp sub-partition sp covers TMEM lanes [32 sp, 32 sp + 32).
     const int wg = (warp - 2) >> 2;
     const int sp = warp & 3;
     const int r = sp * 32 + lane;       // TMEM lane: key row of S^T, column d of O^T
     const int gt = ((warp - 2) & 3) * 32 + lane;  // 0..127 within the warpgroup
     const int bar_id = kSoftmaxBar + wg;
-    const int q0 = wg * 32;
+    const int q0 = wg * kQW;
     const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
     int active = 0;
     long gp0 = 0;
     bool reported = false;
     uint32_t sync_phase = 0;
-    // Both warpgroups meet here; false if the other one never arrives (timeout / abort).
+    // All softmax warpgroups meet here; false if one never arrives (timeout / abort).
     auto rendezvous = [&]() -> bool {
       mbar_arrive(&s.wg_sync);
       const bool r_ok = mbar_wait(&s.wg_sync, sync_phase, abort_flag);
       sync_phase ^= 1u;
       return r_ok;
     };
-    float lpart[32];
+    float lpart[kQW];
     for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
       const UnitInfo ui = unit_info(g, a, u);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
@@ -329,16 +342,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long ld = (long)g.heads * kD;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
       if (ui.npairs == 0) {
-        // No kept key tile: this warpgroup's 32 output rows are zero.
-        for (int e = gt; e < 32 * kD / 8; e += kSoftmaxThreads) {
+        // No kept key tile: this warpgroup's output rows are zero.
+        for (int e = gt; e < kQW * kD / 8; e += kSoftmaxThreads) {
           const int rr = q0 + e / (kD / 8), c = e % (kD / 8);
           *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = make_uint4(0u, 0u, 0u, 0u);
         }
         continue;
       }
-      if (gt < 32) s.shift[q0 + gt] = -INFINITY;
+      if (gt < kQW) {
+        s.shift[q0 + gt] = -INFINITY;
+        s.thr[q0 + gt] = -INFINITY;
+        s.nsh[q0 + gt] = 0.f;
+      }
 #pragma unroll
-      for (int q = 0; q < 32; ++q) lpart[q] = 0.f;
+      for (int q = 0; q < kQW; ++q) lpart[q] = 0.f;
       named_bar(bar_id, kSoftmaxThreads);
       // Key tile of this thread's row for the first step (list entries are prefetched a step ahead).
       int raw_next = ((r >> 6) < ui.cnt) ? ui.list[r >> 6] : kAbsent;
@@ -350,16 +367,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int raw = raw_next;
         const int e_next = 2 * (n + 1) + (r >> 6);
         raw_next = (e_next < ui.cnt) ? ui.list[e_next] : kAbsent;
+        // S^T of this step, and P^T buffer sb free again (its PV MMAs of step gp - 2 complete).
         bool ok = mbar_wait(&s.s_full[sb], ph, abort_flag);
         ok = ok && mbar_wait(&s.p_empty[sb], ph ^ 1, abort_flag);
         tc_fence_after();
-        float x[32];
+        float x[kQW];
         {
-          uint32_t v[32];
-          tmem_ld32(lane_base + kColS + sb * 64 + q0, v);
+          uint32_t v[kQW];
+          tmem_ld<kQW>(lane_base + kColS + sb * 64 + q0, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 32; ++q) x[q] = __uint_as_float(v[q]);
+          for (int q = 0; q < kQW; ++q) x[q] = __uint_as_float(v[q]);
         }
         tc_fence_before();
         mbar_arrive(&s.s_empty[sb]);
@@ -369,35 +387,36 @@ __global__ void __launch_bounds__(kThreads, 1)
           report(a.dev_status, T3D_DEV_INDEX_RANGE);
           reported = true;
         }
-        float sh[32];
+        if (!valid) {
 #pragma unroll
-        for (int q = 0; q < 32; q += 4) {
-          const float4 v4 = *reinterpret_cast<const float4*>(&s.shift[q0 + q]);
-          sh[q] = v4.x; sh[q + 1] = v4.y; sh[q + 2] = v4.z; sh[q + 3] = v4.w;
+          for (int q = 0; q < kQW; ++q) x[q] = -INFINITY;
         }
+        // x holds raw logits; the softmax scale (> 0) is folded into the thresholds and the exp2.
         bool over = false;
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-          x[q] = valid ? x[q] * sl2 : -INFINITY;
-          over |= (x[q] - sh[q]) > kShiftSlack;
+        for (int q = 0; q < kQW; q += 4) {
+          const float4 t4 = *reinterpret_cast<const float4*>(&s.thr[q0 + q]);
+          over |= (x[q] > t4.x) | (x[q + 1] > t4.y) | (x[q + 2] > t4.z) | (x[q + 3] > t4.w);
         }
         const bool bad = !ok || *abort_flag;
         if (named_bar_or(bar_id, kSoftmaxThreads, over || bad)) {
           if (named_bar_or(bar_id, kSoftmaxThreads, bad)) { failed = true; break; }
           // Slow step: raise the shifts to the running maxima and rescale what was accumulated.
 #pragma unroll
-          for (int q = 0; q < 32; ++q) {
+          for (int q = 0; q < kQW; ++q) {
             const float mq = redux_max(x[q]);
             if (lane == q) s.red[sp][q0 + q] = mq;
           }
           named_bar(bar_id, kSoftmaxThreads);
-          if (gt < 32) {
+          if (gt < kQW) {
             const int qq = q0 + gt;
             const float old = s.shift[qq];
             float mx = fmaxf(fmaxf(s.red[0][qq], s.red[1][qq]), fmaxf(s.red[2][qq], s.red[3][qq]));
-            mx = fmaxf(mx, old);
+            mx = fmaxf(mx * sl2, old);
             s.alpha[qq] = (old == -INFINITY) ? (mx == -INFINITY ? 1.f : 0.f) : ex2(old - mx);
             s.shift[qq] = mx;
+            s.thr[qq] = mx == -INFINITY ? -INFINITY : (mx + kShiftSlack) / sl2;
+            s.nsh[qq] = mx == -INFINITY ? 0.f : -mx;
           }
           named_bar(bar_id, kSoftmaxThreads);
           bool wok = true;
@@ -406,43 +425,43 @@ __global__ void __launch_bounds__(kThreads, 1)
             // last PV MMA has landed.
             wok = mbar_wait(&s.p_empty[(gp - 1) & 1], ((gp - 1) >> 1) & 1, abort_flag);
             tc_fence_after();
-            uint32_t v[32];
-            tmem_ld32(lane_base + kColO + q0, v);
+            uint32_t v[kQW];
+            tmem_ld<kQW>(lane_base + kColO + q0, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < 32; ++q)
+            for (int q = 0; q < kQW; ++q)
               v[q] = __float_as_uint(__uint_as_float(v[q]) * s.alpha[q0 + q]);
-            tmem_st32(lane_base + kColO + q0, v);
+            tmem_st<kQW>(lane_base + kColO + q0, v);
             tmem_wait_st();
             tc_fence_before();
           }
 #pragma unroll
-          for (int q = 0; q < 32; q += 4) {
+          for (int q = 0; q < kQW; q += 4) {
             const float4 a4 = *reinterpret_cast<const float4*>(&s.alpha[q0 + q]);
             lpart[q] *= a4.x; lpart[q + 1] *= a4.y; lpart[q + 2] *= a4.z; lpart[q + 3] *= a4.w;
-            const float4 v4 = *reinterpret_cast<const float4*>(&s.shift[q0 + q]);
-            sh[q] = v4.x; sh[q + 1] = v4.y; sh[q + 2] = v4.z; sh[q + 3] = v4.w;
           }
           if (named_bar_or(bar_id, kSoftmaxThreads, !wok)) { failed = true; break; }
         }
         // P = exp2(x - shift), running sums, bf16 into this row of P^T (MN-major, 128B swizzle:
-        // 16-byte chunk c of row r lives at chunk c ^ (r & 7); this warpgroup owns chunks 4wg..4wg+3).
+        // 16-byte chunk c of row r lives at chunk c ^ (r & 7); this warpgroup owns kQW / 8 chunks).
         uint8_t* prow = s.p[sb] + r * 128;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < kQW / 8; ++c) {
           uint32_t w[4];
+          const float4 n0 = *reinterpret_cast<const float4*>(&s.nsh[q0 + c * 8]);
+          const float4 n1 = *reinterpret_cast<const float4*>(&s.nsh[q0 + c * 8 + 4]);
+          const float nsh[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int q = c * 8 + 2 * e;
-            const float b0 = sh[q] == -INFINITY ? 0.f : sh[q];
-            const float b1 = sh[q + 1] == -INFINITY ? 0.f : sh[q + 1];
-            const float p0 = ex2(x[q] - b0), p1 = ex2(x[q + 1] - b1);
+            const float p0 = ex2(fmaf(x[q], sl2, nsh[2 * e]));
+            const float p1 = ex2(fmaf(x[q + 1], sl2, nsh[2 * e + 1]));
             lpart[q] += p0;
             lpart[q + 1] += p1;
             __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
             w[e] = *reinterpret_cast<uint32_t*>(&pk);
           }
-          const int chunk = 4 * wg + c;
+          const int chunk = (kQW / 8) * wg + c;
           *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) =
               make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -452,19 +471,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (failed) break;
       // ---- epilogue: denominators (reduce the 128 per-key partial sums of each query)
 #pragma unroll
-      for (int o = 16, c = 32; o >= 1; o >>= 1, c >>= 1) {
-        const bool hi = (lane & o) != 0;
+      for (int q = 0; q < kQW; ++q) {
+        float v = lpart[q];
 #pragma unroll
-        for (int j = 0; j < c / 2; ++j) {
-          const float send = hi ? lpart[j] : lpart[j + c / 2];
-          const float keep = hi ? lpart[j + c / 2] : lpart[j];
-          lpart[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
+        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == q) s.red[sp][q0 + q] = v;
       }
-      s.red[sp][q0 + lane] = lpart[0];  // after the halving, lane l holds query q0 + l
       const bool ook = mbar_wait(&s.o_full, active & 1, abort_flag);
       named_bar(bar_id, kSoftmaxThreads);
-      if (gt < 32) {
+      if (gt < kQW) {
         const int qq = q0 + gt;
         s.lsum[qq] = s.red[0][qq] + s.red[1][qq] + s.red[2][qq] + s.red[3][qq];
       }
@@ -472,14 +487,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // O^T row r (= column d of O) for this warpgroup's queries: divide by the denominators and
       // stage O as [64 q][128 d] bf16 in the P^T buffer 0 (idle here: every PV MMA of the unit is
-      // complete and the next unit's first P^T write waits for the closing barrier below).
+      // complete and the next unit's first P^T write waits for the closing rendezvous below).
       __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(s.p[0]);
       {
-        uint32_t v[32];
-        tmem_ld32(lane_base + kColO + q0, v);
+        uint32_t v[kQW];
+        tmem_ld<kQW>(lane_base + kColO + q0, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
+        for (int q = 0; q < kQW; ++q) {
           const int qq = q0 + q;
           const float l = s.lsum[qq];
           const float val = l > 0.f ? __uint_as_float(v[q]) / l : 0.f;
@@ -492,10 +507,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
       const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
       const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
-      if (keep != nullptr) {  // source rows span both halves
+      if (keep != nullptr) {  // source rows span every warpgroup's staging rows
         if (named_bar_or(bar_id, kSoftmaxThreads, !rendezvous())) break;
       }
-      for (int e = gt; e < 32 * kD / 8; e += kSoftmaxThreads) {
+      for (int e = gt; e < kQW * kD / 8; e += kSoftmaxThreads) {
         const int rr = q0 + e / (kD / 8), c = e % (kD / 8);
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
         if (rr < vci) {
@@ -508,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = val;
       }
-      // The staging buffer is free for the next unit once both warpgroups are done with it.
+      // The staging buffer is free for the next unit once every warpgroup is done with it.
       if (named_bar_or(bar_id, kSoftmaxThreads, !rendezvous())) break;
       gp0 += ui.npairs;
       ++active;
