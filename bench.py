@@ -239,7 +239,7 @@ def _source_sha() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_video_tile3d_b200", "csrc")
     for n in sorted(os.listdir(csrc)):
-        if n.startswith("attn") or n in ("common.cuh", "kernels.h"):
+        if n.startswith("attn") or n in ("common.cuh", "kernels.h", "sm100.cuh"):
             with open(os.path.join(csrc, n), "rb") as f:
                 h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
@@ -247,14 +247,18 @@ def _source_sha() -> str:
 
 def _ncu_traffic(workload: str):
     """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, if it was
-    taken on the current kernel source; else None."""
-    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    taken on the current kernel source; else None. The summary carries one line per workload:
+    ``traffic: workload=<name> source_sha=<sha> dram_bytes_per_launch=<bytes>``."""
+    p = os.path.join(ROOT, "profiles", "attn_sm100_small_topk56.md")
     try:
         with open(p) as f:
-            d = json.load(f)
-        e = d.get(workload)
-        if e and e.get("source_sha") == _source_sha():
-            return float(e["dram_bytes_per_launch"])
+            for line in f:
+                line = line.strip().strip("`")
+                if not line.startswith("traffic:"):
+                    continue
+                kv = dict(t.split("=", 1) for t in line[len("traffic:"):].split())
+                if kv.get("workload") == workload and kv.get("source_sha") == _source_sha():
+                    return float(kv["dram_bytes_per_launch"])
     except Exception:
         pass
     return None

@@ -15,19 +15,23 @@
 // itself whose keys are all masked.
 //
 // Roles (one persistent CTA per SM, work units = (batch, head, query tile), static round robin):
-//   warp 0      TMA producer for Q (once per unit) and the K pairs (3-stage ring)
-//   warp 1      TMEM allocation; one thread issues every tcgen05.mma and tcgen05.commit
-//   warps 2..9  softmax and epilogue, two warpgroups splitting the 64 query columns; a thread owns
-//               TMEM lane t (a key of S^T, a column d of O^T) for its warpgroup's 32 queries
-//   warp 10     TMA producer for the V pairs (2-stage ring)
+//   warp 0        TMA producer for Q (once per unit) and the K pairs (2-stage ring)
+//   warp 1        TMEM allocation; one thread issues the S^T MMA chains and their commits
+//   warps 2..17   softmax and epilogue: four warpgroups, each owning 16 of the 64 query columns; a
+//                 thread owns TMEM lane t (a key of S^T, a column d of O^T) for those 16 queries
+//   warp 18       TMA producer for the V pairs (3-stage ring: a V pair waits for its PV MMAs)
+//   warp 19       one thread issues the PV MMA chains and their commits
+// The softmax is latency-bound (short dependent chains per step, barriers, shared-memory traffic
+// that the tensor core's operand reads crowd out), so it is spread over 16 warps, four per SM
+// sub-partition; the two MMA-issuing threads let the next scores be computed while P^T waits.
 //
-// Softmax. Each softmax thread holds one key's 32 logits (its warpgroup's half of the queries). The shift subtracted before exp2 is a
+// Softmax. Each softmax thread holds one key's 16 logits. The shift subtracted before exp2 is a
 // per-query value m[q] shared through shared memory; it is only raised (a "slow step": per-query
 // maxima by warp reductions, then a rescale of O^T and of the running sums) when some logit exceeds
 // m[q] by more than kShiftSlack (log2 units). Any shift gives the same softmax; the bound keeps P
 // within [0, 2^kShiftSlack] so nothing overflows. The first step of a unit is always slow. Each
 // thread keeps running sums of P for its own key over all steps; they are reduced across the 128
-// threads once per unit.
+// threads of its warpgroup once per unit.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA records T3D_DEV_TIMEOUT, stops issuing work,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
@@ -41,8 +45,8 @@ using namespace sm100;
 
 constexpr int kD = 128;             // head dimension handled by this kernel
 constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a row
-constexpr int kKStages = 3;         // K-pair ring depth
-constexpr int kVStages = 2;         // V-pair ring depth
+constexpr int kKStages = 2;         // K-pair ring depth
+constexpr int kVStages = 3;         // V-pair ring depth (V waits longer: until its PV MMAs)
 constexpr int kQW = 16;             // query columns per softmax warpgroup
 constexpr int kWGs = 64 / kQW;      // softmax warpgroups
 constexpr int kSoftmaxThreads = 128;
@@ -50,9 +54,10 @@ constexpr int kSoftmaxBar = 1;      // named barrier ids 1 .. kWGs: one per soft
 constexpr int kSoftmaxWarps = 4 * kWGs;
 constexpr int kThreads = 32 * (kSoftmaxWarps + 4);  // + Q/K producer, two MMA issuers, V producer
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;       // S^T buffers: columns [0, 64) and [64, 128)
-constexpr uint32_t kColO = 128;     // O^T: columns [128, 192)
+constexpr int kSBufs = 2;           // S^T buffers in TMEM
+constexpr uint32_t kColS = 0;       // S^T buffer b: columns [64 b, 64 b + 64)
+constexpr uint32_t kColO = 64 * kSBufs;  // O^T: 64 columns after the S^T buffers
+constexpr uint32_t kTmemCols = kColO + 64 <= 256 ? 256 : 512;
 
 constexpr uint32_t kTileBytes = 64 * 128;                  // 64 rows x 128 B (one half of a tile)
 constexpr uint32_t kQBytes = kHalves * kTileBytes;         // 16 KB
@@ -67,7 +72,7 @@ struct alignas(1024) SmemLayout {
   uint64_t q_full, q_empty, o_full, o_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[kSBufs], s_empty[kSBufs];
   uint64_t p_full[2], p_empty[2];
   uint64_t drain;
   uint64_t wg_sync;  // rendezvous of both softmax warpgroups (bounded, unlike bar.sync)
@@ -140,10 +145,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < kKStages; ++t) { mbar_init(&s.k_full[t], 1); mbar_init(&s.k_empty[t], 1); }
     for (int t = 0; t < kVStages; ++t) { mbar_init(&s.v_full[t], 1); mbar_init(&s.v_empty[t], 1); }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.s_empty[t], kWGs * kSoftmaxThreads);
       mbar_init(&s.p_full[t], kWGs * kSoftmaxThreads);
       mbar_init(&s.p_empty[t], 1);
+    }
+    for (int t = 0; t < kSBufs; ++t) {
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.s_empty[t], kWGs * kSoftmaxThreads);
     }
     mbar_init(&s.drain, 2);  // one commit from each MMA-issuing thread
     mbar_init(&s.wg_sync, kWGs * kSoftmaxThreads);
@@ -214,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int n = 0; n < ui.npairs; ++n) {
           const long gp = gp0 + n;
-          const int vs = (int)(gp & 1);
-          if (!mbar_wait(&s.v_empty[vs], ((gp >> 1) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          const int vs = (int)(gp % kVStages);
+          if (!mbar_wait(&s.v_empty[vs], ((gp / kVStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
           int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
           if (ja < 0) ja = 0;
           if (jb < 0) jb = ja;
@@ -232,7 +239,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         gp0 += ui.npairs;
       }
       for (long gp = issued - kVStages; gp < issued; ++gp)
-        if (gp >= 0) mbar_wait(&s.v_full[gp & 1], (gp >> 1) & 1, nullptr);
+        if (gp >= 0) mbar_wait(&s.v_full[gp % kVStages], (gp / kVStages) & 1, nullptr);
     }
   } else if (warp == 1 || warp == 3 + kSoftmaxWarps) {
     // ------------------------------------------------------------- MMA issuers
@@ -259,9 +266,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int n = 0; n < ui.npairs && ok; ++n) {
             const long gp = gp0 + n;
             const int ks = (int)(gp % kKStages);
-            const int sb = (int)(gp & 1);
+            const int sb = (int)(gp % kSBufs);
             if (!mbar_wait(&s.k_full[ks], (gp / kKStages) & 1, abort_flag) ||
-                !mbar_wait(&s.s_empty[sb], ((gp >> 1) & 1) ^ 1, abort_flag)) {
+                !mbar_wait(&s.s_empty[sb], ((gp / kSBufs) & 1) ^ 1, abort_flag)) {
               ok = false;
               break;
             }
@@ -283,22 +290,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int n = 0; n < ui.npairs && ok; ++n) {
             const long gp = gp0 + n;
             const bool first = n == 0;
-            const int vs = (int)(gp & 1);
-            const uint32_t ph = (uint32_t)((gp >> 1) & 1);
+            const int vs = (int)(gp % kVStages);
+            const int pb = (int)(gp & 1);  // P^T buffer
             if ((first && !mbar_wait(&s.o_empty, (active & 1) ^ 1, abort_flag)) ||
-                !mbar_wait(&s.v_full[vs], ph, abort_flag) ||
-                !mbar_wait(&s.p_full[vs], ph, abort_flag)) {
+                !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
+                !mbar_wait(&s.p_full[pb], (uint32_t)((gp >> 1) & 1), abort_flag)) {
               ok = false;
               break;
             }
             tc_fence_after();
             const uint64_t da0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
-            const uint64_t db0 = dp + (uint64_t)(vs * (kPBytes >> 4));
+            const uint64_t db0 = dp + (uint64_t)(pb * (kPBytes >> 4));
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V^T and of P^T) per MMA
               mma_bf16(tmem + kColO, da0 + kk * (2048 >> 4), db0 + kk * (2048 >> 4), idesc_o,
                        (first && kk == 0) ? 0u : 1u);
-            mma_commit(&s.p_empty[vs]);
+            mma_commit(&s.p_empty[pb]);
             mma_commit(&s.v_empty[vs]);
           }
           if (ok) mma_commit(&s.o_full);
@@ -362,14 +369,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool failed = false;
       for (int n = 0; n < ui.npairs; ++n) {
         const long gp = gp0 + n;
-        const int sb = (int)(gp & 1);
+        const int sb = (int)(gp % kSBufs);  // S^T buffer
+        const int pb = (int)(gp & 1);       // P^T buffer
         const uint32_t ph = (uint32_t)((gp >> 1) & 1);
         const int raw = raw_next;
         const int e_next = 2 * (n + 1) + (r >> 6);
         raw_next = (e_next < ui.cnt) ? ui.list[e_next] : kAbsent;
         // S^T of this step, and P^T buffer sb free again (its PV MMAs of step gp - 2 complete).
-        bool ok = mbar_wait(&s.s_full[sb], ph, abort_flag);
-        ok = ok && mbar_wait(&s.p_empty[sb], ph ^ 1, abort_flag);
+        bool ok = mbar_wait(&s.s_full[sb], (uint32_t)((gp / kSBufs) & 1), abort_flag);
+        ok = ok && mbar_wait(&s.p_empty[pb], ph ^ 1, abort_flag);
         tc_fence_after();
         float x[kQW];
         {
@@ -444,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // P = exp2(x - shift), running sums, bf16 into this row of P^T (MN-major, 128B swizzle:
         // 16-byte chunk c of row r lives at chunk c ^ (r & 7); this warpgroup owns kQW / 8 chunks).
-        uint8_t* prow = s.p[sb] + r * 128;
+        uint8_t* prow = s.p[pb] + r * 128;
 #pragma unroll
         for (int c = 0; c < kQW / 8; ++c) {
           uint32_t w[4];
@@ -466,7 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               make_uint4(w[0], w[1], w[2], w[3]);
         }
         fence_proxy_async();
-        mbar_arrive(&s.p_full[sb]);
+        mbar_arrive(&s.p_full[pb]);
       }
       if (failed) break;
       // ---- epilogue: denominators (reduce the 128 per-key partial sums of each query)

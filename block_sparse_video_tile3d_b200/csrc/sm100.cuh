@@ -208,17 +208,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// Per-warpgroup register reallocation: every warp of a warpgroup executes the same call, and the
-// registers given to the growing warpgroups never exceed those released plus the launch allocation.
-template <int kRegs>
-__device__ __forceinline__ void setmaxnreg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-template <int kRegs>
-__device__ __forceinline__ void setmaxnreg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-
 __device__ __forceinline__ float redux_max(float v) {
   float r;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
