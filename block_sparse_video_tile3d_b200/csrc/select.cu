@@ -14,45 +14,42 @@ namespace t3d {
 namespace {
 
 constexpr int kSelThreads = 256;  // 8 warps
-constexpr int kKeyChunk = 64;     // pooled key rows staged in shared memory at a time
-constexpr int kPad = 4;           // row padding (floats): rows 16 B apart modulo 128 B
+constexpr int kKeyChunk = 128;    // pooled key rows staged in shared memory at a time (one per thread pair)
+constexpr int kPad = 4;           // key row padding (floats): consecutive rows 4 banks apart
 
-// Query tiles per CTA: 16 (two per warp, enough CTAs to fill the GPU), or 8 when 16 score rows
-// would not fit next to the staged operands (~200 KB of shared memory).
-__host__ __device__ inline int sel_rows(int D, int nT) {
-  return ((size_t)(16 + kKeyChunk) * (D + kPad) * 4 + (size_t)16 * nT * 4 + 8 * 1024 <= 200 * 1024)
-             ? 16 : 8;
-}
-
-// Shared memory (floats): pq rows [R][D+4], a key chunk [64][D+4], the R score rows [R][nT], then
-// one 256-bin histogram per warp.
+// Query tiles per CTA: 16 (two CTAs per SM for the common sizes), or 8 when 16 score rows would not
+// fit next to the staged operands (~200 KB of shared memory).
 __host__ __device__ inline size_t sel_smem_floats(int D, int nT, int R) {
-  return (size_t)(R + kKeyChunk) * (D + kPad) + (size_t)R * nT + 8 * 256;
+  return (size_t)R * D + (size_t)kKeyChunk * (D + kPad) + (size_t)R * nT + 8 * 256;
+}
+__host__ __device__ inline int sel_rows(int D, int nT) {
+  return sel_smem_floats(D, nT, 16) * 4 <= 200 * 1024 ? 16 : 8;
 }
 
-// Scores S[i, j] = pq_i . pk_j in fp32 (accumulated over d in order, four at a time) for the CTA's
-// R query tiles i0 .. i0 + R - 1; row r lands in vals[r * nT + j]. Register blocking: thread
-// (row group, key group) computes RT rows x 4 keys of each 64-key chunk, keys kg + 16 j so that
-// the lanes of a quarter warp read consecutive padded rows (no bank conflicts).
-template <int RT>
+// Scores S[i, j] = pq_i . pk_j in fp32 (fused multiply-adds over d in order) for the CTA's R query
+// tiles i0 .. i0 + R - 1; row r lands in vals[r * nT + j]. Shared memory (floats): pq rows [R][D],
+// a key chunk [128][D + 4], the score rows [R][nT], then the per-warp histograms of the radix
+// select. Thread t owns key j0 + (t mod 128) of each chunk and the R / 2 rows of half t / 128: its
+// key row is one conflict-free 16-byte load per four d, the query rows are warp-wide broadcasts.
+template <int RH>
 __device__ void compute_scores(const Geo& g, const float* __restrict__ pq,
-                               const float* __restrict__ pk, long bh, int i0, int R, float* sm) {
-  const int D = g.D, nT = g.nT, ldp = D + kPad;
+                               const float* __restrict__ pk, long bh, int i0, float* sm) {
+  constexpr int R = 2 * RH;
+  const int D = g.D, nT = g.nT, ldk = D + kPad, d4 = D / 4;
   float* pq_s = sm;
-  float* pk_s = pq_s + R * ldp;
-  float* vals = pk_s + kKeyChunk * ldp;
+  float* pk_s = pq_s + R * D;
+  float* vals = pk_s + kKeyChunk * ldk;
   const int tid = threadIdx.x;
-  const int d4 = D / 4;
   for (int e = tid; e < R * d4; e += kSelThreads) {
     const int r = e / d4, c = e - r * d4;
     const int i = i0 + r;
     const float4 v = (i < nT) ? reinterpret_cast<const float4*>(pq + (bh * nT + i) * D)[c]
                               : make_float4(0.f, 0.f, 0.f, 0.f);
-    *reinterpret_cast<float4*>(pq_s + r * ldp + 4 * c) = v;
+    *reinterpret_cast<float4*>(pq_s + r * D + 4 * c) = v;
   }
   const float* pkh = pk + bh * nT * D;
-  const int rg = tid >> 4, kg = tid & 15;
-  const bool active = rg * RT < R;
+  const int kc = tid & (kKeyChunk - 1), rh = tid / kKeyChunk;
+  const float* qrow = pq_s + rh * RH * D;
   for (int j0 = 0; j0 < nT; j0 += kKeyChunk) {
     __syncthreads();
     const int rows = imin(kKeyChunk, nT - j0);
@@ -60,40 +57,27 @@ __device__ void compute_scores(const Geo& g, const float* __restrict__ pq,
       const int r = e / d4, c = e - r * d4;
       const float4 v = (r < rows) ? reinterpret_cast<const float4*>(pkh + (long)(j0 + r) * D)[c]
                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(pk_s + r * ldp + 4 * c) = v;
+      *reinterpret_cast<float4*>(pk_s + r * ldk + 4 * c) = v;
     }
     __syncthreads();
-    if (active) {
-      float acc[RT][4];
+    float acc[RH];
 #pragma unroll
-      for (int a = 0; a < RT; ++a)
+    for (int a = 0; a < RH; ++a) acc[a] = 0.f;
+    const float* krow = pk_s + kc * ldk;
+    for (int d = 0; d < D; d += 4) {
+      const float4 kb = *reinterpret_cast<const float4*>(krow + d);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) acc[a][b] = 0.f;
-      for (int d = 0; d < D; d += 4) {
-        float4 qa[RT], kb[4];
-#pragma unroll
-        for (int a = 0; a < RT; ++a)
-          qa[a] = *reinterpret_cast<const float4*>(pq_s + (rg * RT + a) * ldp + d);
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-          kb[b] = *reinterpret_cast<const float4*>(pk_s + (kg + 16 * b) * ldp + d);
-#pragma unroll
-        for (int a = 0; a < RT; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            acc[a][b] = fmaf(qa[a].x, kb[b].x, acc[a][b]);
-            acc[a][b] = fmaf(qa[a].y, kb[b].y, acc[a][b]);
-            acc[a][b] = fmaf(qa[a].z, kb[b].z, acc[a][b]);
-            acc[a][b] = fmaf(qa[a].w, kb[b].w, acc[a][b]);
-          }
+      for (int a = 0; a < RH; ++a) {
+        const float4 qa = *reinterpret_cast<const float4*>(qrow + a * D + d);
+        acc[a] = fmaf(qa.x, kb.x, acc[a]);
+        acc[a] = fmaf(qa.y, kb.y, acc[a]);
+        acc[a] = fmaf(qa.z, kb.z, acc[a]);
+        acc[a] = fmaf(qa.w, kb.w, acc[a]);
       }
+    }
+    if (kc < rows) {
 #pragma unroll
-      for (int a = 0; a < RT; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int j = kg + 16 * b;
-          if (j < rows) vals[(rg * RT + a) * nT + j0 + j] = acc[a][b];
-        }
+      for (int a = 0; a < RH; ++a) vals[(rh * RH + a) * nT + j0 + kc] = acc[a];
     }
   }
   __syncthreads();
@@ -101,9 +85,52 @@ __device__ void compute_scores(const Geo& g, const float* __restrict__ pq,
 
 __device__ void compute_scores_any(const Geo& g, const float* pq, const float* pk, long bh, int i0,
                                    int R, float* sm) {
-  if (R >= 64) compute_scores<4>(g, pq, pk, bh, i0, R, sm);
-  else if (R == 32) compute_scores<2>(g, pq, pk, bh, i0, R, sm);
-  else compute_scores<1>(g, pq, pk, bh, i0, R, sm);
+  if (R == 16) compute_scores<8>(g, pq, pk, bh, i0, sm);
+  else compute_scores<4>(g, pq, pk, bh, i0, sm);
+}
+
+// Top-k of a row of at most 32 * KPL values held in registers (lane l owns entries l + 32 i):
+// the k-th largest order-preserving key is found bit by bit from the top (largest T with at least k
+// keys >= T), then every key above it and the first (by index) ties at it are emitted in
+// ascending index order. Same result as the radix select below; no shared-memory histograms.
+template <int KPL>
+__device__ int select_topk_row_reg(const float* row, int n, int k, int32_t* out) {
+  k = imin(k, n);
+  if (k <= 0) return 0;
+  const int lane = threadIdx.x & 31;
+  uint32_t key[KPL];
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int j = lane + 32 * i;
+    key[i] = j < n ? float_key(row[j]) : 0u;  // 0 ranks below every float's key
+  }
+  uint32_t thr = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = thr | (1u << bit);
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) c += key[i] >= cand ? 1 : 0;
+    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) thr = cand;
+  }
+  int gt = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) gt += key[i] > thr ? 1 : 0;
+  const int need_eq = k - (int)__reduce_add_sync(0xffffffffu, (unsigned)gt);
+  const unsigned lt = lanemask_lt();
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int j = lane + 32 * i;
+    const bool eq = j < n && key[i] == thr;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool sel = (j < n && key[i] > thr) || (eq && eq_seen + __popc(eqb & lt) < need_eq);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    const int pos = written + __popc(sb & lt);
+    if (sel && pos < k) out[pos] = j;
+    written += __popc(sb);
+    eq_seen += __popc(eqb);
+  }
+  return k;
 }
 
 // Key of the k-th largest value of row[0..n) (1 <= k <= n): radix select on the order-preserving
@@ -217,13 +244,19 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(Geo g, const float* _
   const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * R;
   compute_scores_any(g, pq, pk, bh, i0, R, sm);
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* vals = sm + (R + kKeyChunk) * (g.D + kPad);
-  int* hist = reinterpret_cast<int*>(sm + (R + kKeyChunk) * (g.D + kPad) + R * nT) + w * 256;
+  const float* vals = sm + R * g.D + kKeyChunk * (g.D + kPad);
+  int* hist = reinterpret_cast<int*>(const_cast<float*>(vals) + R * nT) + w * 256;
   const int kk = imin(k, nT);
   for (int r = w; r < R; r += kSelThreads / 32) {
     const int i = i0 + r;
     if (i >= nT) break;
-    const int n = select_topk_row(vals + r * nT, nT, kk, kv_idx + (bh * nT + i) * kk, hist);
+    const float* row = vals + r * nT;
+    int32_t* out = kv_idx + (bh * nT + i) * kk;
+    int n;
+    if (nT <= 128) n = select_topk_row_reg<4>(row, nT, kk, out);
+    else if (nT <= 256) n = select_topk_row_reg<8>(row, nT, kk, out);
+    else if (nT <= 512) n = select_topk_row_reg<16>(row, nT, kk, out);
+    else n = select_topk_row(row, nT, kk, out, hist);
     if (lane == 0) kv_cnt[bh * nT + i] = n;
   }
 }
@@ -314,7 +347,7 @@ __global__ void __launch_bounds__(kSelThreads) mass_kernel(Geo g, const float* _
   const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * R;
   compute_scores_any(g, pq, pk, bh, i0, R, sm);
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* vals = sm + (R + kKeyChunk) * (g.D + kPad);
+  float* vals = sm + R * g.D + kKeyChunk * (g.D + kPad);
   int* hist = reinterpret_cast<int*>(vals + R * nT) + w * 256;
   for (int r = w; r < R; r += kSelThreads / 32) {
     const int i = i0 + r;
