@@ -6,32 +6,35 @@
 // one KV head per query head, softmax scale 1/sqrt(D), tile-ordered [B, L, heads, D] bf16 tensors,
 // sparse attention per kept block pair, pruned query rows reconstructed afterwards.
 //
-// Shape of the computation. A query tile has 64 rows, and a tcgen05 MMA with M = 64 costs as much
-// as one with M = 128, so the kernel puts KEYS on the M dimension: each step takes a PAIR of kept key
-// tiles (128 keys) and computes
-//     S^T[128 keys, 64 queries]  = K_pair . Q^T          (A = K pair, K-major; B = Q, K-major)
-//     O^T[D, 64 queries]        += V_pair^T . P^T        (A = V pair, MN-major; B = P^T, MN-major)
-// both with M = 128, N = 64, accumulating in fp32 in TMEM. An odd last tile is paired with a copy of
-// itself whose keys are all masked.
+// Shape of the computation. A work unit is one (batch, head, query tile): 64 query rows. Each step
+// takes a PAIR of its kept key tiles (128 keys; an odd last tile is paired with a fully masked copy
+// of itself) and computes, with M = 64 query rows,
+//     S[64 q, 128 keys]  = Q . K_pair^T      (A = Q in TMEM, B = K pair in shared memory, K-major)
+//     O[64 q, D]        += P . V_pair         (A = P in TMEM, B = V pair in shared memory, MN-major)
+// fp32 accumulation in TMEM. Q and P live in TMEM, so the only shared-memory operands are the K and
+// V tiles: the tensor core's operand reads (which at N = 64 took the whole shared-memory bandwidth)
+// no longer compete with P^T or with re-reads of Q.
 //
-// Roles (one persistent CTA per SM, work units = (batch, head, query tile), static round robin):
-//   warp 0        TMA producer for Q (once per unit) and the K pairs (2-stage ring)
-//   warp 1        TMEM allocation; one thread issues the S^T MMA chains and their commits
-//   warps 2..17   softmax and epilogue: four warpgroups, each owning 16 of the 64 query columns; a
-//                 thread owns TMEM lane t (a key of S^T, a column d of O^T) for those 16 queries
-//   warp 18       TMA producer for the V pairs (3-stage ring: a V pair waits for its PV MMAs)
-//   warp 19       one thread issues the PV MMA chains and their commits
-// The softmax is latency-bound (short dependent chains per step, barriers, shared-memory traffic
-// that the tensor core's operand reads crowd out), so it is spread over 16 warps, four per SM
-// sub-partition; the two MMA-issuing threads let the next scores be computed while P^T waits.
+// TMEM (512 columns; an M = 64 tile occupies lanes 0..15 of each 32-lane sub-partition):
+//   S buffer b: columns 128 b .. 128 b + 127 (fp32)    O: 256 .. 383 (fp32)
+//   P: 384 .. 447 (bf16 pairs: column c holds keys 2c, 2c + 1)   Q: 448 .. 511 (bf16 pairs of d)
 //
-// Softmax. Each softmax thread holds one key's 16 logits. The shift subtracted before exp2 is a
-// per-query value m[q] shared through shared memory; it is only raised (a "slow step": per-query
-// maxima by warp reductions, then a rescale of O^T and of the running sums) when some logit exceeds
-// m[q] by more than kShiftSlack (log2 units). Any shift gives the same softmax; the bound keeps P
-// within [0, 2^kShiftSlack] so nothing overflows. The first step of a unit is always slow. Each
-// thread keeps running sums of P for its own key over all steps; they are reduced across the 128
-// threads of its warpgroup once per unit.
+// Roles (one persistent CTA per SM, 8 warps, units in static round robin, head-major):
+//   warp 0      TMA producer for the K pairs (3-stage ring)
+//   warp 1      TMEM allocation; one thread issues every tcgen05.mma and tcgen05.commit
+//   warp 2      TMA producer for the V pairs (3-stage ring)
+//   warps 4..7  softmax and epilogue: thread t of warp w owns query rows 16 (w - 4) + t/4 and that
+//               + 8, and the key columns 8j + 2(t%4) + {0, 1} of each step (tcgen05.ld 16x256b); it
+//               also writes the unit's Q into TMEM.
+// MMA order: S(0), S(1), then per step n: S(n + 2) (same unit only), PV(n); the next unit's first
+// two S wait for its Q, which the softmax writes as soon as the current unit's last S has completed.
+//
+// Softmax. Each row's online-softmax state (shift m, running sum l) is private to the 4 threads
+// that share the row: the row maximum is two shuffles away, no barrier spans the warpgroup. The
+// shift (log2 units) is raised only when a row's logits exceed it by more than kShiftSlack — then
+// the warp rescales the O rows of its 16 queries in TMEM (factor 1 for the rows that did not move)
+// once the previous PV has landed. Any shift gives the same softmax; the bound keeps P within
+// [0, 2^kShiftSlack] so nothing overflows.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA records T3D_DEV_TIMEOUT, stops issuing work,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
@@ -45,44 +48,34 @@ using namespace sm100;
 
 constexpr int kD = 128;             // head dimension handled by this kernel
 constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a row
-constexpr int kKStages = 2;         // K-pair ring depth
-constexpr int kVStages = 3;         // V-pair ring depth (V waits longer: until its PV MMAs)
-constexpr int kQW = 16;             // query columns per softmax warpgroup
-constexpr int kWGs = 64 / kQW;      // softmax warpgroups
+constexpr int kKStages = 3;         // K-pair ring depth
+constexpr int kVStages = 3;         // V-pair ring depth
+constexpr int kThreads = 256;       // 8 warps: producers / MMA, softmax warpgroup
 constexpr int kSoftmaxThreads = 128;
-constexpr int kSoftmaxBar = 1;      // named barrier ids 1 .. kWGs: one per softmax warpgroup
-constexpr int kSoftmaxWarps = 4 * kWGs;
-constexpr int kThreads = 32 * (kSoftmaxWarps + 4);  // + Q/K producer, two MMA issuers, V producer
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
-constexpr int kSBufs = 2;           // S^T buffers in TMEM
-constexpr uint32_t kColS = 0;       // S^T buffer b: columns [64 b, 64 b + 64)
-constexpr uint32_t kColO = 64 * kSBufs;  // O^T: 64 columns after the S^T buffers
-constexpr uint32_t kTmemCols = kColO + 64 <= 256 ? 256 : 512;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;       // S buffer b at 128 b
+constexpr uint32_t kColO = 256;
+constexpr uint32_t kColP = 384;
+constexpr uint32_t kColQ = 448;
 
 constexpr uint32_t kTileBytes = 64 * 128;                  // 64 rows x 128 B (one half of a tile)
-constexpr uint32_t kQBytes = kHalves * kTileBytes;         // 16 KB
 constexpr uint32_t kPairBytes = kHalves * 2 * kTileBytes;  // 32 KB: two tiles, both halves
-constexpr uint32_t kPBytes = 128 * 128;                    // P^T: 128 keys x 64 queries bf16
 
 struct alignas(1024) SmemLayout {
-  uint8_t q[kQBytes];
   uint8_t k[kKStages][kPairBytes];
   uint8_t v[kVStages][kPairBytes];
-  uint8_t p[2][kPBytes];
-  uint64_t q_full, q_empty, o_full, o_empty;
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[kSBufs], s_empty[kSBufs];
-  uint64_t p_full[2], p_empty[2];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full;    // P of the step written to TMEM (softmax -> MMA)
+  uint64_t pv_done;   // the step's PV MMAs complete: P free, O current (MMA -> softmax)
+  uint64_t q_ready;   // the unit's Q written to TMEM (softmax -> MMA)
+  uint64_t q_free;    // the unit's last S MMA complete: Q may be overwritten (MMA -> softmax)
+  uint64_t o_full;    // the unit's last PV complete (MMA -> softmax)
+  uint64_t o_empty;   // O read by the epilogue (softmax -> MMA)
   uint64_t drain;
-  uint64_t wg_sync;  // rendezvous of both softmax warpgroups (bounded, unlike bar.sync)
-  alignas(16) float shift[64];   // current per-query shift (log2 units)
-  alignas(16) float thr[64];     // raw logit above which a step is slow: (shift + slack) / scale
-  alignas(16) float nsh[64];     // -shift, or 0 while the shift is -inf
-  alignas(16) float red[4][64];  // per-warp partial results
-  alignas(16) float alpha[64];   // rescale factors of a slow step
-  alignas(16) float lsum[64];    // per-query softmax denominators
-  uint8_t vc[kMaxTiles];         // valid token count of every tile
+  uint8_t vc[kMaxTiles];  // valid token count of every tile
   uint32_t tmem_base;
   int abort;
 };
@@ -90,8 +83,8 @@ struct alignas(1024) SmemLayout {
 static_assert(sizeof(SmemLayout) + 1024 <= 232448, "shared memory per CTA");
 constexpr int kAbsent = -0x7fffffff - 1;  // list entry beyond kv_cnt
 
-constexpr uint32_t idesc_s = idesc_bf16(128, 64, false, false);
-constexpr uint32_t idesc_o = idesc_bf16(128, 64, true, true);
+constexpr uint32_t idesc_s = idesc_bf16(64, 128, false, false);  // A = Q (TMEM), B = K, K-major
+constexpr uint32_t idesc_o = idesc_bf16(64, 128, false, true);   // A = P (TMEM), B = V, MN-major
 
 struct UnitInfo {
   int b, h, i, cnt, npairs;
@@ -125,8 +118,46 @@ __device__ __forceinline__ void fail(SmemLayout& s, int32_t* status) {
 }
 
 struct Maps {
-  CUtensorMap q, k, v;
+  CUtensorMap k, v;
 };
+
+// Streams the kept key (or value) tile pairs of every unit of this CTA, in step order, into a ring
+// of kStages pair buffers (lane 0 of a producer warp).
+template <int kStages>
+__device__ __forceinline__ void produce_pairs(SmemLayout& s, const Geo& g, const AttnArgs& a,
+                                              const CUtensorMap* map, uint8_t (*ring)[kPairBytes],
+                                              uint64_t* full, uint64_t* empty,
+                                              volatile int* abort_flag) {
+  const int total_units = g.B * g.heads * g.nT;
+  long gp0 = 0, issued = 0;
+  bool ok = true;
+  for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
+    const UnitInfo ui = unit_info(g, a, u);
+    for (int n = 0; n < ui.npairs; ++n) {
+      const long gp = gp0 + n;
+      const int st = (int)(gp % kStages);
+      if (!mbar_wait(&empty[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag)) {
+        ok = false;
+        break;
+      }
+      int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
+      if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
+      if (jb < 0) jb = ja;
+      mbar_expect_tx(&full[st], kPairBytes);
+      for (int hh = 0; hh < kHalves; ++hh) {
+        uint8_t* dst = ring[st] + hh * 2 * kTileBytes;
+        tma_load_3d(dst, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
+        tma_load_3d(dst + kTileBytes, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + jb * kTileElems);
+      }
+      ++issued;
+    }
+    gp0 += ui.npairs;
+  }
+  if (!ok) fail(s, a.dev_status);
+  // Drain: the last loads issued must land before the CTA can exit.
+  for (long gp = issued - kStages; gp < issued; ++gp)
+    if (gp >= 0) mbar_wait(&full[gp % kStages], (uint32_t)((gp / kStages) & 1), nullptr);
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ Maps maps, Geo g, AttnArgs a, float sl2) {
@@ -138,28 +169,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &s.abort;
 
   if (threadIdx.x == 0) {
-    mbar_init(&s.q_full, 1);
-    mbar_init(&s.q_empty, 1);
-    mbar_init(&s.o_full, 1);
-    mbar_init(&s.o_empty, kWGs * kSoftmaxThreads);
     for (int t = 0; t < kKStages; ++t) { mbar_init(&s.k_full[t], 1); mbar_init(&s.k_empty[t], 1); }
     for (int t = 0; t < kVStages; ++t) { mbar_init(&s.v_full[t], 1); mbar_init(&s.v_empty[t], 1); }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&s.p_full[t], kWGs * kSoftmaxThreads);
-      mbar_init(&s.p_empty[t], 1);
-    }
-    for (int t = 0; t < kSBufs; ++t) {
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.s_empty[t], kWGs * kSoftmaxThreads);
+      mbar_init(&s.s_empty[t], kSoftmaxThreads);
     }
-    mbar_init(&s.drain, 2);  // one commit from each MMA-issuing thread
-    mbar_init(&s.wg_sync, kWGs * kSoftmaxThreads);
+    mbar_init(&s.p_full, kSoftmaxThreads);
+    mbar_init(&s.pv_done, 1);
+    mbar_init(&s.q_ready, kSoftmaxThreads);
+    mbar_init(&s.q_free, 1);
+    mbar_init(&s.o_full, 1);
+    mbar_init(&s.o_empty, kSoftmaxThreads);
+    mbar_init(&s.drain, 1);
     s.abort = 0;
     fence_mbar_init();
   }
   for (int t = threadIdx.x; t < g.nT; t += kThreads) s.vc[t] = (uint8_t)tile_valid_count(g, t);
   if (warp == 0 && lane == 0) {
-    tma_prefetch(&maps.q);
     tma_prefetch(&maps.k);
     tma_prefetch(&maps.v);
   }
@@ -173,145 +200,75 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------- Q and K producer
-    if (lane == 0) {
-      int active = 0;
-      long gp0 = 0;
-      long issued = 0;  // K pairs issued
-      for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
-        const UnitInfo ui = unit_info(g, a, u);
-        if (ui.npairs == 0) continue;
-        if (!mbar_wait(&s.q_empty, (active & 1) ^ 1, abort_flag)) { fail(s, a.dev_status); break; }
-        const int row0 = ui.b * g.Lp + ui.i * kTileElems;
-        mbar_expect_tx(&s.q_full, kQBytes);
-        for (int hh = 0; hh < kHalves; ++hh)
-          tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
-        bool ok = true;
-        for (int n = 0; n < ui.npairs; ++n) {
-          const long gp = gp0 + n;
-          const int ks = (int)(gp % kKStages);
-          if (!mbar_wait(&s.k_empty[ks], ((gp / kKStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
-          if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
-          if (jb < 0) jb = ja;
-          mbar_expect_tx(&s.k_full[ks], kPairBytes);
-          for (int hh = 0; hh < kHalves; ++hh) {
-            uint8_t* dst = s.k[ks] + hh * 2 * kTileBytes;
-            tma_load_3d(dst, &maps.k, &s.k_full[ks], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
-            tma_load_3d(dst + kTileBytes, &maps.k, &s.k_full[ks], 64 * hh, ui.h,
-                        ui.b * g.Lp + jb * kTileElems);
-          }
-          ++issued;
-        }
-        if (!ok) { fail(s, a.dev_status); break; }
-        gp0 += ui.npairs;
-        ++active;
-      }
-      // Drain: the last loads issued must land before the CTA can exit.
-      for (long gp = issued - kKStages; gp < issued; ++gp)
-        if (gp >= 0) mbar_wait(&s.k_full[gp % kKStages], (gp / kKStages) & 1, nullptr);
-    }
-  } else if (warp == 2 + kSoftmaxWarps) {
+    // ------------------------------------------------------------- K producer
+    if (lane == 0) produce_pairs<kKStages>(s, g, a, &maps.k, s.k, s.k_full, s.k_empty, abort_flag);
+  } else if (warp == 2) {
     // ------------------------------------------------------------- V producer
+    if (lane == 0) produce_pairs<kVStages>(s, g, a, &maps.v, s.v, s.v_full, s.v_empty, abort_flag);
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
-      long gp0 = 0, issued = 0;
-      for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
-        const UnitInfo ui = unit_info(g, a, u);
-        if (ui.npairs == 0) continue;
-        bool ok = true;
-        for (int n = 0; n < ui.npairs; ++n) {
-          const long gp = gp0 + n;
-          const int vs = (int)(gp % kVStages);
-          if (!mbar_wait(&s.v_empty[vs], ((gp / kVStages) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
-          if (ja < 0) ja = 0;
-          if (jb < 0) jb = ja;
-          mbar_expect_tx(&s.v_full[vs], kPairBytes);
-          for (int hh = 0; hh < kHalves; ++hh) {
-            uint8_t* dst = s.v[vs] + hh * 2 * kTileBytes;
-            tma_load_3d(dst, &maps.v, &s.v_full[vs], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
-            tma_load_3d(dst + kTileBytes, &maps.v, &s.v_full[vs], 64 * hh, ui.h,
-                        ui.b * g.Lp + jb * kTileElems);
-          }
-          ++issued;
-        }
-        if (!ok) { fail(s, a.dev_status); break; }
-        gp0 += ui.npairs;
-      }
-      for (long gp = issued - kVStages; gp < issued; ++gp)
-        if (gp >= 0) mbar_wait(&s.v_full[gp % kVStages], (gp / kVStages) & 1, nullptr);
-    }
-  } else if (warp == 1 || warp == 3 + kSoftmaxWarps) {
-    // ------------------------------------------------------------- MMA issuers
-    // Two threads issue the MMAs: warp 1 the S^T chains, warp 11 the PV chains. Each waits only on
-    // what its own chains read, so a late P^T never holds back the next scores (and vice versa);
-    // each commit tracks the MMAs of the thread that issues it.
-    if (lane == 0) {
-      int active = 0;
-      long gp0 = 0;
+      int active = 0;  // units with at least one pair, in order
+      long gp0 = 0;    // global step index of the unit's first pair
       bool ok = true;
       // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4 and
-      // every buffer lies below 256 KB), so each MMA's operands are a base descriptor plus a
-      // constant: the issuing thread builds none of them in the loop.
-      const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
+      // every buffer lies below 256 KB), so each MMA's operand is a base descriptor plus a constant.
       const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
       const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
-      const uint64_t dp = sdesc_sw128(smem_u32(s.p[0]), kPBytes, 1024);
-      const bool s_issuer = warp == 1;
+      // S(gp) = Q . K_pair^T into S buffer gp & 1.
+      auto issue_s = [&](long gp, bool last_of_unit) -> bool {
+        const int ks = (int)(gp % kKStages);
+        const int b = (int)(gp & 1);
+        if (!mbar_wait(&s.k_full[ks], (uint32_t)((gp / kKStages) & 1), abort_flag) ||
+            !mbar_wait(&s.s_empty[b], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag))
+          return false;
+        tc_fence_after();
+        const uint64_t db0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
+        const uint32_t d_s = tmem + kColS + 128 * b;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
+          const int hh = kk >> 2, st = kk & 3;
+          mma_bf16_ts(d_s, tmem + kColQ + 8 * kk,
+                      db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
+        }
+        mma_commit(&s.s_full[b]);
+        mma_commit(&s.k_empty[ks]);
+        if (last_of_unit) mma_commit(&s.q_free);
+        return true;
+      };
+      // O (+)= P . V_pair of step gp.
+      auto issue_pv = [&](long gp, bool first_of_unit, bool last_of_unit) -> bool {
+        const int vs = (int)(gp % kVStages);
+        if ((first_of_unit && !mbar_wait(&s.o_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) ||
+            !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
+            !mbar_wait(&s.p_full, (uint32_t)(gp & 1), abort_flag))
+          return false;
+        tc_fence_after();
+        const uint64_t db0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V) per MMA
+          mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, db0 + kk * (2048 >> 4), idesc_o,
+                      (first_of_unit && kk == 0) ? 0u : 1u);
+        mma_commit(&s.pv_done);
+        mma_commit(&s.v_empty[vs]);
+        if (last_of_unit) mma_commit(&s.o_full);
+        return true;
+      };
       for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
         const UnitInfo ui = unit_info(g, a, u);
-        if (ui.npairs == 0) continue;
-        if (s_issuer) {
-          if (!mbar_wait(&s.q_full, active & 1, abort_flag)) { ok = false; break; }
-          for (int n = 0; n < ui.npairs && ok; ++n) {
-            const long gp = gp0 + n;
-            const int ks = (int)(gp % kKStages);
-            const int sb = (int)(gp % kSBufs);
-            if (!mbar_wait(&s.k_full[ks], (gp / kKStages) & 1, abort_flag) ||
-                !mbar_wait(&s.s_empty[sb], ((gp / kSBufs) & 1) ^ 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t da0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
-            const uint32_t d_s = tmem + kColS + sb * 64;
-#pragma unroll
-            for (int hh = 0; hh < kHalves; ++hh) {
-#pragma unroll
-              for (int st = 0; st < 4; ++st)  // 16 elements of D (32 bytes) per MMA
-                mma_bf16(d_s, da0 + ((hh * 2 * kTileBytes + st * 32) >> 4),
-                         dq + ((hh * kTileBytes + st * 32) >> 4), idesc_s, (hh | st) ? 1u : 0u);
-            }
-            mma_commit(&s.s_full[sb]);
-            mma_commit(&s.k_empty[ks]);
-            if (n == ui.npairs - 1) mma_commit(&s.q_empty);
-          }
-        } else {
-          for (int n = 0; n < ui.npairs && ok; ++n) {
-            const long gp = gp0 + n;
-            const bool first = n == 0;
-            const int vs = (int)(gp % kVStages);
-            const int pb = (int)(gp & 1);  // P^T buffer
-            if ((first && !mbar_wait(&s.o_empty, (active & 1) ^ 1, abort_flag)) ||
-                !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
-                !mbar_wait(&s.p_full[pb], (uint32_t)((gp >> 1) & 1), abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint64_t da0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
-            const uint64_t db0 = dp + (uint64_t)(pb * (kPBytes >> 4));
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V^T and of P^T) per MMA
-              mma_bf16(tmem + kColO, da0 + kk * (2048 >> 4), db0 + kk * (2048 >> 4), idesc_o,
-                       (first && kk == 0) ? 0u : 1u);
-            mma_commit(&s.p_empty[pb]);
-            mma_commit(&s.v_empty[vs]);
-          }
-          if (ok) mma_commit(&s.o_full);
+        const int np = ui.npairs;
+        if (np == 0) continue;
+        if (!mbar_wait(&s.q_ready, (uint32_t)(active & 1), abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        ok = issue_s(gp0, np == 1) && (np < 2 || issue_s(gp0 + 1, np == 2));
+        for (int n = 0; n < np && ok; ++n) {
+          // S(n + 2) only needs step n's S buffer, which the softmax frees as soon as it has read
+          // it, so it goes ahead of PV(n), which waits for the whole of step n's softmax.
+          if (n + 2 < np) ok = issue_s(gp0 + n + 2, n + 2 == np - 1);
+          if (ok) ok = issue_pv(gp0 + n, n == 0, n == np - 1);
         }
         if (!ok) break;
-        gp0 += ui.npairs;
+        gp0 += np;
         ++active;
       }
       if (!ok) fail(s, a.dev_status);
@@ -319,223 +276,247 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&s.drain);
       mbar_wait(&s.drain, 0, nullptr);
     }
-  } else {
-    // ------------------------------------------------------------- softmax + epilogue
-    // kWGs warpgroups split the 64 query columns: warpgroup wg owns columns [kQW wg, kQW wg + kQW).
-    // Within a warpgroup, warp sub-partition sp covers TMEM lanes [32 sp, 32 sp + 32).
-    const int wg = (warp - 2) >> 2;
-    const int sp = warp & 3;
-    const int r = sp * 32 + lane;       // TMEM lane: key row of S^T, column d of O^T
-    const int gt = ((warp - 2) & 3) * 32 + lane;  // 0..127 within the warpgroup
-    const int bar_id = kSoftmaxBar + wg;
-    const int q0 = wg * kQW;
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- softmax + epilogue (warps 4..7)
+    const int sp = warp & 3;            // TMEM sub-partition: lanes [32 sp, 32 sp + 32)
+    const int t0 = lane & 3;
+    const int r0 = 16 * sp + (lane >> 2), r1 = r0 + 8;  // this thread's two query rows
     const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
+    const long ld = (long)g.heads * kD;
     int active = 0;
-    long gp0 = 0;
+    long gp = 0;  // global step index
     bool reported = false;
-    uint32_t sync_phase = 0;
-    // All softmax warpgroups meet here; false if one never arrives (timeout / abort).
-    auto rendezvous = [&]() -> bool {
-      mbar_arrive(&s.wg_sync);
-      const bool r_ok = mbar_wait(&s.wg_sync, sync_phase, abort_flag);
-      sync_phase ^= 1u;
-      return r_ok;
+    bool failed = false;
+    // Writes the query tile of unit u into TMEM as the A operand of the S MMAs (row r at lane
+    // (r % 16) + 32 (r / 16); column c holds d = 2c, 2c + 1).
+    auto write_q = [&](int u) {
+      const UnitInfo ui = unit_info(g, a, u);
+      const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
+      const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + (long)ui.h * kD;
+      uint32_t w[32];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {  // d = 16 j + 4 t0 .. + 3: columns 8 j + 2 t0, + 1
+        const uint2 x0 = *reinterpret_cast<const uint2*>(qb + (row0 + r0) * ld + 16 * j + 4 * t0);
+        const uint2 x1 = *reinterpret_cast<const uint2*>(qb + (row0 + r1) * ld + 16 * j + 4 * t0);
+        w[4 * j] = x0.x; w[4 * j + 1] = x0.y; w[4 * j + 2] = x1.x; w[4 * j + 3] = x1.y;
+      }
+      tmem_st_16x256b_x8(lane_base + kColQ, w);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&s.q_ready);
     };
-    float lpart[kQW];
-    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+    // Next unit (from u) with at least one kept pair, or total_units.
+    auto next_busy = [&](int u) -> int {
+      for (; u < total_units; u += gridDim.x)
+        if (unit_info(g, a, u).npairs > 0) return u;
+      return total_units;
+    };
+    int ub = next_busy(blockIdx.x);
+    if (ub < total_units) write_q(ub);
+    for (int u = blockIdx.x; u < total_units && !failed; u += gridDim.x) {
       const UnitInfo ui = unit_info(g, a, u);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
       const int vci = s.vc[ui.i];
-      const long ld = (long)g.heads * kD;
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
       if (ui.npairs == 0) {
-        // No kept key tile: this warpgroup's output rows are zero.
-        for (int e = gt; e < kQW * kD / 8; e += kSoftmaxThreads) {
-          const int rr = q0 + e / (kD / 8), c = e % (kD / 8);
-          *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = make_uint4(0u, 0u, 0u, 0u);
+        // No kept key tile: this thread's two output rows are zero.
+        for (int c = 2 * t0; c < kD; c += 8) {
+          *reinterpret_cast<uint32_t*>(out + r0 * ld + c) = 0u;
+          *reinterpret_cast<uint32_t*>(out + r1 * ld + c) = 0u;
         }
         continue;
       }
-      if (gt < kQW) {
-        s.shift[q0 + gt] = -INFINITY;
-        s.thr[q0 + gt] = -INFINITY;
-        s.nsh[q0 + gt] = 0.f;
-      }
-#pragma unroll
-      for (int q = 0; q < kQW; ++q) lpart[q] = 0.f;
-      named_bar(bar_id, kSoftmaxThreads);
-      // Key tile of this thread's row for the first step (list entries are prefetched a step ahead).
-      int raw_next = ((r >> 6) < ui.cnt) ? ui.list[r >> 6] : kAbsent;
-      bool failed = false;
-      for (int n = 0; n < ui.npairs; ++n) {
-        const long gp = gp0 + n;
-        const int sb = (int)(gp % kSBufs);  // S^T buffer
-        const int pb = (int)(gp & 1);       // P^T buffer
-        const uint32_t ph = (uint32_t)((gp >> 1) & 1);
-        const int raw = raw_next;
-        const int e_next = 2 * (n + 1) + (r >> 6);
-        raw_next = (e_next < ui.cnt) ? ui.list[e_next] : kAbsent;
-        // S^T of this step, and P^T buffer sb free again (its PV MMAs of step gp - 2 complete).
-        bool ok = mbar_wait(&s.s_full[sb], (uint32_t)((gp / kSBufs) & 1), abort_flag);
-        ok = ok && mbar_wait(&s.p_empty[pb], ph ^ 1, abort_flag);
+      float m0 = -INFINITY, m1 = -INFINITY;  // shifts (log2 units) of rows r0, r1
+      float l0 = 0.f, l1 = 0.f;              // running sums over this thread's columns
+      // Key tiles of the first step (list entries are prefetched a step ahead).
+      int ea = (0 < ui.cnt) ? ui.list[0] : kAbsent, eb = (1 < ui.cnt) ? ui.list[1] : kAbsent;
+      for (int n = 0; n < ui.npairs; ++n, ++gp) {
+        const int ja = ea, jb = eb;
+        ea = (2 * n + 2 < ui.cnt) ? ui.list[2 * n + 2] : kAbsent;
+        eb = (2 * n + 3 < ui.cnt) ? ui.list[2 * n + 3] : kAbsent;
+        const int b = (int)(gp & 1);
+        bool ok = mbar_wait(&s.s_full[b], (uint32_t)((gp >> 1) & 1), abort_flag);
         tc_fence_after();
-        float x[kQW];
-        {
-          uint32_t v[kQW];
-          tmem_ld<kQW>(lane_base + kColS + sb * 64 + q0, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int q = 0; q < kQW; ++q) x[q] = __uint_as_float(v[q]);
-        }
+        uint32_t v[64];
+        tmem_ld_16x256b_x16(lane_base + kColS + 128 * b, v);
+        tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&s.s_empty[sb]);
-        const bool in_range = raw >= 0 && raw < g.nT;
-        const bool valid = in_range && (r & 63) < s.vc[in_range ? raw : 0];
-        if (!reported && raw != kAbsent && !in_range) {
+        mbar_arrive(&s.s_empty[b]);
+        // Valid keys: tile a gives keys 0..63, tile b keys 64..127.
+        const bool ina = ja >= 0 && ja < g.nT, inb = jb >= 0 && jb < g.nT;
+        if (!reported && ((ja != kAbsent && !ina) || (jb != kAbsent && !inb))) {
           report(a.dev_status, T3D_DEV_INDEX_RANGE);
           reported = true;
         }
-        if (!valid) {
+        const int ca = ina ? s.vc[ja] : 0, cb = inb ? s.vc[jb] : 0;
+        if (ca < kTileElems || cb < kTileElems) {
 #pragma unroll
-          for (int q = 0; q < kQW; ++q) x[q] = -INFINITY;
-        }
-        // x holds raw logits; the softmax scale (> 0) is folded into the thresholds and the exp2.
-        bool over = false;
+          for (int j = 0; j < 16; ++j) {
 #pragma unroll
-        for (int q = 0; q < kQW; q += 4) {
-          const float4 t4 = *reinterpret_cast<const float4*>(&s.thr[q0 + q]);
-          over |= (x[q] > t4.x) | (x[q + 1] > t4.y) | (x[q + 2] > t4.z) | (x[q + 3] > t4.w);
-        }
-        const bool bad = !ok || *abort_flag;
-        if (named_bar_or(bar_id, kSoftmaxThreads, over || bad)) {
-          if (named_bar_or(bar_id, kSoftmaxThreads, bad)) { failed = true; break; }
-          // Slow step: raise the shifts to the running maxima and rescale what was accumulated.
-#pragma unroll
-          for (int q = 0; q < kQW; ++q) {
-            const float mq = redux_max(x[q]);
-            if (lane == q) s.red[sp][q0 + q] = mq;
+            for (int e = 0; e < 2; ++e) {
+              const int key = 8 * j + 2 * t0 + e;  // 0..127
+              const bool valid = key < 64 ? key < ca : key - 64 < cb;
+              if (!valid) {
+                v[4 * j + e] = __float_as_uint(-INFINITY);
+                v[4 * j + 2 + e] = __float_as_uint(-INFINITY);
+              }
+            }
           }
-          named_bar(bar_id, kSoftmaxThreads);
-          if (gt < kQW) {
-            const int qq = q0 + gt;
-            const float old = s.shift[qq];
-            float mx = fmaxf(fmaxf(s.red[0][qq], s.red[1][qq]), fmaxf(s.red[2][qq], s.red[3][qq]));
-            mx = fmaxf(mx * sl2, old);
-            s.alpha[qq] = (old == -INFINITY) ? (mx == -INFINITY ? 1.f : 0.f) : ex2(old - mx);
-            s.shift[qq] = mx;
-            s.thr[qq] = mx == -INFINITY ? -INFINITY : (mx + kShiftSlack) / sl2;
-            s.nsh[qq] = mx == -INFINITY ? 0.f : -mx;
+        }
+        // Row maxima (the 4 threads of a row hold its 128 columns), as balanced trees.
+        float t0r[16], t1r[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          t0r[j] = fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]));
+          t1r[j] = fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int j = 0; j < w; ++j) {
+            t0r[j] = fmaxf(t0r[j], t0r[j + w]);
+            t1r[j] = fmaxf(t1r[j], t1r[j + w]);
           }
-          named_bar(bar_id, kSoftmaxThreads);
-          bool wok = true;
+        float x0 = t0r[0], x1 = t1r[0];
+        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
+        x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
+        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 1));
+        x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2));
+        x0 *= sl2;  // log2 units (the scale is positive)
+        x1 *= sl2;
+        const bool up0 = x0 > m0 + kShiftSlack || (m0 == -INFINITY && x0 > -INFINITY);
+        const bool up1 = x1 > m1 + kShiftSlack || (m1 == -INFINITY && x1 > -INFINITY);
+        if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
+        // P (and O) may only be rewritten once the previous step's PV MMAs have landed; the wait
+        // is taken as late as possible (before a rescale of O, else before the P store).
+        bool pv_waited = gp == 0;
+        if (__any_sync(0xffffffffu, up0 || up1)) {
+          const float n0 = up0 ? fmaxf(m0, x0) : m0, n1 = up1 ? fmaxf(m1, x1) : m1;
+          const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - n0);
+          const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - n1);
+          l0 *= a0;
+          l1 *= a1;
+          m0 = n0;
+          m1 = n1;
           if (n > 0) {
-            // O^T holds the contributions of earlier steps: rescale column q by alpha[q] once the
-            // last PV MMA has landed.
-            wok = mbar_wait(&s.p_empty[(gp - 1) & 1], ((gp - 1) >> 1) & 1, abort_flag);
+            // Rescale the O rows of this warp's queries (factor 1 where the shift did not move).
+            const bool pv_ok = mbar_wait(&s.pv_done, (uint32_t)((gp - 1) & 1), abort_flag);
+            if (__any_sync(0xffffffffu, !pv_ok)) { failed = true; break; }
+            pv_waited = true;
             tc_fence_after();
-            uint32_t v[kQW];
-            tmem_ld<kQW>(lane_base + kColO + q0, v);
-            tmem_wait_ld();
 #pragma unroll
-            for (int q = 0; q < kQW; ++q)
-              v[q] = __float_as_uint(__uint_as_float(v[q]) * s.alpha[q0 + q]);
-            tmem_st<kQW>(lane_base + kColO + q0, v);
+            for (int hc = 0; hc < 2; ++hc) {
+              uint32_t o[32];
+              tmem_ld_16x256b_x8(lane_base + kColO + 64 * hc, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                o[4 * j] = __float_as_uint(__uint_as_float(o[4 * j]) * a0);
+                o[4 * j + 1] = __float_as_uint(__uint_as_float(o[4 * j + 1]) * a0);
+                o[4 * j + 2] = __float_as_uint(__uint_as_float(o[4 * j + 2]) * a1);
+                o[4 * j + 3] = __float_as_uint(__uint_as_float(o[4 * j + 3]) * a1);
+              }
+              tmem_st_16x256b_x8(lane_base + kColO + 64 * hc, o);
+            }
             tmem_wait_st();
-            tc_fence_before();
           }
-#pragma unroll
-          for (int q = 0; q < kQW; q += 4) {
-            const float4 a4 = *reinterpret_cast<const float4*>(&s.alpha[q0 + q]);
-            lpart[q] *= a4.x; lpart[q + 1] *= a4.y; lpart[q + 2] *= a4.z; lpart[q + 3] *= a4.w;
-          }
-          if (named_bar_or(bar_id, kSoftmaxThreads, !wok)) { failed = true; break; }
         }
-        // P = exp2(x - shift), running sums, bf16 into this row of P^T (MN-major, 128B swizzle:
-        // 16-byte chunk c of row r lives at chunk c ^ (r & 7); this warpgroup owns kQW / 8 chunks).
-        uint8_t* prow = s.p[pb] + r * 128;
+        // P = exp2(x * scale - shift), packed as bf16 pairs (keys 8j + 2 t0, + 1 -> column 4j + t0).
+        const float ns0 = m0 == -INFINITY ? 0.f : -m0, ns1 = m1 == -INFINITY ? 0.f : -m1;
+        uint32_t pw[32];
+        float ls0[4] = {0.f, 0.f, 0.f, 0.f}, ls1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kQW / 8; ++c) {
-          uint32_t w[4];
-          const float4 n0 = *reinterpret_cast<const float4*>(&s.nsh[q0 + c * 8]);
-          const float4 n1 = *reinterpret_cast<const float4*>(&s.nsh[q0 + c * 8 + 4]);
-          const float nsh[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int q = c * 8 + 2 * e;
-            const float p0 = ex2(fmaf(x[q], sl2, nsh[2 * e]));
-            const float p1 = ex2(fmaf(x[q + 1], sl2, nsh[2 * e + 1]));
-            lpart[q] += p0;
-            lpart[q + 1] += p1;
-            __nv_bfloat162 pk = __floats2bfloat162_rn(p0, p1);
-            w[e] = *reinterpret_cast<uint32_t*>(&pk);
-          }
-          const int chunk = (kQW / 8) * wg + c;
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(w[0], w[1], w[2], w[3]);
+        for (int j = 0; j < 16; ++j) {
+          const float p00 = ex2(fmaf(__uint_as_float(v[4 * j]), sl2, ns0));
+          const float p01 = ex2(fmaf(__uint_as_float(v[4 * j + 1]), sl2, ns0));
+          const float p10 = ex2(fmaf(__uint_as_float(v[4 * j + 2]), sl2, ns1));
+          const float p11 = ex2(fmaf(__uint_as_float(v[4 * j + 3]), sl2, ns1));
+          ls0[j & 3] += p00 + p01;
+          ls1[j & 3] += p10 + p11;
+          __nv_bfloat162 q0 = __floats2bfloat162_rn(p00, p01);
+          __nv_bfloat162 q1 = __floats2bfloat162_rn(p10, p11);
+          pw[2 * j] = *reinterpret_cast<uint32_t*>(&q0);
+          pw[2 * j + 1] = *reinterpret_cast<uint32_t*>(&q1);
         }
-        fence_proxy_async();
-        mbar_arrive(&s.p_full[pb]);
+        if (!pv_waited) {
+          const bool pv_ok = mbar_wait(&s.pv_done, (uint32_t)((gp - 1) & 1), abort_flag);
+          if (__any_sync(0xffffffffu, !pv_ok)) { failed = true; break; }
+          tc_fence_after();
+        }
+        l0 += (ls0[0] + ls0[1]) + (ls0[2] + ls0[3]);
+        l1 += (ls1[0] + ls1[1]) + (ls1[2] + ls1[3]);
+        tmem_st_16x128b_x16(lane_base + kColP, pw);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&s.p_full);
       }
       if (failed) break;
-      // ---- epilogue: denominators (reduce the 128 per-key partial sums of each query)
-#pragma unroll
-      for (int q = 0; q < kQW; ++q) {
-        float v = lpart[q];
-#pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == q) s.red[sp][q0 + q] = v;
+      // The next unit's Q goes into TMEM as soon as this unit's last S MMA is done, so that its
+      // first scores are computed while this unit's epilogue runs.
+      ub = next_busy(u + gridDim.x);
+      if (ub < total_units) {
+        const bool qok = mbar_wait(&s.q_free, (uint32_t)(active & 1), abort_flag);
+        if (__any_sync(0xffffffffu, !qok)) { failed = true; break; }
+        tc_fence_after();
+        write_q(ub);
       }
-      const bool ook = mbar_wait(&s.o_full, active & 1, abort_flag);
-      named_bar(bar_id, kSoftmaxThreads);
-      if (gt < kQW) {
-        const int qq = q0 + gt;
-        s.lsum[qq] = s.red[0][qq] + s.red[1][qq] + s.red[2][qq] + s.red[3][qq];
-      }
-      if (named_bar_or(bar_id, kSoftmaxThreads, !ook || *abort_flag)) break;
+      // ---- epilogue: O / l for this thread's rows, bf16, into the tiled output
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      const bool ook = mbar_wait(&s.o_full, (uint32_t)(active & 1), abort_flag);
+      if (__any_sync(0xffffffffu, !ook)) { failed = true; break; }
       tc_fence_after();
-      // O^T row r (= column d of O) for this warpgroup's queries: divide by the denominators and
-      // stage O as [64 q][128 d] bf16 in the P^T buffer 0 (idle here: every PV MMA of the unit is
-      // complete and the next unit's first P^T write waits for the closing rendezvous below).
-      __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(s.p[0]);
-      {
-        uint32_t v[kQW];
-        tmem_ld<kQW>(lane_base + kColO + q0, v);
+      uint32_t ob0[32], ob1[32];  // bf16 pairs: (row r0 | r1, columns 64 hc + 8 j + 2 t0, + 1)
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        uint32_t o[32];
+        tmem_ld_16x256b_x8(lane_base + kColO + 64 * hc, o);
         tmem_wait_ld();
 #pragma unroll
-        for (int q = 0; q < kQW; ++q) {
-          const int qq = q0 + q;
-          const float l = s.lsum[qq];
-          const float val = l > 0.f ? __uint_as_float(v[q]) / l : 0.f;
-          stage[qq * kD + r] = __float2bfloat16_rn(val);
+        for (int j = 0; j < 8; ++j) {
+          __nv_bfloat162 y0 = __floats2bfloat162_rn(__uint_as_float(o[4 * j]) * i0,
+                                                    __uint_as_float(o[4 * j + 1]) * i0);
+          __nv_bfloat162 y1 = __floats2bfloat162_rn(__uint_as_float(o[4 * j + 2]) * i1,
+                                                    __uint_as_float(o[4 * j + 3]) * i1);
+          ob0[16 * hc + 2 * j] = *reinterpret_cast<uint32_t*>(&y0);
+          ob1[16 * hc + 2 * j] = *reinterpret_cast<uint32_t*>(&y1);
         }
       }
       tc_fence_before();
       mbar_arrive(&s.o_empty);
-      named_bar(bar_id, kSoftmaxThreads);
+      // Row rr of the output takes the result of row src(rr): rr itself, or for a query row
+      // pruned by BSA its kept source row. Rows past the tile's valid count are zero.
       const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
       const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
       const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
-      if (keep != nullptr) {  // source rows span every warpgroup's staging rows
-        if (named_bar_or(bar_id, kSoftmaxThreads, !rendezvous())) break;
-      }
-      for (int e = gt; e < kQW * kD / 8; e += kSoftmaxThreads) {
-        const int rr = q0 + e / (kD / 8), c = e % (kD / 8);
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (rr < vci) {
+      auto put = [&](int rr, const uint32_t (&ob)[32], bool zero) {
+#pragma unroll
+        for (int hc = 0; hc < 2; ++hc)
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint32_t*>(out + rr * ld + 64 * hc + 8 * j + 2 * t0) =
+                zero ? 0u : ob[16 * hc + 2 * j];
+      };
+      if (keep == nullptr) {
+        put(r0, ob0, r0 >= vci);
+        put(r1, ob1, r1 >= vci);
+      } else {
+        for (int rr = 0; rr < kTileElems; ++rr) {
           int sr = rr;
-          if (keep != nullptr && !keep[rr]) {
+          if (!keep[rr]) {
             sr = srcr[rr];
             if (sr >= kTileElems) sr = rr;
           }
-          val = *reinterpret_cast<const uint4*>(stage + sr * kD + c * 8);
+          if (sr == r0) put(rr, ob0, rr >= vci);
+          else if (sr == r1) put(rr, ob1, rr >= vci);
         }
-        *reinterpret_cast<uint4*>(out + rr * ld + c * 8) = val;
       }
-      // The staging buffer is free for the next unit once every warpgroup is done with it.
-      if (named_bar_or(bar_id, kSoftmaxThreads, !rendezvous())) break;
-      gp0 += ui.npairs;
       ++active;
     }
+    if (failed && lane == 0) fail(s, a.dev_status);
   }
 
   tc_fence_before();
@@ -588,8 +569,7 @@ int sm_count() {
 
 cudaError_t launch_attn_sm100(const Geo& g, const AttnArgs& a, cudaStream_t s) {
   Maps maps;
-  if (!make_map(&maps.q, a.q, g) || !make_map(&maps.k, a.k, g) || !make_map(&maps.v, a.v, g))
-    return cudaErrorInvalidValue;
+  if (!make_map(&maps.k, a.k, g) || !make_map(&maps.v, a.v, g)) return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemLayout) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
