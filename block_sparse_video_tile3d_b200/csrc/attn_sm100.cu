@@ -9,25 +9,24 @@
 // Shape of the computation. A work unit is one (batch, head, query tile): 64 query rows. Each step
 // takes a PAIR of its kept key tiles (128 keys; an odd last tile is paired with a fully masked copy
 // of itself) and computes, with M = 64 query rows,
-//     S[64 q, 128 keys]  = Q . K_pair^T      (A = Q in TMEM, B = K pair in shared memory, K-major)
+//     S[64 q, 128 keys]  = Q . K_pair^T      (A = Q, B = K pair: shared memory, K-major)
 //     O[64 q, D]        += P . V_pair         (A = P in TMEM, B = V pair in shared memory, MN-major)
-// fp32 accumulation in TMEM. Q and P live in TMEM, so the only shared-memory operands are the K and
-// V tiles: the tensor core's operand reads (which at N = 64 took the whole shared-memory bandwidth)
-// no longer compete with P^T or with re-reads of Q.
+// fp32 accumulation in TMEM. P lives in TMEM, so the tensor core's shared-memory operands are the
+// query tile and the K and V pairs; its operand reads no longer compete with a P^T in shared memory.
 //
 // TMEM (512 columns; an M = 64 tile occupies lanes 0..15 of each 32-lane sub-partition):
 //   S buffer b: columns 128 b .. 128 b + 127 (fp32)    O: 256 .. 383 (fp32)
-//   P: 384 .. 447 (bf16 pairs: column c holds keys 2c, 2c + 1)   Q: 448 .. 511 (bf16 pairs of d)
+//   P: 384 .. 447 (bf16 pairs: column c holds keys 2c, 2c + 1)
 //
 // Roles (one persistent CTA per SM, 8 warps, units in static round robin, head-major):
 //   warp 0      TMA producer for the K pairs (3-stage ring)
 //   warp 1      TMEM allocation; one thread issues every tcgen05.mma and tcgen05.commit
 //   warp 2      TMA producer for the V pairs (3-stage ring)
+//   warp 3      TMA producer for each unit's query tile (one buffer, refilled once the previous
+//               unit's last S has completed, so the next unit's scores start during the epilogue)
 //   warps 4..7  softmax and epilogue: thread t of warp w owns query rows 16 (w - 4) + t/4 and that
-//               + 8, and the key columns 8j + 2(t%4) + {0, 1} of each step (tcgen05.ld 16x256b); it
-//               also writes the unit's Q into TMEM.
-// MMA order: S(0), S(1), then per step n: S(n + 2) (same unit only), PV(n); the next unit's first
-// two S wait for its Q, which the softmax writes as soon as the current unit's last S has completed.
+//               + 8, and the key columns 8j + 2(t%4) + {0, 1} of each step (tcgen05.ld 16x256b).
+// MMA order: S(0), S(1), then per step n: S(n + 2) (same unit only), PV(n).
 //
 // Softmax. Each row's online-softmax state (shift m, running sum l) is private to the 4 threads
 // that share the row: the row maximum is two shuffles away, no barrier spans the warpgroup. The
@@ -57,21 +56,22 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;       // S buffer b at 128 b
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kColP = 384;
-constexpr uint32_t kColQ = 448;
 
 constexpr uint32_t kTileBytes = 64 * 128;                  // 64 rows x 128 B (one half of a tile)
 constexpr uint32_t kPairBytes = kHalves * 2 * kTileBytes;  // 32 KB: two tiles, both halves
+constexpr uint32_t kQBytes = kHalves * kTileBytes;         // 16 KB
 
 struct alignas(1024) SmemLayout {
   uint8_t k[kKStages][kPairBytes];
   uint8_t v[kVStages][kPairBytes];
+  uint8_t q[kQBytes];
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_empty[2];
   uint64_t p_full;    // P of the step written to TMEM (softmax -> MMA)
   uint64_t pv_done;   // the step's PV MMAs complete: P free, O current (MMA -> softmax)
-  uint64_t q_ready;   // the unit's Q written to TMEM (softmax -> MMA)
-  uint64_t q_free;    // the unit's last S MMA complete: Q may be overwritten (MMA -> softmax)
+  uint64_t q_full;    // the unit's Q loaded (TMA -> MMA)
+  uint64_t q_empty;   // the unit's last S MMA complete: Q may be overwritten (MMA -> producer)
   uint64_t o_full;    // the unit's last PV complete (MMA -> softmax)
   uint64_t o_empty;   // O read by the epilogue (softmax -> MMA)
   uint64_t drain;
@@ -83,7 +83,7 @@ struct alignas(1024) SmemLayout {
 static_assert(sizeof(SmemLayout) + 1024 <= 232448, "shared memory per CTA");
 constexpr int kAbsent = -0x7fffffff - 1;  // list entry beyond kv_cnt
 
-constexpr uint32_t idesc_s = idesc_bf16(64, 128, false, false);  // A = Q (TMEM), B = K, K-major
+constexpr uint32_t idesc_s = idesc_bf16(64, 128, false, false);  // A = Q, B = K, K-major
 constexpr uint32_t idesc_o = idesc_bf16(64, 128, false, true);   // A = P (TMEM), B = V, MN-major
 
 struct UnitInfo {
@@ -118,7 +118,7 @@ __device__ __forceinline__ void fail(SmemLayout& s, int32_t* status) {
 }
 
 struct Maps {
-  CUtensorMap k, v;
+  CUtensorMap q, k, v;
 };
 
 // Streams the kept key (or value) tile pairs of every unit of this CTA, in step order, into a ring
@@ -177,8 +177,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&s.p_full, kSoftmaxThreads);
     mbar_init(&s.pv_done, 1);
-    mbar_init(&s.q_ready, kSoftmaxThreads);
-    mbar_init(&s.q_free, 1);
+    mbar_init(&s.q_full, 1);
+    mbar_init(&s.q_empty, 1);
     mbar_init(&s.o_full, 1);
     mbar_init(&s.o_empty, kSoftmaxThreads);
     mbar_init(&s.drain, 1);
@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   for (int t = threadIdx.x; t < g.nT; t += kThreads) s.vc[t] = (uint8_t)tile_valid_count(g, t);
   if (warp == 0 && lane == 0) {
+    tma_prefetch(&maps.q);
     tma_prefetch(&maps.k);
     tma_prefetch(&maps.v);
   }
@@ -205,6 +206,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 2) {
     // ------------------------------------------------------------- V producer
     if (lane == 0) produce_pairs<kVStages>(s, g, a, &maps.v, s.v, s.v_full, s.v_empty, abort_flag);
+  } else if (warp == 3) {
+    // ------------------------------------------------------------- Q producer
+    if (lane == 0) {
+      int active = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
+        const UnitInfo ui = unit_info(g, a, u);
+        if (ui.npairs == 0) continue;
+        if (!mbar_wait(&s.q_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) { ok = false; break; }
+        mbar_expect_tx(&s.q_full, kQBytes);
+        const int row0 = ui.b * g.Lp + ui.i * kTileElems;
+        for (int hh = 0; hh < kHalves; ++hh)
+          tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
+        ++active;
+      }
+      if (!ok) fail(s, a.dev_status);
+      // Drain: the last query tile loaded must land before the CTA can exit.
+      if (active > 0) mbar_wait(&s.q_full, (uint32_t)((active - 1) & 1), nullptr);
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
@@ -215,6 +235,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every buffer lies below 256 KB), so each MMA's operand is a base descriptor plus a constant.
       const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
       const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
+      const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
       // S(gp) = Q . K_pair^T into S buffer gp & 1.
       auto issue_s = [&](long gp, bool last_of_unit) -> bool {
         const int ks = (int)(gp % kKStages);
@@ -228,12 +249,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
           const int hh = kk >> 2, st = kk & 3;
-          mma_bf16_ts(d_s, tmem + kColQ + 8 * kk,
-                      db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
+          mma_bf16(d_s, dq + ((hh * kTileBytes + st * 32) >> 4),
+                   db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
         }
         mma_commit(&s.s_full[b]);
         mma_commit(&s.k_empty[ks]);
-        if (last_of_unit) mma_commit(&s.q_free);
+        if (last_of_unit) mma_commit(&s.q_empty);
         return true;
       };
       // O (+)= P . V_pair of step gp.
@@ -258,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const UnitInfo ui = unit_info(g, a, u);
         const int np = ui.npairs;
         if (np == 0) continue;
-        if (!mbar_wait(&s.q_ready, (uint32_t)(active & 1), abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag)) { ok = false; break; }
         tc_fence_after();
         ok = issue_s(gp0, np == 1) && (np < 2 || issue_s(gp0 + 1, np == 2));
         for (int n = 0; n < np && ok; ++n) {
@@ -287,32 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     long gp = 0;  // global step index
     bool reported = false;
     bool failed = false;
-    // Writes the query tile of unit u into TMEM as the A operand of the S MMAs (row r at lane
-    // (r % 16) + 32 (r / 16); column c holds d = 2c, 2c + 1).
-    auto write_q = [&](int u) {
-      const UnitInfo ui = unit_info(g, a, u);
-      const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
-      const __nv_bfloat16* qb = static_cast<const __nv_bfloat16*>(a.q) + (long)ui.h * kD;
-      uint32_t w[32];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {  // d = 16 j + 4 t0 .. + 3: columns 8 j + 2 t0, + 1
-        const uint2 x0 = *reinterpret_cast<const uint2*>(qb + (row0 + r0) * ld + 16 * j + 4 * t0);
-        const uint2 x1 = *reinterpret_cast<const uint2*>(qb + (row0 + r1) * ld + 16 * j + 4 * t0);
-        w[4 * j] = x0.x; w[4 * j + 1] = x0.y; w[4 * j + 2] = x1.x; w[4 * j + 3] = x1.y;
-      }
-      tmem_st_16x256b_x8(lane_base + kColQ, w);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&s.q_ready);
-    };
-    // Next unit (from u) with at least one kept pair, or total_units.
-    auto next_busy = [&](int u) -> int {
-      for (; u < total_units; u += gridDim.x)
-        if (unit_info(g, a, u).npairs > 0) return u;
-      return total_units;
-    };
-    int ub = next_busy(blockIdx.x);
-    if (ub < total_units) write_q(ub);
     for (int u = blockIdx.x; u < total_units && !failed; u += gridDim.x) {
       const UnitInfo ui = unit_info(g, a, u);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
@@ -451,15 +446,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&s.p_full);
       }
       if (failed) break;
-      // The next unit's Q goes into TMEM as soon as this unit's last S MMA is done, so that its
-      // first scores are computed while this unit's epilogue runs.
-      ub = next_busy(u + gridDim.x);
-      if (ub < total_units) {
-        const bool qok = mbar_wait(&s.q_free, (uint32_t)(active & 1), abort_flag);
-        if (__any_sync(0xffffffffu, !qok)) { failed = true; break; }
-        tc_fence_after();
-        write_q(ub);
-      }
       // ---- epilogue: O / l for this thread's rows, bf16, into the tiled output
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -469,51 +455,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ook = mbar_wait(&s.o_full, (uint32_t)(active & 1), abort_flag);
       if (__any_sync(0xffffffffu, !ook)) { failed = true; break; }
       tc_fence_after();
-      uint32_t ob0[32], ob1[32];  // bf16 pairs: (row r0 | r1, columns 64 hc + 8 j + 2 t0, + 1)
+      // O rows are read with the 32-lane shape: lane L < 16 of this warp holds row 16 sp + L (the
+      // M = 64 layout), 32 columns per load, so a row goes out in 16-byte stores. Its 1 / l comes
+      // from the threads that own the row in the 16x256b layout (row r0 of lanes 4L.., or r1).
+      const int rown = 16 * sp + (lane & 15);
+      const float ia = __shfl_sync(0xffffffffu, i0, 4 * (lane & 7));
+      const float ib = __shfl_sync(0xffffffffu, i1, 4 * (lane & 7));
+      const float inv = (lane & 15) < 8 ? ia : ib;
+      const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
+      const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
+      const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
 #pragma unroll
-      for (int hc = 0; hc < 2; ++hc) {
+      for (int c = 0; c < kD / 32; ++c) {
         uint32_t o[32];
-        tmem_ld_16x256b_x8(lane_base + kColO + 64 * hc, o);
+        tmem_ld32(lane_base + kColO + 32 * c, o);
         tmem_wait_ld();
+        if (lane < 16) {
+          uint4 w4[4];
+          uint32_t* w = reinterpret_cast<uint32_t*>(w4);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          __nv_bfloat162 y0 = __floats2bfloat162_rn(__uint_as_float(o[4 * j]) * i0,
-                                                    __uint_as_float(o[4 * j + 1]) * i0);
-          __nv_bfloat162 y1 = __floats2bfloat162_rn(__uint_as_float(o[4 * j + 2]) * i1,
-                                                    __uint_as_float(o[4 * j + 3]) * i1);
-          ob0[16 * hc + 2 * j] = *reinterpret_cast<uint32_t*>(&y0);
-          ob1[16 * hc + 2 * j] = *reinterpret_cast<uint32_t*>(&y1);
+          for (int e = 0; e < 16; ++e) {
+            __nv_bfloat162 y = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                     __uint_as_float(o[2 * e + 1]) * inv);
+            w[e] = *reinterpret_cast<uint32_t*>(&y);
+          }
+          // Row rr of the output takes the result of row src(rr): rr itself, or for a query row
+          // pruned by BSA its kept source row. Rows past the tile's valid count are zero.
+          auto put = [&](int rr) {
+            uint4* dst = reinterpret_cast<uint4*>(out + rr * ld + 32 * c);
+            const bool zero = rr >= vci;
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = zero ? make_uint4(0u, 0u, 0u, 0u) : w4[q4];
+          };
+          if (keep == nullptr) {
+            put(rown);
+          } else {
+            for (int rr = 0; rr < kTileElems; ++rr) {
+              int sr = rr;
+              if (!keep[rr]) {
+                sr = srcr[rr];
+                if (sr >= kTileElems) sr = rr;
+              }
+              if (sr == rown) put(rr);
+            }
+          }
         }
       }
       tc_fence_before();
       mbar_arrive(&s.o_empty);
-      // Row rr of the output takes the result of row src(rr): rr itself, or for a query row
-      // pruned by BSA its kept source row. Rows past the tile's valid count are zero.
-      const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
-      const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
-      const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
-      auto put = [&](int rr, const uint32_t (&ob)[32], bool zero) {
-#pragma unroll
-        for (int hc = 0; hc < 2; ++hc)
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            *reinterpret_cast<uint32_t*>(out + rr * ld + 64 * hc + 8 * j + 2 * t0) =
-                zero ? 0u : ob[16 * hc + 2 * j];
-      };
-      if (keep == nullptr) {
-        put(r0, ob0, r0 >= vci);
-        put(r1, ob1, r1 >= vci);
-      } else {
-        for (int rr = 0; rr < kTileElems; ++rr) {
-          int sr = rr;
-          if (!keep[rr]) {
-            sr = srcr[rr];
-            if (sr >= kTileElems) sr = rr;
-          }
-          if (sr == r0) put(rr, ob0, rr >= vci);
-          else if (sr == r1) put(rr, ob1, rr >= vci);
-        }
-      }
       ++active;
     }
     if (failed && lane == 0) fail(s, a.dev_status);
@@ -569,7 +558,8 @@ int sm_count() {
 
 cudaError_t launch_attn_sm100(const Geo& g, const AttnArgs& a, cudaStream_t s) {
   Maps maps;
-  if (!make_map(&maps.k, a.k, g) || !make_map(&maps.v, a.v, g)) return cudaErrorInvalidValue;
+  if (!make_map(&maps.q, a.q, g) || !make_map(&maps.k, a.k, g) || !make_map(&maps.v, a.v, g))
+    return cudaErrorInvalidValue;
   const size_t smem = sizeof(SmemLayout) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
