@@ -18,7 +18,8 @@ from ._lib import Geom, Tile3dError, check, lib
 __all__ = [
     "Geom", "Tile3dError", "geometry", "tile3d_scatter", "tile3d_gather", "tile_pool",
     "tile3d_scatter_pool",
-    "tile_select_topk", "tile_select_mass", "tile_prune_queries", "block_mask_to_index",
+    "tile_select_topk", "tile_select_mass", "tile_prune_queries", "tile_prune_queries_ratio",
+    "block_mask_to_index",
     "block_sparse_attn_fwd", "block_sparse_attn_workspace_size", "TileSparseAttention",
 ]
 
@@ -181,6 +182,27 @@ def tile_prune_queries(qt, T, H, W, cos_thresh, keep=None, src_row=None, pq_kept
     return keep, src_row, pq_kept
 
 
+def tile_prune_queries_ratio(qt, T, H, W, keep_ratio, keep=None, src_row=None, pq_kept=None):
+    """BSA query pruning keeping ``max(1, floor(64 * keep_ratio))`` rows per block (the rows least
+    similar to the block mean). Same inputs and outputs as ``tile_prune_queries``."""
+    B, Lp, nh, D = qt.shape
+    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh, D)
+    _need(qt, "q", torch.bfloat16, (B, Lp2, nh, D))
+    dev = qt.device
+    keep = torch.empty((B, nh, nT, 64), dtype=torch.uint8, device=dev) if keep is None else keep
+    src_row = torch.empty((B, nh, nT, 64), dtype=torch.uint8, device=dev) if src_row is None \
+        else src_row
+    pq_kept = torch.empty((B, nh, nT, D), dtype=torch.float32, device=dev) if pq_kept is None \
+        else pq_kept
+    _need(keep, "keep", torch.uint8, (B, nh, nT, 64))
+    _need(src_row, "src_row", torch.uint8, (B, nh, nT, 64))
+    _need(pq_kept, "pq_kept", torch.float32, (B, nh, nT, D))
+    g = _geom(B, T, H, W, nh, D)
+    check(lib.tile_prune_queries_ratio(ctypes.byref(g), _ptr(qt), float(keep_ratio), _ptr(keep),
+                                       _ptr(src_row), _ptr(pq_kept), _stream()))
+    return keep, src_row, pq_kept
+
+
 def block_mask_to_index(mask, T, H, W, D, kmax=None, kv_idx=None, kv_cnt=None, dev_status=None):
     """uint8 block map ``[B, heads, nT, nT]`` -> ascending ``(kv_idx, kv_cnt)`` int32."""
     B, nh, nT, nT2 = mask.shape
@@ -237,20 +259,22 @@ class TileSparseAttention:
 
     ``mode``: ``"topk"`` (keep ``topk`` key tiles per query tile by pooled score), ``"mass"``
     (cumulative softmax mass ``mass`` with floor ``min_k``), ``"bsa"`` (query pruning at cosine
-    ``cos_thresh``, then mass selection from the kept queries) or ``"mask"`` (a fixed uint8 block
-    map ``[B, heads, nT, nT]``).
+    ``cos_thresh`` — or, with ``keep_ratio`` given, a fixed ``max(1, floor(64 * keep_ratio))`` rows
+    per block — then mass selection from the kept queries) or ``"mask"`` (a fixed uint8 block map
+    ``[B, heads, nT, nT]``).
 
     ``forward(q, k, v)`` takes raster ``[B, L, heads, D]`` bf16 CUDA tensors and returns the raster
     output; one call = scatter Q, K, V -> coarse selection -> block-sparse attention -> gather.
     """
 
     def __init__(self, B, T, H, W, heads, D, mode="topk", topk=None, mass=0.9, min_k=1,
-                 cos_thresh=0.95, mask=None, device="cuda"):
+                 cos_thresh=0.95, mask=None, keep_ratio=None, device="cuda"):
         self.B, self.T, self.H, self.W, self.heads, self.D = B, T, H, W, heads, D
         self.mode = mode
         self.nT, self.Lp, self.vc = geometry(T, H, W, B, heads, D)
         self.scale = 1.0 / math.sqrt(D)
         self.topk, self.mass, self.min_k, self.cos_thresh = topk, mass, min_k, cos_thresh
+        self.keep_ratio = keep_ratio
         dev = torch.device(device)
         shp = (B, self.Lp, heads, D)
         self.qt = torch.empty(shp, dtype=torch.bfloat16, device=dev)
@@ -308,7 +332,10 @@ class TileSparseAttention:
                 ("scatter_pool_k", lambda: tile3d_scatter_pool(k, T, H, W, self.kt, self.pk)),
                 ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt)),
             ]
-            if self.mode == "bsa":
+            if self.mode == "bsa" and self.keep_ratio is not None:
+                st.append(("prune_q", lambda: tile_prune_queries_ratio(
+                    self.qt, T, H, W, self.keep_ratio, self.keep, self.src_row, self.pq)))
+            elif self.mode == "bsa":
                 st.append(("prune_q", lambda: tile_prune_queries(
                     self.qt, T, H, W, self.cos_thresh, self.keep, self.src_row, self.pq)))
             if self.mode == "topk":

@@ -171,8 +171,30 @@ t3d_status tile_prune_queries(const t3d_geom* g, const void* q, float cos_thresh
                 "query pruning needs every tile full (L=%d must equal 64 * nT = %d)", geo.L, geo.Lp);
   if (isnan(cos_thresh)) return fail(T3D_ERR_INVALID, "cos_thresh is NaN");
   return cuda_status(
-      t3d::launch_prune(geo, q, cos_thresh, keep, src_row, pq_kept, as_stream(stream)),
+      t3d::launch_prune(geo, q, cos_thresh, 0, keep, src_row, pq_kept, as_stream(stream)),
       "tile_prune_queries");
+}
+
+t3d_status tile_prune_queries_ratio(const t3d_geom* g, const void* q, float keep_ratio,
+                                    uint8_t* keep, uint8_t* src_row, float* pq_kept,
+                                    t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_ptr(q, "q"));
+  T3D_CHECK(check_ptr(keep, "keep"));
+  T3D_CHECK(check_ptr(src_row, "src_row"));
+  T3D_CHECK(check_ptr(pq_kept, "pq_kept"));
+  if (geo.L != geo.Lp)
+    return fail(T3D_ERR_INVALID,
+                "query pruning needs every tile full (L=%d must equal 64 * nT = %d)", geo.L, geo.Lp);
+  if (!(keep_ratio > 0.f && keep_ratio <= 1.f))
+    return fail(T3D_ERR_INVALID, "keep_ratio=%g must lie in (0, 1]", (double)keep_ratio);
+  // Kept rows per block, in double so that the count is the exact floor of 64 * keep_ratio.
+  int keep_size = (int)floor((double)keep_ratio * t3d::kTileElems);
+  keep_size = keep_size < 1 ? 1 : (keep_size > t3d::kTileElems ? t3d::kTileElems : keep_size);
+  return cuda_status(
+      t3d::launch_prune(geo, q, 0.f, keep_size, keep, src_row, pq_kept, as_stream(stream)),
+      "tile_prune_queries_ratio");
 }
 
 t3d_status block_mask_to_index(const t3d_geom* g, const uint8_t* mask, int kmax, int32_t* kv_idx,

@@ -24,7 +24,7 @@ cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, f
                                int32_t* dev_status, cudaStream_t s);
 cudaError_t launch_mask_to_index(const Geo& g, const uint8_t* mask, int kmax, int32_t* kv_idx,
                                  int32_t* kv_cnt, int32_t* dev_status, cudaStream_t s);
-cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, uint8_t* keep,
+cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, int keep_size, uint8_t* keep,
                          uint8_t* src_row, float* pq_kept, cudaStream_t s);
 
 struct AttnArgs {

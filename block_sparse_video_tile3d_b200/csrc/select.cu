@@ -389,8 +389,11 @@ __global__ void mask_to_index_kernel(Geo g, const uint8_t* __restrict__ mask, in
 // BSA query pruning, one CTA (8 warps) per (batch, head, block of 64 rows).
 constexpr int kPruneThreads = 256;
 
+// keep_size == 0: threshold mode (rows with cosine to the block mean above cos_thresh are pruned);
+// keep_size > 0: ratio mode (the keep_size rows with the lowest cosine are kept, lowest index on
+// ties). Either way a pruned row copies its most cosine-similar kept row.
 __global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_bfloat16* __restrict__ q,
-                                                              float cos_thresh,
+                                                              float cos_thresh, int keep_size,
                                                               uint8_t* __restrict__ keep,
                                                               uint8_t* __restrict__ src_row,
                                                               float* __restrict__ pq_kept) {
@@ -448,7 +451,20 @@ __global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_
     }
   }
   __syncthreads();
-  if (w == 0) {
+  if (w == 0 && keep_size > 0) {
+    // Ratio mode: rank of row r among (cosine, index) pairs in increasing order.
+    for (int r0 = 0; r0 < kTileElems; r0 += 32) {
+      const int r = r0 + lane;
+      const float c = cosm[r];
+      int rank = 0;
+      for (int j = 0; j < kTileElems; ++j) {
+        const float cj = cosm[j];
+        rank += (cj < c || (cj == c && j < r)) ? 1 : 0;
+      }
+      keep_s[r] = rank < keep_size ? 1 : 0;
+    }
+    if (lane == 0) n_keep = keep_size;
+  } else if (w == 0) {
     int nk = 0;
     for (int r0 = 0; r0 < kTileElems; r0 += 32) {
       const int r = r0 + lane;
@@ -551,7 +567,7 @@ cudaError_t launch_mask_to_index(const Geo& g, const uint8_t* mask, int kmax, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, uint8_t* keep,
+cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, int keep_size, uint8_t* keep,
                          uint8_t* src_row, float* pq_kept, cudaStream_t s) {
   const size_t smem = ((size_t)kTileElems * (g.D + 1) + g.D + 2 * kTileElems) * sizeof(float) +
                       2 * kTileElems * sizeof(int);
@@ -560,7 +576,7 @@ cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, uint8_t*
   if (e != cudaSuccess) return e;
   dim3 grid(g.nT, g.heads, g.B);
   prune_kernel<<<grid, kPruneThreads, smem, s>>>(g, static_cast<const __nv_bfloat16*>(q),
-                                                 cos_thresh, keep, src_row, pq_kept);
+                                                 cos_thresh, keep_size, keep, src_row, pq_kept);
   return cudaGetLastError();
 }
 

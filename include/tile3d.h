@@ -166,6 +166,21 @@ t3d_status tile_prune_queries(const t3d_geom* g, const void* q, float cos_thresh
                               uint8_t* src_row, float* pq_kept, t3d_stream stream);
 
 /*
+ * tile_prune_queries_ratio — BSA query pruning with a fixed count of kept rows per block.
+ * FastVideo API docs, bsa_attn page, BSAAttentionImpl.forward: the pruning helper takes the
+ * metadata's query_keep_ratio and returns a keep_size. Reading: keep_size = max(1, floor(64 *
+ * keep_ratio)) (computed in double on the host) rows per block are kept — the rows least similar to
+ * the block mean (lowest cosine, lowest index on ties); a pruned row copies the output of the kept
+ * row it is most cosine-similar to (lowest index on ties), as in tile_prune_queries.
+ * Requires L == Lp (every tile full).
+ *   keep_ratio: in (0, 1], else T3D_ERR_INVALID.
+ *   q, keep, src_row, pq_kept: as in tile_prune_queries.
+ */
+t3d_status tile_prune_queries_ratio(const t3d_geom* g, const void* q, float keep_ratio,
+                                    uint8_t* keep, uint8_t* src_row, float* pq_kept,
+                                    t3d_stream stream);
+
+/*
  * block_mask_to_index — 0/1 block map -> ascending index lists.
  * FastVideo API docs, fastvideo.attention.backends page, sla.get_block_map (the same selection
  * as a block map and as a LUT); video_sparse_attn_h3 page (mask route of the sm100a kernel).

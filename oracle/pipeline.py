@@ -27,8 +27,11 @@ def as_f64(x) -> np.ndarray:
 
 
 def coarse_select(qt, kt, vc, mode: str, *, k: int = 0, scale: float = 1.0, tau: float = 0.9,
-                  min_k: int = 1, cos_thresh: float = 0.95, mask=None) -> dict:
-    """Stage 2 on tile-ordered tensors. Returns a dict with ``sets`` and the intermediates."""
+                  min_k: int = 1, cos_thresh: float = 0.95, mask=None, keep_ratio=None) -> dict:
+    """Stage 2 on tile-ordered tensors. Returns a dict with ``sets`` and the intermediates.
+
+    In ``"bsa"`` mode a ``keep_ratio`` selects the ratio form of the query pruning (a fixed count
+    of kept rows per block) instead of the cosine threshold."""
     res: dict = {}
     if mode == "mask":
         res["sets"] = select.map_to_sets(np.asarray(mask))
@@ -36,7 +39,10 @@ def coarse_select(qt, kt, vc, mode: str, *, k: int = 0, scale: float = 1.0, tau:
     pk = pool.tile_mean_pool(kt, vc)
     res["pk"] = pk
     if mode == "bsa":
-        keep, src, cosm = bsa.prune_queries(qt, cos_thresh)
+        if keep_ratio is not None:
+            keep, src, cosm = bsa.prune_queries_ratio(qt, keep_ratio)
+        else:
+            keep, src, cosm = bsa.prune_queries(qt, cos_thresh)
         pq = bsa.pooled_kept_queries(qt, keep)
         res.update(keep=keep, src=src, cos=cosm)
     else:
@@ -55,7 +61,7 @@ def coarse_select(qt, kt, vc, mode: str, *, k: int = 0, scale: float = 1.0, tau:
 
 def forward(q, k, v, T: int, H: int, W: int, mode: str, *, scale: float, topk: int = 0,
             tau: float = 0.9, min_k: int = 1, cos_thresh: float = 0.95, mask=None,
-            q_tiles=None) -> dict:
+            q_tiles=None, keep_ratio=None) -> dict:
     """Raster ``[B, L, heads, D]`` Q, K, V -> raster output plus every intermediate (fp64)."""
     q, k, v = as_f64(q), as_f64(k), as_f64(v)
     vc = tiling.variable_block_sizes(T, H, W)
@@ -63,7 +69,7 @@ def forward(q, k, v, T: int, H: int, W: int, mode: str, *, scale: float, topk: i
     kt = tiling.tile_scatter(k, T, H, W)
     vt = tiling.tile_scatter(v, T, H, W)
     res = coarse_select(qt, kt, vc, mode, k=topk, scale=scale, tau=tau, min_k=min_k,
-                        cos_thresh=cos_thresh, mask=mask)
+                        cos_thresh=cos_thresh, mask=mask, keep_ratio=keep_ratio)
     ot = attention.block_sparse_attention(qt, kt, vt, vc, res["sets"], scale,
                                           keep=res.get("keep"), src=res.get("src"),
                                           q_tiles=q_tiles)

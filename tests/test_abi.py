@@ -25,7 +25,8 @@ def _declared():
 def test_every_declared_symbol_is_exported_and_bound():
     names = _declared()
     assert {"tile3d_scatter", "tile_pool", "tile_select_topk", "block_sparse_attn_fwd",
-            "tile3d_gather", "tile_select_mass", "tile_prune_queries", "block_mask_to_index",
+            "tile3d_gather", "tile_select_mass", "tile_prune_queries", "tile_prune_queries_ratio",
+            "block_mask_to_index",
             "tile3d_geometry", "block_sparse_attn_workspace_size", "t3d_last_error_string",
             "t3d_version"} <= names
     for n in names:
@@ -96,6 +97,13 @@ def test_other_calls_reject_bad_arguments():
     assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 0.9, 1, 9, FAKE, FAKE, None, None) == \
         _lib.T3D_ERR_INVALID
     assert lib.tile_prune_queries(_g(T=5), FAKE, 0.95, FAKE, FAKE, FAKE, None) == \
+        _lib.T3D_ERR_INVALID
+    for ratio in (0.0, -0.5, 1.5, float("nan")):  # the keep ratio must lie in (0, 1]
+        assert lib.tile_prune_queries_ratio(g, FAKE, ratio, FAKE, FAKE, FAKE, None) == \
+            _lib.T3D_ERR_INVALID
+    assert lib.tile_prune_queries_ratio(_g(T=5), FAKE, 0.5, FAKE, FAKE, FAKE, None) == \
+        _lib.T3D_ERR_INVALID  # ragged grid
+    assert lib.tile_prune_queries_ratio(g, None, 0.5, FAKE, FAKE, FAKE, None) == \
         _lib.T3D_ERR_INVALID
     assert lib.block_mask_to_index(g, None, 4, FAKE, FAKE, None, None) == _lib.T3D_ERR_INVALID
     assert lib.block_mask_to_index(g, FAKE, 0, FAKE, FAKE, None, None) == _lib.T3D_ERR_INVALID

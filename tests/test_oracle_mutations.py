@@ -15,6 +15,7 @@ import oracle.pool
 import oracle.select
 import oracle.tiling
 from tests import test_oracle_attention as ta
+from tests import test_oracle_bsa_ratio as tr
 from tests import test_oracle_pool_select as tp
 from tests import test_oracle_tiling as tt
 
@@ -69,6 +70,17 @@ def _prune_argmin(rows, thresh):
 _orig_prune = oracle.bsa.prune_block
 
 
+def _ratio_keep_most_similar(rows, ratio):
+    rows = rows.astype(np.float64)
+    n = rows.shape[0]
+    mu = rows.sum(axis=0) / n
+    cmean = np.array([oracle.bsa._cos(rows[i], mu) for i in range(n)])
+    order = sorted(range(n), key=lambda i: (-cmean[i], i))  # most similar first: wrong
+    keep = np.zeros(n, dtype=bool)
+    keep[order[:oracle.bsa.keep_size_for_ratio(ratio, n)]] = True
+    return keep, oracle.bsa._sources(rows, keep), cmean
+
+
 @pytest.mark.parametrize("patch,pin", [
     ((oracle.tiling, "tile_partition_indices", _swapped_partition),
      lambda: tt.test_partition_matches_sort_by_tile_key((5, 9, 9))),
@@ -79,6 +91,10 @@ _orig_prune = oracle.bsa.prune_block
     ((oracle.attention, "_key_rows", _keys_all_slots),
      lambda: ta.test_full_selection_is_dense_attention((5, 6, 7))),
     ((oracle.bsa, "prune_block", _prune_argmin), ta.test_prune_cosine_against_torch),
+    ((oracle.bsa, "prune_block_ratio", _ratio_keep_most_similar),
+     tr.test_fan_keeps_the_widest_angles_and_copies_the_nearest_kept_row),
+    ((oracle.bsa, "keep_size_for_ratio", lambda ratio, n=64: max(1, int(round(ratio * n)))),
+     lambda: tr.test_keep_size(0.2, 12)),
 ])
 def test_planted_mistake_is_caught(monkeypatch, patch, pin):
     mod, name, fn = patch
