@@ -16,27 +16,35 @@
 //
 // TMEM (512 columns; an M = 64 tile occupies lanes 0..15 of each 32-lane sub-partition):
 //   S buffer b: columns 128 b .. 128 b + 127 (fp32)    O: 256 .. 383 (fp32)
-//   P: 384 .. 447 (bf16 pairs: column c holds keys 2c, 2c + 1)
+//   P buffer b: 384 + 64 b .. 447 + 64 b (bf16 pairs: column c holds keys 2c, 2c + 1)
+// Step n uses S and P buffer n & 1, so the softmax of step n + 1 never waits for the PV of step n.
 //
-// Roles (one persistent CTA per SM, 8 warps, units in static round robin, head-major):
-//   warp 0      TMA producer for the K pairs (3-stage ring)
-//   warp 1      TMEM allocation; one thread issues every tcgen05.mma and tcgen05.commit
-//   warp 2      TMA producer for the V pairs (3-stage ring)
-//   warp 3      TMA producer for each unit's query tile (one buffer, refilled once the previous
-//               unit's last S has completed, so the next unit's scores start during the epilogue)
-//   warps 4..7  softmax and epilogue: thread t of warp w owns query rows 16 (w - 4) + t/4 and that
-//               + 8, and the key columns 8j + 2(t%4) + {0, 1} of each step (tcgen05.ld 16x256b).
-// MMA order: S(0), S(1), then per step n: S(n + 2) (same unit only), PV(n).
+// Roles (one persistent CTA per SM, 12 warps, units in static round robin, head-major):
+//   warp 0       TMA producer for the K and V pairs (3-stage rings each)
+//   warp 1       TMEM allocation; one thread issues the S MMAs and their commits
+//   warp 2       one thread issues the PV MMAs and their commits
+//   warp 3       TMA producer for each unit's query tile (one buffer, refilled once the previous
+//                unit's last S has completed, so the next unit's scores start during the epilogue)
+//   warps 4..11  softmax and epilogue, two halves of 4 warps: half h takes key tile h of every pair
+//                (score columns 64 h .. 64 h + 63) and output columns 64 h .. 64 h + 63. Thread t of
+//                warp w owns query rows 16 (w % 4) + t/4 and that + 8, and the key columns
+//                64 h + 8j + 2(t%4) + {0, 1} (tcgen05.ld 16x256b). Warps w and w + 4 read the same
+//                TMEM lanes and pair up through shared memory.
+// S(n) is issued as soon as its K pair has landed and the softmax has read S(n - 2), so scores run
+// up to two steps ahead; PV(n) as soon as P(n) is in TMEM.
 //
-// Softmax. Each row's online-softmax state (shift m, running sum l) is private to the 4 threads
-// that share the row: the row maximum is two shuffles away, no barrier spans the warpgroup. The
-// shift (log2 units) is raised only when a row's logits exceed it by more than kShiftSlack — then
-// the warp rescales the O rows of its 16 queries in TMEM (factor 1 for the rows that did not move)
-// once the previous PV has landed. Any shift gives the same softmax; the bound keeps P within
-// [0, 2^kShiftSlack] so nothing overflows.
+// Softmax. A row's online-softmax state (shift m, running sum l) lives with the 8 threads that
+// share the row, 4 in each half: each half reduces its 64 columns with two shuffles, and the two
+// halves swap their row maxima through shared memory (one 64-thread named barrier per warp pair and
+// step), so both raise the shift identically and keep partial sums of their own columns. The shift
+// (log2 units) is raised only when a row's logits exceed it by more than kShiftSlack; each half then
+// rescales its O columns of the rows concerned in TMEM (factor 1 for rows that did not move) once
+// the previous PV has landed. Any shift gives the same softmax; the bound keeps P within
+// [0, 2^kShiftSlack] so nothing overflows. Two warps per scheduler overlap each other's latencies.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA records T3D_DEV_TIMEOUT, stops issuing work,
-// waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
+// waits (bounded) for its copies and MMAs in flight, frees TMEM and returns. The two warps of a pair
+// leave their loops together: a failure is carried to the pair's next barrier, which ORs it.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -49,13 +57,13 @@ constexpr int kD = 128;             // head dimension handled by this kernel
 constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a row
 constexpr int kKStages = 3;         // K-pair ring depth
 constexpr int kVStages = 3;         // V-pair ring depth
-constexpr int kThreads = 256;       // 8 warps: producers / MMA, softmax warpgroup
-constexpr int kSoftmaxThreads = 128;
+constexpr int kThreads = 384;       // 12 warps: producers / MMA, two softmax halves
+constexpr int kSoftmaxThreads = 256;
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;       // S buffer b at 128 b
 constexpr uint32_t kColO = 256;
-constexpr uint32_t kColP = 384;
+constexpr uint32_t kColP = 384;     // P buffer b at 384 + 64 b
 
 constexpr uint32_t kTileBytes = 64 * 128;                  // 64 rows x 128 B (one half of a tile)
 constexpr uint32_t kPairBytes = kHalves * 2 * kTileBytes;  // 32 KB: two tiles, both halves
@@ -68,14 +76,16 @@ struct alignas(1024) SmemLayout {
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full;    // P of the step written to TMEM (softmax -> MMA)
-  uint64_t pv_done;   // the step's PV MMAs complete: P free, O current (MMA -> softmax)
+  uint64_t p_full[2];   // P of a step written to TMEM buffer (step & 1) (softmax -> MMA)
+  uint64_t pv_done[2];  // that step's PV MMAs complete: its P buffer free, O current (MMA -> softmax)
   uint64_t q_full;    // the unit's Q loaded (TMA -> MMA)
   uint64_t q_empty;   // the unit's last S MMA complete: Q may be overwritten (MMA -> producer)
   uint64_t o_full;    // the unit's last PV complete (MMA -> softmax)
   uint64_t o_empty;   // O read by the epilogue (softmax -> MMA)
-  uint64_t drain;
-  uint8_t vc[kMaxTiles];  // valid token count of every tile
+  uint64_t drain[2];  // all MMAs of the S issuer / the PV issuer complete
+  float xmax[2][2][4][16];  // [step & 1][half][warp % 4][row]: row maxima swapped between halves
+  float xsum[2][4][16];     // [half][warp % 4][row]: row sums swapped at the end of a unit
+  uint8_t vc[kMaxTiles];    // valid token count of every tile
   uint32_t tmem_base;
   int abort;
 };
@@ -121,43 +131,54 @@ struct Maps {
   CUtensorMap q, k, v;
 };
 
-// Streams the kept key (or value) tile pairs of every unit of this CTA, in step order, into a ring
-// of kStages pair buffers (lane 0 of a producer warp).
-template <int kStages>
+// Streams the kept key and value tile pairs of every unit of this CTA, in step order, into their
+// rings (lane 0 of the producer warp). Step gp's K pair goes to K stage gp % kKStages once S(gp -
+// kKStages) has completed, its V pair to V stage gp % kVStages once PV(gp - kVStages) has.
 __device__ __forceinline__ void produce_pairs(SmemLayout& s, const Geo& g, const AttnArgs& a,
-                                              const CUtensorMap* map, uint8_t (*ring)[kPairBytes],
-                                              uint64_t* full, uint64_t* empty,
-                                              volatile int* abort_flag) {
+                                              const Maps& maps, volatile int* abort_flag) {
   const int total_units = g.B * g.heads * g.nT;
-  long gp0 = 0, issued = 0;
+  long gp = 0, nk = 0, nv = 0;  // steps begun, K and V pairs issued
   bool ok = true;
   for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
     const UnitInfo ui = unit_info(g, a, u);
-    for (int n = 0; n < ui.npairs; ++n) {
-      const long gp = gp0 + n;
-      const int st = (int)(gp % kStages);
-      if (!mbar_wait(&empty[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag)) {
-        ok = false;
-        break;
-      }
+    for (int n = 0; n < ui.npairs; ++n, ++gp) {
       int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
       if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
       if (jb < 0) jb = ja;
-      mbar_expect_tx(&full[st], kPairBytes);
-      for (int hh = 0; hh < kHalves; ++hh) {
-        uint8_t* dst = ring[st] + hh * 2 * kTileBytes;
-        tma_load_3d(dst, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
-        tma_load_3d(dst + kTileBytes, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + jb * kTileElems);
+      const int za = ui.b * g.Lp + ja * kTileElems, zb = ui.b * g.Lp + jb * kTileElems;
+      const int ks = (int)(gp % kKStages), vs = (int)(gp % kVStages);
+      if (!mbar_wait(&s.k_empty[ks], (uint32_t)(((gp / kKStages) & 1) ^ 1), abort_flag)) {
+        ok = false;
+        break;
       }
-      ++issued;
+      mbar_expect_tx(&s.k_full[ks], kPairBytes);
+      for (int hh = 0; hh < kHalves; ++hh) {
+        uint8_t* dst = s.k[ks] + hh * 2 * kTileBytes;
+        tma_load_3d(dst, &maps.k, &s.k_full[ks], 64 * hh, ui.h, za);
+        tma_load_3d(dst + kTileBytes, &maps.k, &s.k_full[ks], 64 * hh, ui.h, zb);
+      }
+      ++nk;
+      if (!mbar_wait(&s.v_empty[vs], (uint32_t)(((gp / kVStages) & 1) ^ 1), abort_flag)) {
+        ok = false;
+        break;
+      }
+      mbar_expect_tx(&s.v_full[vs], kPairBytes);
+      for (int hh = 0; hh < kHalves; ++hh) {
+        uint8_t* dst = s.v[vs] + hh * 2 * kTileBytes;
+        tma_load_3d(dst, &maps.v, &s.v_full[vs], 64 * hh, ui.h, za);
+        tma_load_3d(dst + kTileBytes, &maps.v, &s.v_full[vs], 64 * hh, ui.h, zb);
+      }
+      ++nv;
     }
-    gp0 += ui.npairs;
   }
   if (!ok) fail(s, a.dev_status);
   // Drain: the last loads issued must land before the CTA can exit.
-  for (long gp = issued - kStages; gp < issued; ++gp)
-    if (gp >= 0) mbar_wait(&full[gp % kStages], (uint32_t)((gp / kStages) & 1), nullptr);
+  for (long t = nk - kKStages; t < nk; ++t)
+    if (t >= 0) mbar_wait(&s.k_full[t % kKStages], (uint32_t)((t / kKStages) & 1), nullptr);
+  for (long t = nv - kVStages; t < nv; ++t)
+    if (t >= 0) mbar_wait(&s.v_full[t % kVStages], (uint32_t)((t / kVStages) & 1), nullptr);
 }
+
 
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ Maps maps, Geo g, AttnArgs a, float sl2) {
@@ -175,13 +196,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.s_full[t], 1);
       mbar_init(&s.s_empty[t], kSoftmaxThreads);
     }
-    mbar_init(&s.p_full, kSoftmaxThreads);
-    mbar_init(&s.pv_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s.p_full[t], kSoftmaxThreads);
+      mbar_init(&s.pv_done[t], 1);
+    }
     mbar_init(&s.q_full, 1);
     mbar_init(&s.q_empty, 1);
     mbar_init(&s.o_full, 1);
     mbar_init(&s.o_empty, kSoftmaxThreads);
-    mbar_init(&s.drain, 1);
+    mbar_init(&s.drain[0], 1);
+    mbar_init(&s.drain[1], 1);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -201,11 +225,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------- K producer
-    if (lane == 0) produce_pairs<kKStages>(s, g, a, &maps.k, s.k, s.k_full, s.k_empty, abort_flag);
-  } else if (warp == 2) {
-    // ------------------------------------------------------------- V producer
-    if (lane == 0) produce_pairs<kVStages>(s, g, a, &maps.v, s.v, s.v_full, s.v_empty, abort_flag);
+    // ------------------------------------------------------------- K and V producer
+    if (lane == 0) produce_pairs(s, g, a, maps, abort_flag);
   } else if (warp == 3) {
     // ------------------------------------------------------------- Q producer
     if (lane == 0) {
@@ -226,96 +247,117 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (active > 0) mbar_wait(&s.q_full, (uint32_t)((active - 1) & 1), nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------- S issuer
+    // A thread's tcgen05.mma issue proceeds at about the rate the tensor pipe retires MMAs, so a
+    // thread that also waits on barriers leaves the pipe idle meanwhile: S and PV have one issuing
+    // thread each, and the pipe takes work from whichever is ready. tcgen05.commit tracks the MMAs
+    // of the committing thread only, which is what each barrier below needs.
     if (lane == 0) {
       int active = 0;  // units with at least one pair, in order
-      long gp0 = 0;    // global step index of the unit's first pair
+      long gp = 0;     // global step index
       bool ok = true;
       // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4 and
       // every buffer lies below 256 KB), so each MMA's operand is a base descriptor plus a constant.
       const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
-      const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
       const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
-      // S(gp) = Q . K_pair^T into S buffer gp & 1.
-      auto issue_s = [&](long gp, bool last_of_unit) -> bool {
-        const int ks = (int)(gp % kKStages);
-        const int b = (int)(gp & 1);
-        if (!mbar_wait(&s.k_full[ks], (uint32_t)((gp / kKStages) & 1), abort_flag) ||
-            !mbar_wait(&s.s_empty[b], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag))
-          return false;
-        tc_fence_after();
-        const uint64_t db0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
-        const uint32_t d_s = tmem + kColS + 128 * b;
-#pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
-          const int hh = kk >> 2, st = kk & 3;
-          mma_bf16(d_s, dq + ((hh * kTileBytes + st * 32) >> 4),
-                   db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
-        }
-        mma_commit(&s.s_full[b]);
-        mma_commit(&s.k_empty[ks]);
-        if (last_of_unit) mma_commit(&s.q_empty);
-        return true;
-      };
-      // O (+)= P . V_pair of step gp.
-      auto issue_pv = [&](long gp, bool first_of_unit, bool last_of_unit) -> bool {
-        const int vs = (int)(gp % kVStages);
-        if ((first_of_unit && !mbar_wait(&s.o_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) ||
-            !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
-            !mbar_wait(&s.p_full, (uint32_t)(gp & 1), abort_flag))
-          return false;
-        tc_fence_after();
-        const uint64_t db0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V) per MMA
-          mma_bf16_ts(tmem + kColO, tmem + kColP + 8 * kk, db0 + kk * (2048 >> 4), idesc_o,
-                      (first_of_unit && kk == 0) ? 0u : 1u);
-        mma_commit(&s.pv_done);
-        mma_commit(&s.v_empty[vs]);
-        if (last_of_unit) mma_commit(&s.o_full);
-        return true;
-      };
       for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
         const UnitInfo ui = unit_info(g, a, u);
         const int np = ui.npairs;
         if (np == 0) continue;
         if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        ok = issue_s(gp0, np == 1) && (np < 2 || issue_s(gp0 + 1, np == 2));
-        for (int n = 0; n < np && ok; ++n) {
-          // S(n + 2) only needs step n's S buffer, which the softmax frees as soon as it has read
-          // it, so it goes ahead of PV(n), which waits for the whole of step n's softmax.
-          if (n + 2 < np) ok = issue_s(gp0 + n + 2, n + 2 == np - 1);
-          if (ok) ok = issue_pv(gp0 + n, n == 0, n == np - 1);
+        for (int n = 0; n < np; ++n, ++gp) {
+          // S(gp) = Q . K_pair^T into S buffer gp & 1, once the softmax has read S(gp - 2).
+          const int ks = (int)(gp % kKStages);
+          const int b = (int)(gp & 1);
+          if (!mbar_wait(&s.k_full[ks], (uint32_t)((gp / kKStages) & 1), abort_flag) ||
+              !mbar_wait(&s.s_empty[b], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t db0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
+          const uint32_t d_s = tmem + kColS + 128 * b;
+#pragma unroll
+          for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
+            const int hh = kk >> 2, st = kk & 3;
+            mma_bf16(d_s, dq + ((hh * kTileBytes + st * 32) >> 4),
+                     db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
+          }
+          mma_commit(&s.s_full[b]);
+          mma_commit(&s.k_empty[ks]);
+          if (n == np - 1) mma_commit(&s.q_empty);
         }
-        if (!ok) break;
-        gp0 += np;
         ++active;
       }
       if (!ok) fail(s, a.dev_status);
       // Every MMA issued must complete before TMEM is released.
-      mma_commit(&s.drain);
-      mbar_wait(&s.drain, 0, nullptr);
+      mma_commit(&s.drain[0]);
+      mbar_wait(&s.drain[0], 0, nullptr);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------- PV issuer
+    if (lane == 0) {
+      int active = 0;
+      long gp = 0;
+      bool ok = true;
+      const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
+      for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
+        const UnitInfo ui = unit_info(g, a, u);
+        const int np = ui.npairs;
+        if (np == 0) continue;
+        for (int n = 0; n < np; ++n, ++gp) {
+          // O (+)= P . V_pair of step gp; the unit's first PV overwrites O once the epilogue of the
+          // previous unit has read it.
+          const int vs = (int)(gp % kVStages);
+          if ((n == 0 && !mbar_wait(&s.o_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) ||
+              !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
+              !mbar_wait(&s.p_full[gp & 1], (uint32_t)((gp >> 1) & 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t db0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V) per MMA
+            mma_bf16_ts(tmem + kColO, tmem + kColP + 64 * (uint32_t)(gp & 1) + 8 * kk,
+                        db0 + kk * (2048 >> 4), idesc_o, (n == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(&s.pv_done[gp & 1]);
+          mma_commit(&s.v_empty[vs]);
+          if (n == np - 1) mma_commit(&s.o_full);
+        }
+        ++active;
+      }
+      if (!ok) fail(s, a.dev_status);
+      mma_commit(&s.drain[1]);
+      mbar_wait(&s.drain[1], 0, nullptr);
     }
   } else if (warp >= 4) {
-    // ------------------------------------------------------------- softmax + epilogue (warps 4..7)
+    // ------------------------------------------------------------- softmax + epilogue (warps 4..11)
+    const int half = (warp - 4) >> 2;   // key tile of each pair, output columns 64 half ..
     const int sp = warp & 3;            // TMEM sub-partition: lanes [32 sp, 32 sp + 32)
+    const int bar_id = 1 + sp;          // named barrier of the warp pair (w, w + 4) on these lanes
     const int t0 = lane & 3;
-    const int r0 = 16 * sp + (lane >> 2), r1 = r0 + 8;  // this thread's two query rows
+    const int q4 = lane >> 2;           // row within the warp's 8-row group
+    const int r0 = 16 * sp + q4, r1 = r0 + 8;  // this thread's two query rows
     const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
     const long ld = (long)g.heads * kD;
+    const int col0 = 64 * half;         // first output column of this half
     int active = 0;
     long gp = 0;  // global step index
     bool reported = false;
-    bool failed = false;
-    for (int u = blockIdx.x; u < total_units && !failed; u += gridDim.x) {
+    bool failed = false;  // a bounded wait gave up; carried to the pair's next barrier
+    auto give_up = [&]() {  // every other wait of the CTA returns at once from here on
+      failed = true;
+      *abort_flag = 1;
+    };
+    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
       const UnitInfo ui = unit_info(g, a, u);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
       const int vci = s.vc[ui.i];
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
       if (ui.npairs == 0) {
-        // No kept key tile: this thread's two output rows are zero.
-        for (int c = 2 * t0; c < kD; c += 8) {
+        // No kept key tile: this thread's two output rows are zero (this half's columns).
+        for (int c = col0 + 2 * t0; c < col0 + 64; c += 8) {
           *reinterpret_cast<uint32_t*>(out + r0 * ld + c) = 0u;
           *reinterpret_cast<uint32_t*>(out + r1 * ld + c) = 0u;
         }
@@ -323,50 +365,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       float m0 = -INFINITY, m1 = -INFINITY;  // shifts (log2 units) of rows r0, r1
       float l0 = 0.f, l1 = 0.f;              // running sums over this thread's columns
-      // Key tiles of the first step (list entries are prefetched a step ahead).
-      int ea = (0 < ui.cnt) ? ui.list[0] : kAbsent, eb = (1 < ui.cnt) ? ui.list[1] : kAbsent;
+      // This half's key tile of the first step (list entries are prefetched a step ahead).
+      int e_next = (half < ui.cnt) ? ui.list[half] : kAbsent;
+      bool stop = false;
       for (int n = 0; n < ui.npairs; ++n, ++gp) {
-        const int ja = ea, jb = eb;
-        ea = (2 * n + 2 < ui.cnt) ? ui.list[2 * n + 2] : kAbsent;
-        eb = (2 * n + 3 < ui.cnt) ? ui.list[2 * n + 3] : kAbsent;
+        const int jt = e_next;
+        e_next = (2 * n + 2 + half < ui.cnt) ? ui.list[2 * n + 2 + half] : kAbsent;
         const int b = (int)(gp & 1);
-        bool ok = mbar_wait(&s.s_full[b], (uint32_t)((gp >> 1) & 1), abort_flag);
+        if (!mbar_wait(&s.s_full[b], (uint32_t)((gp >> 1) & 1), abort_flag)) give_up();
         tc_fence_after();
-        uint32_t v[64];
-        tmem_ld_16x256b_x16(lane_base + kColS + 128 * b, v);
+        uint32_t v[32];
+        tmem_ld_16x256b_x8(lane_base + kColS + 128 * b + col0, v);
         tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(&s.s_empty[b]);
-        // Valid keys: tile a gives keys 0..63, tile b keys 64..127.
-        const bool ina = ja >= 0 && ja < g.nT, inb = jb >= 0 && jb < g.nT;
-        if (!reported && ((ja != kAbsent && !ina) || (jb != kAbsent && !inb))) {
+        // Valid keys of this half's tile: 0 .. vc - 1.
+        const bool in = jt >= 0 && jt < g.nT;
+        if (!reported && jt != kAbsent && !in) {
           report(a.dev_status, T3D_DEV_INDEX_RANGE);
           reported = true;
         }
-        const int ca = ina ? s.vc[ja] : 0, cb = inb ? s.vc[jb] : 0;
-        if (ca < kTileElems || cb < kTileElems) {
+        const int cv = in ? s.vc[jt] : 0;
+        if (cv < kTileElems) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int key = 8 * j + 2 * t0 + e;  // 0..127
-              const bool valid = key < 64 ? key < ca : key - 64 < cb;
-              if (!valid) {
+              if (8 * j + 2 * t0 + e >= cv) {
                 v[4 * j + e] = __float_as_uint(-INFINITY);
                 v[4 * j + 2 + e] = __float_as_uint(-INFINITY);
               }
             }
           }
         }
-        // Row maxima (the 4 threads of a row hold its 128 columns), as balanced trees.
-        float t0r[16], t1r[16];
+        // Row maxima over this half's 64 columns (4 threads per row), as balanced trees.
+        float t0r[8], t1r[8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           t0r[j] = fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]));
           t1r[j] = fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
         }
 #pragma unroll
-        for (int w = 8; w >= 1; w >>= 1)
+        for (int w = 4; w >= 1; w >>= 1)
 #pragma unroll
           for (int j = 0; j < w; ++j) {
             t0r[j] = fmaxf(t0r[j], t0r[j + w]);
@@ -377,14 +417,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
         x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 1));
         x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2));
-        x0 *= sl2;  // log2 units (the scale is positive)
-        x1 *= sl2;
+        // Swap the row maxima with the other half; the barrier also ORs the failure flags, so both
+        // warps of the pair leave together.
+        if (t0 == 0) {
+          s.xmax[b][half][sp][q4] = x0;
+          s.xmax[b][half][sp][q4 + 8] = x1;
+        }
+        if (named_bar_or(bar_id, 64, failed)) {
+          failed = true;
+          stop = true;
+          break;
+        }
+        x0 = fmaxf(x0, s.xmax[b][half ^ 1][sp][q4]) * sl2;  // log2 units (the scale is positive)
+        x1 = fmaxf(x1, s.xmax[b][half ^ 1][sp][q4 + 8]) * sl2;
         const bool up0 = x0 > m0 + kShiftSlack || (m0 == -INFINITY && x0 > -INFINITY);
         const bool up1 = x1 > m1 + kShiftSlack || (m1 == -INFINITY && x1 > -INFINITY);
-        if (__any_sync(0xffffffffu, !ok)) { failed = true; break; }
-        // P (and O) may only be rewritten once the previous step's PV MMAs have landed; the wait
-        // is taken as late as possible (before a rescale of O, else before the P store).
-        bool pv_waited = gp == 0;
+        // O may only be rescaled once the previous step's PV MMAs have landed, and this step's P
+        // buffer rewritten once the PV of two steps back has.
         if (__any_sync(0xffffffffu, up0 || up1)) {
           const float n0 = up0 ? fmaxf(m0, x0) : m0, n1 = up1 ? fmaxf(m1, x1) : m1;
           const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - n0);
@@ -394,115 +443,127 @@ __global__ void __launch_bounds__(kThreads, 1)
           m0 = n0;
           m1 = n1;
           if (n > 0) {
-            // Rescale the O rows of this warp's queries (factor 1 where the shift did not move).
-            const bool pv_ok = mbar_wait(&s.pv_done, (uint32_t)((gp - 1) & 1), abort_flag);
-            if (__any_sync(0xffffffffu, !pv_ok)) { failed = true; break; }
-            pv_waited = true;
+            // Rescale this half's O columns of the warp's rows (factor 1 where the shift held).
+            if (!mbar_wait(&s.pv_done[(gp - 1) & 1], (uint32_t)(((gp - 1) >> 1) & 1), abort_flag))
+              give_up();
             tc_fence_after();
+            uint32_t o[32];
+            tmem_ld_16x256b_x8(lane_base + kColO + col0, o);
+            tmem_wait_ld();
 #pragma unroll
-            for (int hc = 0; hc < 2; ++hc) {
-              uint32_t o[32];
-              tmem_ld_16x256b_x8(lane_base + kColO + 64 * hc, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                o[4 * j] = __float_as_uint(__uint_as_float(o[4 * j]) * a0);
-                o[4 * j + 1] = __float_as_uint(__uint_as_float(o[4 * j + 1]) * a0);
-                o[4 * j + 2] = __float_as_uint(__uint_as_float(o[4 * j + 2]) * a1);
-                o[4 * j + 3] = __float_as_uint(__uint_as_float(o[4 * j + 3]) * a1);
-              }
-              tmem_st_16x256b_x8(lane_base + kColO + 64 * hc, o);
+            for (int j = 0; j < 8; ++j) {
+              o[4 * j] = __float_as_uint(__uint_as_float(o[4 * j]) * a0);
+              o[4 * j + 1] = __float_as_uint(__uint_as_float(o[4 * j + 1]) * a0);
+              o[4 * j + 2] = __float_as_uint(__uint_as_float(o[4 * j + 2]) * a1);
+              o[4 * j + 3] = __float_as_uint(__uint_as_float(o[4 * j + 3]) * a1);
             }
+            tmem_st_16x256b_x8(lane_base + kColO + col0, o);
             tmem_wait_st();
           }
         }
-        // P = exp2(x * scale - shift), packed as bf16 pairs (keys 8j + 2 t0, + 1 -> column 4j + t0).
+        // P = exp2(x * scale - shift) as bf16 pairs: keys 8j + 2 t0, + 1 of this half go to P
+        // column 32 half + 4j + t0 (the layout tcgen05.st 16x128b writes).
         const float ns0 = m0 == -INFINITY ? 0.f : -m0, ns1 = m1 == -INFINITY ? 0.f : -m1;
-        uint32_t pw[32];
-        float ls0[4] = {0.f, 0.f, 0.f, 0.f}, ls1[4] = {0.f, 0.f, 0.f, 0.f};
+        uint32_t pw[16];
+        float ls0[2] = {0.f, 0.f}, ls1[2] = {0.f, 0.f};
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           const float p00 = ex2(fmaf(__uint_as_float(v[4 * j]), sl2, ns0));
           const float p01 = ex2(fmaf(__uint_as_float(v[4 * j + 1]), sl2, ns0));
           const float p10 = ex2(fmaf(__uint_as_float(v[4 * j + 2]), sl2, ns1));
           const float p11 = ex2(fmaf(__uint_as_float(v[4 * j + 3]), sl2, ns1));
-          ls0[j & 3] += p00 + p01;
-          ls1[j & 3] += p10 + p11;
+          ls0[j & 1] += p00 + p01;
+          ls1[j & 1] += p10 + p11;
           __nv_bfloat162 q0 = __floats2bfloat162_rn(p00, p01);
           __nv_bfloat162 q1 = __floats2bfloat162_rn(p10, p11);
           pw[2 * j] = *reinterpret_cast<uint32_t*>(&q0);
           pw[2 * j + 1] = *reinterpret_cast<uint32_t*>(&q1);
         }
-        if (!pv_waited) {
-          const bool pv_ok = mbar_wait(&s.pv_done, (uint32_t)((gp - 1) & 1), abort_flag);
-          if (__any_sync(0xffffffffu, !pv_ok)) { failed = true; break; }
+        l0 += ls0[0] + ls0[1];
+        l1 += ls1[0] + ls1[1];
+        if (gp >= 2) {
+          if (!mbar_wait(&s.pv_done[b], (uint32_t)(((gp - 2) >> 1) & 1), abort_flag)) give_up();
           tc_fence_after();
         }
-        l0 += (ls0[0] + ls0[1]) + (ls0[2] + ls0[3]);
-        l1 += (ls1[0] + ls1[1]) + (ls1[2] + ls1[3]);
-        tmem_st_16x128b_x16(lane_base + kColP, pw);
+        tmem_st_16x128b_x8(lane_base + kColP + 64 * b + 32 * half, pw);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&s.p_full);
+        mbar_arrive(&s.p_full[b]);
       }
-      if (failed) break;
+      if (stop) break;
       // ---- epilogue: O / l for this thread's rows, bf16, into the tiled output
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      if (t0 == 0) {
+        s.xsum[half][sp][q4] = l0;
+        s.xsum[half][sp][q4 + 8] = l1;
+      }
+      if (named_bar_or(bar_id, 64, failed)) {
+        failed = true;
+        break;
+      }
+      l0 += s.xsum[half ^ 1][sp][q4];
+      l1 += s.xsum[half ^ 1][sp][q4 + 8];
+      // The sums are read before either warp of the pair can write them again: the next write
+      // follows at least one more pair barrier (every unit that reaches here has a step).
       const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-      const bool ook = mbar_wait(&s.o_full, (uint32_t)(active & 1), abort_flag);
-      if (__any_sync(0xffffffffu, !ook)) { failed = true; break; }
+      if (!mbar_wait(&s.o_full, (uint32_t)(active & 1), abort_flag)) give_up();
       tc_fence_after();
-      // O rows are read with the 32-lane shape: lane L < 16 of this warp holds row 16 sp + L (the
-      // M = 64 layout), 32 columns per load, so a row goes out in 16-byte stores. Its 1 / l comes
-      // from the threads that own the row in the 16x256b layout (row r0 of lanes 4L.., or r1).
-      const int rown = 16 * sp + (lane & 15);
-      const float ia = __shfl_sync(0xffffffffu, i0, 4 * (lane & 7));
-      const float ib = __shfl_sync(0xffffffffu, i1, 4 * (lane & 7));
-      const float inv = (lane & 15) < 8 ? ia : ib;
-      const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
-      const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
-      const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
+      failed = __any_sync(0xffffffffu, failed);  // the TMEM loads below are warp-collective
+      if (!failed) {
+        // O rows are read with the 32-lane shape: lane L < 16 of this warp holds row 16 sp + L
+        // (the M = 64 layout), 32 columns per load, so a row goes out in 16-byte stores. Its 1 / l
+        // comes from the threads that own the row in the 16x256b layout (row r0 of lanes 4L.., or
+        // r1).
+        const int rown = 16 * sp + (lane & 15);
+        const float ia = __shfl_sync(0xffffffffu, i0, 4 * (lane & 7));
+        const float ib = __shfl_sync(0xffffffffu, i1, 4 * (lane & 7));
+        const float inv = (lane & 15) < 8 ? ia : ib;
+        const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
+        const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
+        const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
 #pragma unroll
-      for (int c = 0; c < kD / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(lane_base + kColO + 32 * c, o);
-        tmem_wait_ld();
-        if (lane < 16) {
-          uint4 w4[4];
-          uint32_t* w = reinterpret_cast<uint32_t*>(w4);
+        for (int c = 0; c < 2; ++c) {
+          const int cc = col0 + 32 * c;
+          uint32_t o[32];
+          tmem_ld32(lane_base + kColO + cc, o);
+          tmem_wait_ld();
+          if (lane < 16) {
+            uint4 w4[4];
+            uint32_t* w = reinterpret_cast<uint32_t*>(w4);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 y = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
-                                                     __uint_as_float(o[2 * e + 1]) * inv);
-            w[e] = *reinterpret_cast<uint32_t*>(&y);
-          }
-          // Row rr of the output takes the result of row src(rr): rr itself, or for a query row
-          // pruned by BSA its kept source row. Rows past the tile's valid count are zero.
-          auto put = [&](int rr) {
-            uint4* dst = reinterpret_cast<uint4*>(out + rr * ld + 32 * c);
-            const bool zero = rr >= vci;
+            for (int e = 0; e < 16; ++e) {
+              __nv_bfloat162 y = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
+                                                       __uint_as_float(o[2 * e + 1]) * inv);
+              w[e] = *reinterpret_cast<uint32_t*>(&y);
+            }
+            // Row rr of the output takes the result of row src(rr): rr itself, or for a query row
+            // pruned by BSA its kept source row. Rows past the tile's valid count are zero.
+            auto put = [&](int rr) {
+              uint4* dst = reinterpret_cast<uint4*>(out + rr * ld + cc);
+              const bool zero = rr >= vci;
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) dst[q4] = zero ? make_uint4(0u, 0u, 0u, 0u) : w4[q4];
-          };
-          if (keep == nullptr) {
-            put(rown);
-          } else {
-            for (int rr = 0; rr < kTileElems; ++rr) {
-              int sr = rr;
-              if (!keep[rr]) {
-                sr = srcr[rr];
-                if (sr >= kTileElems) sr = rr;
+              for (int k4 = 0; k4 < 4; ++k4) dst[k4] = zero ? make_uint4(0u, 0u, 0u, 0u) : w4[k4];
+            };
+            if (keep == nullptr) {
+              put(rown);
+            } else {
+              for (int rr = 0; rr < kTileElems; ++rr) {
+                int sr = rr;
+                if (!keep[rr]) {
+                  sr = srcr[rr];
+                  if (sr >= kTileElems) sr = rr;
+                }
+                if (sr == rown) put(rr);
               }
-              if (sr == rown) put(rr);
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(&s.o_empty);
       }
-      tc_fence_before();
-      mbar_arrive(&s.o_empty);
       ++active;
     }
     if (failed && lane == 0) fail(s, a.dev_status);
