@@ -25,22 +25,22 @@
 //   warp 2       one thread issues the PV MMAs and their commits
 //   warp 3       TMA producer for each unit's query tile (one buffer, refilled once the previous
 //                unit's last S has completed, so the next unit's scores start during the epilogue)
-//   warps 4..11  softmax and epilogue, two halves of 4 warps: half h takes key tile h of every pair
-//                (score columns 64 h .. 64 h + 63) and output columns 64 h .. 64 h + 63. Thread t of
-//                warp w owns query rows 16 (w % 4) + t/4 and that + 8, and the key columns
-//                64 h + 8j + 2(t%4) + {0, 1} (tcgen05.ld 16x256b). Warps w and w + 4 read the same
-//                TMEM lanes and pair up through shared memory.
+//   warps 4..11  softmax and epilogue, two warpgroups: warpgroup X takes the steps n with n % 2 == X
+//                (S and P buffer X) and, in the epilogue, output columns 64 X .. 64 X + 63. Thread t
+//                of warp w owns query rows 16 (w % 4) + t/4 and that + 8, and the key columns
+//                8j + 2(t%4) + {0, 1} of its steps (tcgen05.ld 16x256b).
 // S(n) is issued as soon as its K pair has landed and the softmax has read S(n - 2), so scores run
 // up to two steps ahead; PV(n) as soon as P(n) is in TMEM.
 //
-// Softmax. A row's online-softmax state (shift m, running sum l) lives with the 8 threads that
-// share the row, 4 in each half: each half reduces its 64 columns with two shuffles, and the two
-// halves swap their row maxima through shared memory (one 64-thread named barrier per warp pair and
-// step), so both raise the shift identically and keep partial sums of their own columns. The shift
-// (log2 units) is raised only when a row's logits exceed it by more than kShiftSlack; each half then
-// rescales its O columns of the rows concerned in TMEM (factor 1 for rows that did not move) once
-// the previous PV has landed. Any shift gives the same softmax; the bound keeps P within
-// [0, 2^kShiftSlack] so nothing overflows. Two warps per scheduler overlap each other's latencies.
+// Softmax. The two warpgroups alternate steps, so each has two steps' time for one and their
+// phases interleave: one computes exponentials while the other loads scores or reduces maxima.
+// The per-row shift m (log2 units) is a chain along the steps: step n takes the shift after step
+// n - 1 from the other warpgroup through shared memory (an mbarrier per parity), raises it only when
+// a row's logits exceed it by more than kShiftSlack, publishes it, and then rescales the O rows
+// concerned in TMEM (factor 1 for rows that did not move) once PV(n - 1) has landed. Any shift gives
+// the same softmax; the bound keeps P within [0, 2^kShiftSlack] so nothing overflows. Each
+// warpgroup keeps the running sums of its own steps relative to the last shift it used; the
+// epilogue brings both to the final (largest) shift and adds them.
 //
 // Every mbarrier wait is bounded; on a timeout the CTA records T3D_DEV_TIMEOUT, stops issuing work,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and returns. The two warps of a pair
@@ -58,7 +58,14 @@ constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a 
 constexpr int kKStages = 3;         // K-pair ring depth
 constexpr int kVStages = 3;         // V-pair ring depth
 constexpr int kThreads = 384;       // 12 warps: producers / MMA, two softmax halves
-constexpr int kSoftmaxThreads = 256;
+constexpr int kSoftmaxThreads = 256;  // both softmax warpgroups
+constexpr int kWgThreads = 128;       // one softmax warpgroup
+constexpr int kTeardownBar = 5;       // named barrier of all threads before TMEM is released
+constexpr int kLaunchRegs = 168;      // 65536 / 384, rounded down to a multiple of 8
+constexpr int kProducerRegs = 56;
+constexpr int kSoftmaxRegs = 224;
+static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs,
+              "register split exceeds the launch allocation");
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;       // S buffer b at 128 b
@@ -83,8 +90,10 @@ struct alignas(1024) SmemLayout {
   uint64_t o_full;    // the unit's last PV complete (MMA -> softmax)
   uint64_t o_empty;   // O read by the epilogue (softmax -> MMA)
   uint64_t drain[2];  // all MMAs of the S issuer / the PV issuer complete
-  float xmax[2][2][4][16];  // [step & 1][half][warp % 4][row]: row maxima swapped between halves
-  float xsum[2][4][16];     // [half][warp % 4][row]: row sums swapped at the end of a unit
+  uint64_t m_ready[2];      // shift of a step (parity b) published by warpgroup b
+  float mrow[2][64];        // [step & 1][row]: that shift
+  float xsum[2][2][4][16];  // [unit & 1][warpgroup][warp % 4][row]: running sums, end of a unit
+  float xm[2][2][4][16];    // [unit & 1][warpgroup][warp % 4][row]: the shift they are relative to
   uint8_t vc[kMaxTiles];    // valid token count of every tile
   uint32_t tmem_base;
   int abort;
@@ -194,10 +203,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < kVStages; ++t) { mbar_init(&s.v_full[t], 1); mbar_init(&s.v_empty[t], 1); }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.s_full[t], 1);
-      mbar_init(&s.s_empty[t], kSoftmaxThreads);
+      mbar_init(&s.s_empty[t], kWgThreads);
     }
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&s.p_full[t], kSoftmaxThreads);
+      mbar_init(&s.p_full[t], kWgThreads);
+      mbar_init(&s.m_ready[t], kWgThreads);
       mbar_init(&s.pv_done[t], 1);
     }
     mbar_init(&s.q_full, 1);
@@ -223,127 +233,139 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------- K and V producer
-    if (lane == 0) produce_pairs(s, g, a, maps, abort_flag);
-  } else if (warp == 3) {
-    // ------------------------------------------------------------- Q producer
-    if (lane == 0) {
-      int active = 0;
-      bool ok = true;
-      for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
-        const UnitInfo ui = unit_info(g, a, u);
-        if (ui.npairs == 0) continue;
-        if (!mbar_wait(&s.q_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) { ok = false; break; }
-        mbar_expect_tx(&s.q_full, kQBytes);
-        const int row0 = ui.b * g.Lp + ui.i * kTileElems;
-        for (int hh = 0; hh < kHalves; ++hh)
-          tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
-        ++active;
-      }
-      if (!ok) fail(s, a.dev_status);
-      // Drain: the last query tile loaded must land before the CTA can exit.
-      if (active > 0) mbar_wait(&s.q_full, (uint32_t)((active - 1) & 1), nullptr);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- S issuer
-    // A thread's tcgen05.mma issue proceeds at about the rate the tensor pipe retires MMAs, so a
-    // thread that also waits on barriers leaves the pipe idle meanwhile: S and PV have one issuing
-    // thread each, and the pipe takes work from whichever is ready. tcgen05.commit tracks the MMAs
-    // of the committing thread only, which is what each barrier below needs.
-    if (lane == 0) {
-      int active = 0;  // units with at least one pair, in order
-      long gp = 0;     // global step index
-      bool ok = true;
-      // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4 and
-      // every buffer lies below 256 KB), so each MMA's operand is a base descriptor plus a constant.
-      const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
-      const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
-      for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
-        const UnitInfo ui = unit_info(g, a, u);
-        const int np = ui.npairs;
-        if (np == 0) continue;
-        if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag)) { ok = false; break; }
-        for (int n = 0; n < np; ++n, ++gp) {
-          // S(gp) = Q . K_pair^T into S buffer gp & 1, once the softmax has read S(gp - 2).
-          const int ks = (int)(gp % kKStages);
-          const int b = (int)(gp & 1);
-          if (!mbar_wait(&s.k_full[ks], (uint32_t)((gp / kKStages) & 1), abort_flag) ||
-              !mbar_wait(&s.s_empty[b], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t db0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
-          const uint32_t d_s = tmem + kColS + 128 * b;
-#pragma unroll
-          for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
-            const int hh = kk >> 2, st = kk & 3;
-            mma_bf16(d_s, dq + ((hh * kTileBytes + st * 32) >> 4),
-                     db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
-          }
-          mma_commit(&s.s_full[b]);
-          mma_commit(&s.k_empty[ks]);
-          if (n == np - 1) mma_commit(&s.q_empty);
+  // Registers move from the producer / issuer warpgroup to the softmax warpgroups: 384 threads
+  // launch with 168 each; 128 x 56 + 256 x 224 is the same total. The two sides never share code
+  // after the split (each ends with its own arrival at the teardown barrier).
+  if (warp < 4) {
+    regs_dec<kProducerRegs>();
+    if (warp == 0) {
+      // ------------------------------------------------------------- K and V producer
+      if (lane == 0) produce_pairs(s, g, a, maps, abort_flag);
+    } else if (warp == 3) {
+      // ------------------------------------------------------------- Q producer
+      if (lane == 0) {
+        int active = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
+          const UnitInfo ui = unit_info(g, a, u);
+          if (ui.npairs == 0) continue;
+          if (!mbar_wait(&s.q_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&s.q_full, kQBytes);
+          const int row0 = ui.b * g.Lp + ui.i * kTileElems;
+          for (int hh = 0; hh < kHalves; ++hh)
+            tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
+          ++active;
         }
-        ++active;
+        if (!ok) fail(s, a.dev_status);
+        // Drain: the last query tile loaded must land before the CTA can exit.
+        if (active > 0) mbar_wait(&s.q_full, (uint32_t)((active - 1) & 1), nullptr);
       }
-      if (!ok) fail(s, a.dev_status);
-      // Every MMA issued must complete before TMEM is released.
-      mma_commit(&s.drain[0]);
-      mbar_wait(&s.drain[0], 0, nullptr);
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------- PV issuer
-    if (lane == 0) {
-      int active = 0;
-      long gp = 0;
-      bool ok = true;
-      const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
-      for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
-        const UnitInfo ui = unit_info(g, a, u);
-        const int np = ui.npairs;
-        if (np == 0) continue;
-        for (int n = 0; n < np; ++n, ++gp) {
-          // O (+)= P . V_pair of step gp; the unit's first PV overwrites O once the epilogue of the
-          // previous unit has read it.
-          const int vs = (int)(gp % kVStages);
-          if ((n == 0 && !mbar_wait(&s.o_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) ||
-              !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
-              !mbar_wait(&s.p_full[gp & 1], (uint32_t)((gp >> 1) & 1), abort_flag)) {
-            ok = false;
-            break;
+    } else if (warp == 1) {
+      // ------------------------------------------------------------- S issuer
+      // A thread's tcgen05.mma issue proceeds at about the rate the tensor pipe retires MMAs, so a
+      // thread that also waits on barriers leaves the pipe idle meanwhile: S and PV have one issuing
+      // thread each, and the pipe takes work from whichever is ready. tcgen05.commit tracks the MMAs
+      // of the committing thread only, which is what each barrier below needs.
+      if (lane == 0) {
+        int active = 0;  // units with at least one pair, in order
+        long gp = 0;     // global step index
+        bool ok = true;
+        // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4 and
+        // every buffer lies below 256 KB), so each MMA's operand is a base descriptor plus a constant.
+        const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
+        const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
+        for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
+          const UnitInfo ui = unit_info(g, a, u);
+          const int np = ui.npairs;
+          if (np == 0) continue;
+          if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag)) { ok = false; break; }
+          for (int n = 0; n < np; ++n, ++gp) {
+            // S(gp) = Q . K_pair^T into S buffer gp & 1, once the softmax has read S(gp - 2).
+            const int ks = (int)(gp % kKStages);
+            const int b = (int)(gp & 1);
+            if (!mbar_wait(&s.k_full[ks], (uint32_t)((gp / kKStages) & 1), abort_flag) ||
+                !mbar_wait(&s.s_empty[b], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t db0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
+            const uint32_t d_s = tmem + kColS + 128 * b;
+  #pragma unroll
+            for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
+              const int hh = kk >> 2, st = kk & 3;
+              mma_bf16(d_s, dq + ((hh * kTileBytes + st * 32) >> 4),
+                       db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
+            }
+            mma_commit(&s.s_full[b]);
+            mma_commit(&s.k_empty[ks]);
+            if (n == np - 1) mma_commit(&s.q_empty);
           }
-          tc_fence_after();
-          const uint64_t db0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V) per MMA
-            mma_bf16_ts(tmem + kColO, tmem + kColP + 64 * (uint32_t)(gp & 1) + 8 * kk,
-                        db0 + kk * (2048 >> 4), idesc_o, (n == 0 && kk == 0) ? 0u : 1u);
-          mma_commit(&s.pv_done[gp & 1]);
-          mma_commit(&s.v_empty[vs]);
-          if (n == np - 1) mma_commit(&s.o_full);
+          ++active;
         }
-        ++active;
+        if (!ok) fail(s, a.dev_status);
+        // Every MMA issued must complete before TMEM is released.
+        mma_commit(&s.drain[0]);
+        mbar_wait(&s.drain[0], 0, nullptr);
       }
-      if (!ok) fail(s, a.dev_status);
-      mma_commit(&s.drain[1]);
-      mbar_wait(&s.drain[1], 0, nullptr);
+    } else if (warp == 2) {
+      // ------------------------------------------------------------- PV issuer
+      if (lane == 0) {
+        int active = 0;
+        long gp = 0;
+        bool ok = true;
+        const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
+        for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
+          const UnitInfo ui = unit_info(g, a, u);
+          const int np = ui.npairs;
+          if (np == 0) continue;
+          for (int n = 0; n < np; ++n, ++gp) {
+            // O (+)= P . V_pair of step gp; the unit's first PV overwrites O once the epilogue of the
+            // previous unit has read it.
+            const int vs = (int)(gp % kVStages);
+            if ((n == 0 && !mbar_wait(&s.o_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) ||
+                !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
+                !mbar_wait(&s.p_full[gp & 1], (uint32_t)((gp >> 1) & 1), abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t db0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
+  #pragma unroll
+            for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V) per MMA
+              mma_bf16_ts(tmem + kColO, tmem + kColP + 64 * (uint32_t)(gp & 1) + 8 * kk,
+                          db0 + kk * (2048 >> 4), idesc_o, (n == 0 && kk == 0) ? 0u : 1u);
+            mma_commit(&s.pv_done[gp & 1]);
+            mma_commit(&s.v_empty[vs]);
+            if (n == np - 1) mma_commit(&s.o_full);
+          }
+          ++active;
+        }
+        if (!ok) fail(s, a.dev_status);
+        mma_commit(&s.drain[1]);
+        mbar_wait(&s.drain[1], 0, nullptr);
+      }
     }
-  } else if (warp >= 4) {
+    tc_fence_before();
+    named_bar(kTeardownBar, kThreads);
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  } else {
+    regs_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------- softmax + epilogue (warps 4..11)
-    const int half = (warp - 4) >> 2;   // key tile of each pair, output columns 64 half ..
+    const int wg = (warp - 4) >> 2;     // this warpgroup takes the steps gp with gp & 1 == wg
     const int sp = warp & 3;            // TMEM sub-partition: lanes [32 sp, 32 sp + 32)
-    const int bar_id = 1 + sp;          // named barrier of the warp pair (w, w + 4) on these lanes
+    const int bar_id = 1 + sp;          // named barrier of warps w and w + 4 (same TMEM lanes)
     const int t0 = lane & 3;
     const int q4 = lane >> 2;           // row within the warp's 8-row group
     const int r0 = 16 * sp + q4, r1 = r0 + 8;  // this thread's two query rows
     const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
+    const uint32_t t_s = lane_base + kColS + 128 * (uint32_t)wg;  // this warpgroup's S buffer
+    const uint32_t t_p = lane_base + kColP + 64 * (uint32_t)wg;   // and P buffer
     const long ld = (long)g.heads * kD;
-    const int col0 = 64 * half;         // first output column of this half
+    const int col0 = 64 * wg;           // output columns this warpgroup writes
     int active = 0;
-    long gp = 0;  // global step index
+    long gp = 0;  // global index of the unit's first step
     bool reported = false;
     bool failed = false;  // a bounded wait gave up; carried to the pair's next barrier
     auto give_up = [&]() {  // every other wait of the CTA returns at once from here on
@@ -356,99 +378,114 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int vci = s.vc[ui.i];
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
       if (ui.npairs == 0) {
-        // No kept key tile: this thread's two output rows are zero (this half's columns).
+        // No kept key tile: this thread's two output rows are zero (this warpgroup's columns).
         for (int c = col0 + 2 * t0; c < col0 + 64; c += 8) {
           *reinterpret_cast<uint32_t*>(out + r0 * ld + c) = 0u;
           *reinterpret_cast<uint32_t*>(out + r1 * ld + c) = 0u;
         }
         continue;
       }
-      float m0 = -INFINITY, m1 = -INFINITY;  // shifts (log2 units) of rows r0, r1
-      float l0 = 0.f, l1 = 0.f;              // running sums over this thread's columns
-      // This half's key tile of the first step (list entries are prefetched a step ahead).
-      int e_next = (half < ui.cnt) ? ui.list[half] : kAbsent;
-      bool stop = false;
-      for (int n = 0; n < ui.npairs; ++n, ++gp) {
-        const int jt = e_next;
-        e_next = (2 * n + 2 + half < ui.cnt) ? ui.list[2 * n + 2 + half] : kAbsent;
-        const int b = (int)(gp & 1);
-        if (!mbar_wait(&s.s_full[b], (uint32_t)((gp >> 1) & 1), abort_flag)) give_up();
+      // mw: the shift this warpgroup used at its latest step of the unit; l is relative to it.
+      float mw0 = -INFINITY, mw1 = -INFINITY;
+      float l0 = 0.f, l1 = 0.f;  // sums over this thread's columns of this warpgroup's steps
+      const int nfirst = (int)((wg ^ (int)(gp & 1)) & 1);  // first step of the unit that is ours
+      // Key tiles of our next step (prefetched one own step ahead).
+      int ea = (2 * nfirst < ui.cnt) ? ui.list[2 * nfirst] : kAbsent;
+      int eb = (2 * nfirst + 1 < ui.cnt) ? ui.list[2 * nfirst + 1] : kAbsent;
+      for (int n = nfirst; n < ui.npairs; n += 2) {
+        const long gs = gp + n;  // global step index; gs & 1 == wg
+        const int ja = ea, jb = eb;
+        ea = (2 * n + 4 < ui.cnt) ? ui.list[2 * n + 4] : kAbsent;
+        eb = (2 * n + 5 < ui.cnt) ? ui.list[2 * n + 5] : kAbsent;
+        if (!mbar_wait(&s.s_full[wg], (uint32_t)((gs >> 1) & 1), abort_flag)) give_up();
         tc_fence_after();
-        uint32_t v[32];
-        tmem_ld_16x256b_x8(lane_base + kColS + 128 * b + col0, v);
+        uint32_t v[64];
+        tmem_ld_16x256b_x16(t_s, v);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&s.s_empty[b]);
-        // Valid keys of this half's tile: 0 .. vc - 1.
-        const bool in = jt >= 0 && jt < g.nT;
-        if (!reported && jt != kAbsent && !in) {
+        mbar_arrive(&s.s_empty[wg]);
+        // Valid keys: tile a gives keys 0..63, tile b keys 64..127.
+        const bool ina = ja >= 0 && ja < g.nT, inb = jb >= 0 && jb < g.nT;
+        if (!reported && ((ja != kAbsent && !ina) || (jb != kAbsent && !inb))) {
           report(a.dev_status, T3D_DEV_INDEX_RANGE);
           reported = true;
         }
-        const int cv = in ? s.vc[jt] : 0;
-        if (cv < kTileElems) {
+        const int ca = ina ? s.vc[ja] : 0, cb = inb ? s.vc[jb] : 0;
+        if (ca < kTileElems || cb < kTileElems) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 16; ++j) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              if (8 * j + 2 * t0 + e >= cv) {
+              const int key = 8 * j + 2 * t0 + e;  // 0..127
+              const bool valid = key < 64 ? key < ca : key - 64 < cb;
+              if (!valid) {
                 v[4 * j + e] = __float_as_uint(-INFINITY);
                 v[4 * j + 2 + e] = __float_as_uint(-INFINITY);
               }
             }
           }
         }
-        // Row maxima over this half's 64 columns (4 threads per row), as balanced trees.
-        float t0r[8], t1r[8];
+        // Row maxima (the 4 threads of a row hold its 128 columns), as balanced trees.
+        float x0, x1;
+        {
+          float t0r[16], t1r[16];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          t0r[j] = fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]));
-          t1r[j] = fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-        }
-#pragma unroll
-        for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-          for (int j = 0; j < w; ++j) {
-            t0r[j] = fmaxf(t0r[j], t0r[j + w]);
-            t1r[j] = fmaxf(t1r[j], t1r[j + w]);
+          for (int j = 0; j < 16; ++j) {
+            t0r[j] = fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]));
+            t1r[j] = fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
           }
-        float x0 = t0r[0], x1 = t1r[0];
+#pragma unroll
+          for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+            for (int j = 0; j < w; ++j) {
+              t0r[j] = fmaxf(t0r[j], t0r[j + w]);
+              t1r[j] = fmaxf(t1r[j], t1r[j + w]);
+            }
+          x0 = t0r[0];
+          x1 = t1r[0];
+        }
         x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
         x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
         x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 1));
         x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2));
-        // Swap the row maxima with the other half; the barrier also ORs the failure flags, so both
-        // warps of the pair leave together.
-        if (t0 == 0) {
-          s.xmax[b][half][sp][q4] = x0;
-          s.xmax[b][half][sp][q4 + 8] = x1;
-        }
-        if (named_bar_or(bar_id, 64, failed)) {
-          failed = true;
-          stop = true;
-          break;
-        }
-        x0 = fmaxf(x0, s.xmax[b][half ^ 1][sp][q4]) * sl2;  // log2 units (the scale is positive)
-        x1 = fmaxf(x1, s.xmax[b][half ^ 1][sp][q4 + 8]) * sl2;
-        const bool up0 = x0 > m0 + kShiftSlack || (m0 == -INFINITY && x0 > -INFINITY);
-        const bool up1 = x1 > m1 + kShiftSlack || (m1 == -INFINITY && x1 > -INFINITY);
-        // O may only be rescaled once the previous step's PV MMAs have landed, and this step's P
-        // buffer rewritten once the PV of two steps back has.
-        if (__any_sync(0xffffffffu, up0 || up1)) {
-          const float n0 = up0 ? fmaxf(m0, x0) : m0, n1 = up1 ? fmaxf(m1, x1) : m1;
-          const float a0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - n0);
-          const float a1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - n1);
-          l0 *= a0;
-          l1 *= a1;
-          m0 = n0;
-          m1 = n1;
+        x0 *= sl2;  // log2 units (the scale is positive)
+        x1 *= sl2;
+        // The shift after the previous step (the other warpgroup's), then ours for this step.
+        // Every step waits for its predecessor's, so the two barriers never run a phase apart.
+        float mp0 = -INFINITY, mp1 = -INFINITY;
+        if (gs > 0) {
+          if (!mbar_wait(&s.m_ready[wg ^ 1], (uint32_t)(((gs - 1) >> 1) & 1), abort_flag))
+            give_up();
           if (n > 0) {
-            // Rescale this half's O columns of the warp's rows (factor 1 where the shift held).
-            if (!mbar_wait(&s.pv_done[(gp - 1) & 1], (uint32_t)(((gp - 1) >> 1) & 1), abort_flag))
-              give_up();
-            tc_fence_after();
+            mp0 = s.mrow[wg ^ 1][r0];
+            mp1 = s.mrow[wg ^ 1][r1];
+          }
+        }
+        const bool up0 = x0 > mp0 + kShiftSlack || (mp0 == -INFINITY && x0 > -INFINITY);
+        const bool up1 = x1 > mp1 + kShiftSlack || (mp1 == -INFINITY && x1 > -INFINITY);
+        const float n0 = up0 ? fmaxf(mp0, x0) : mp0, n1 = up1 ? fmaxf(mp1, x1) : mp1;
+        if (t0 == 0) {
+          s.mrow[wg][r0] = n0;
+          s.mrow[wg][r1] = n1;
+        }
+        mbar_arrive(&s.m_ready[wg]);
+        // Our running sums follow the shift (it never decreases).
+        if (mw0 != n0) l0 = (mw0 == -INFINITY) ? 0.f : l0 * ex2(mw0 - n0);
+        if (mw1 != n1) l1 = (mw1 == -INFINITY) ? 0.f : l1 * ex2(mw1 - n1);
+        mw0 = n0;
+        mw1 = n1;
+        // O follows it too: rescale the warp's rows (factor 1 where the shift held) once the
+        // previous step's PV has landed; our own PV of this step is issued only after our P.
+        if (n > 0 && __any_sync(0xffffffffu, up0 || up1)) {
+          if (!mbar_wait(&s.pv_done[wg ^ 1], (uint32_t)(((gs - 1) >> 1) & 1), abort_flag))
+            give_up();
+          tc_fence_after();
+          const float a0 = !up0 ? 1.f : (mp0 == -INFINITY ? 0.f : ex2(mp0 - n0));
+          const float a1 = !up1 ? 1.f : (mp1 == -INFINITY ? 0.f : ex2(mp1 - n1));
+#pragma unroll
+          for (int hc = 0; hc < 2; ++hc) {
             uint32_t o[32];
-            tmem_ld_16x256b_x8(lane_base + kColO + col0, o);
+            tmem_ld_16x256b_x8(lane_base + kColO + 64 * hc, o);
             tmem_wait_ld();
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
@@ -457,58 +494,75 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[4 * j + 2] = __float_as_uint(__uint_as_float(o[4 * j + 2]) * a1);
               o[4 * j + 3] = __float_as_uint(__uint_as_float(o[4 * j + 3]) * a1);
             }
-            tmem_st_16x256b_x8(lane_base + kColO + col0, o);
-            tmem_wait_st();
+            tmem_st_16x256b_x8(lane_base + kColO + 64 * hc, o);
           }
+          tmem_wait_st();
         }
-        // P = exp2(x * scale - shift) as bf16 pairs: keys 8j + 2 t0, + 1 of this half go to P
-        // column 32 half + 4j + t0 (the layout tcgen05.st 16x128b writes).
-        const float ns0 = m0 == -INFINITY ? 0.f : -m0, ns1 = m1 == -INFINITY ? 0.f : -m1;
-        uint32_t pw[16];
-        float ls0[2] = {0.f, 0.f}, ls1[2] = {0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float p00 = ex2(fmaf(__uint_as_float(v[4 * j]), sl2, ns0));
-          const float p01 = ex2(fmaf(__uint_as_float(v[4 * j + 1]), sl2, ns0));
-          const float p10 = ex2(fmaf(__uint_as_float(v[4 * j + 2]), sl2, ns1));
-          const float p11 = ex2(fmaf(__uint_as_float(v[4 * j + 3]), sl2, ns1));
-          ls0[j & 1] += p00 + p01;
-          ls1[j & 1] += p10 + p11;
-          __nv_bfloat162 q0 = __floats2bfloat162_rn(p00, p01);
-          __nv_bfloat162 q1 = __floats2bfloat162_rn(p10, p11);
-          pw[2 * j] = *reinterpret_cast<uint32_t*>(&q0);
-          pw[2 * j + 1] = *reinterpret_cast<uint32_t*>(&q1);
-        }
-        l0 += ls0[0] + ls0[1];
-        l1 += ls1[0] + ls1[1];
-        if (gp >= 2) {
-          if (!mbar_wait(&s.pv_done[b], (uint32_t)(((gp - 2) >> 1) & 1), abort_flag)) give_up();
+        // Our P buffer is free once the PV of our previous step (two steps back) has landed.
+        if (gs >= 2) {
+          if (!mbar_wait(&s.pv_done[wg], (uint32_t)(((gs - 2) >> 1) & 1), abort_flag)) give_up();
           tc_fence_after();
         }
-        tmem_st_16x128b_x8(lane_base + kColP + 64 * b + 32 * half, pw);
+        // P = exp2(x * scale - shift) as bf16 pairs: keys 8j + 2 t0, + 1 go to P column 4j + t0
+        // (the layout tcgen05.st 16x128b writes), in two stores of 32 columns.
+        const float ns0 = n0 == -INFINITY ? 0.f : -n0, ns1 = n1 == -INFINITY ? 0.f : -n1;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t pw[16];
+          float ls0[2] = {0.f, 0.f}, ls1[2] = {0.f, 0.f};
+#pragma unroll
+          for (int jj = 0; jj < 8; ++jj) {
+            const int j = 8 * hh + jj;
+            const float p00 = ex2(fmaf(__uint_as_float(v[4 * j]), sl2, ns0));
+            const float p01 = ex2(fmaf(__uint_as_float(v[4 * j + 1]), sl2, ns0));
+            const float p10 = ex2(fmaf(__uint_as_float(v[4 * j + 2]), sl2, ns1));
+            const float p11 = ex2(fmaf(__uint_as_float(v[4 * j + 3]), sl2, ns1));
+            ls0[jj & 1] += p00 + p01;
+            ls1[jj & 1] += p10 + p11;
+            __nv_bfloat162 q0 = __floats2bfloat162_rn(p00, p01);
+            __nv_bfloat162 q1 = __floats2bfloat162_rn(p10, p11);
+            pw[2 * jj] = *reinterpret_cast<uint32_t*>(&q0);
+            pw[2 * jj + 1] = *reinterpret_cast<uint32_t*>(&q1);
+          }
+          l0 += ls0[0] + ls0[1];
+          l1 += ls1[0] + ls1[1];
+          tmem_st_16x128b_x8(t_p + 32 * hh, pw);
+        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&s.p_full[b]);
+        mbar_arrive(&s.p_full[wg]);
       }
-      if (stop) break;
+      gp += ui.npairs;
       // ---- epilogue: O / l for this thread's rows, bf16, into the tiled output
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+      const int ub = active & 1;  // the swap buffers alternate by unit
       if (t0 == 0) {
-        s.xsum[half][sp][q4] = l0;
-        s.xsum[half][sp][q4 + 8] = l1;
+        s.xsum[ub][wg][sp][q4] = l0;
+        s.xsum[ub][wg][sp][q4 + 8] = l1;
+        s.xm[ub][wg][sp][q4] = mw0;
+        s.xm[ub][wg][sp][q4 + 8] = mw1;
       }
       if (named_bar_or(bar_id, 64, failed)) {
         failed = true;
         break;
       }
-      l0 += s.xsum[half ^ 1][sp][q4];
-      l1 += s.xsum[half ^ 1][sp][q4 + 8];
-      // The sums are read before either warp of the pair can write them again: the next write
-      // follows at least one more pair barrier (every unit that reaches here has a step).
-      const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+      // The two warpgroups' sums, each relative to the last shift it used, brought to the final
+      // shift (the larger: the shift never decreases along the steps).
+      float i0, i1;
+      {
+        const float om0 = s.xm[ub][wg ^ 1][sp][q4], om1 = s.xm[ub][wg ^ 1][sp][q4 + 8];
+        const float ol0 = s.xsum[ub][wg ^ 1][sp][q4], ol1 = s.xsum[ub][wg ^ 1][sp][q4 + 8];
+        const float mf0 = fmaxf(mw0, om0), mf1 = fmaxf(mw1, om1);
+        const float s0 = (mw0 == -INFINITY ? 0.f : l0 * ex2(mw0 - mf0)) +
+                         (om0 == -INFINITY ? 0.f : ol0 * ex2(om0 - mf0));
+        const float s1 = (mw1 == -INFINITY ? 0.f : l1 * ex2(mw1 - mf1)) +
+                         (om1 == -INFINITY ? 0.f : ol1 * ex2(om1 - mf1));
+        i0 = s0 > 0.f ? 1.f / s0 : 0.f;
+        i1 = s1 > 0.f ? 1.f / s1 : 0.f;
+      }
       if (!mbar_wait(&s.o_full, (uint32_t)(active & 1), abort_flag)) give_up();
       tc_fence_after();
       failed = __any_sync(0xffffffffu, failed);  // the TMEM loads below are warp-collective
@@ -567,12 +621,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++active;
     }
     if (failed && lane == 0) fail(s, a.dev_status);
+    tc_fence_before();
+    named_bar(kTeardownBar, kThreads);
   }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
 // ---------------------------------------------------------------------------------- host side
