@@ -20,11 +20,12 @@
 // Step n uses S and P buffer n & 1, so the softmax of step n + 1 never waits for the PV of step n.
 //
 // Roles (one persistent CTA per SM, 12 warps, units in static round robin, head-major):
-//   warp 0       TMA producer for the K and V pairs (3-stage rings each)
+//   warp 0       TMA producer for the K pairs (3-stage ring)
 //   warp 1       TMEM allocation; one thread issues the S MMAs and their commits
 //   warp 2       one thread issues the PV MMAs and their commits
-//   warp 3       TMA producer for each unit's query tile (one buffer, refilled once the previous
-//                unit's last S has completed, so the next unit's scores start during the epilogue)
+//   warp 3       TMA producer for the V pairs (3-stage ring) and for each unit's query tile (one
+//                buffer, refilled once the previous unit's last S has completed, so the next unit's
+//                scores start during the epilogue)
 //   warps 4..11  softmax and epilogue, two warpgroups: warpgroup X takes the steps n with n % 2 == X
 //                (S and P buffer X) and, in the epilogue, output columns 64 X .. 64 X + 63. Thread t
 //                of warp w owns query rows 16 (w % 4) + t/4 and that + 8, and the key columns
@@ -140,52 +141,57 @@ struct Maps {
   CUtensorMap q, k, v;
 };
 
-// Streams the kept key and value tile pairs of every unit of this CTA, in step order, into their
-// rings (lane 0 of the producer warp). Step gp's K pair goes to K stage gp % kKStages once S(gp -
-// kKStages) has completed, its V pair to V stage gp % kVStages once PV(gp - kVStages) has.
+// Streams one operand's kept tile pairs (K or V) of every unit of this CTA, in step order, into a
+// ring of kStages pair buffers (lane 0 of a producer warp): step gp's pair goes to stage
+// gp % kStages once the MMAs that read the stage's previous pair have completed. With kLoadQ the
+// thread also loads each unit's query tile, ahead of the unit's pairs, once the previous unit's last
+// S has completed (the V producer: its pairs are needed only after the unit's first scores).
+template <int kStages, bool kLoadQ>
 __device__ __forceinline__ void produce_pairs(SmemLayout& s, const Geo& g, const AttnArgs& a,
-                                              const Maps& maps, volatile int* abort_flag) {
+                                              const Maps& maps, const CUtensorMap* map,
+                                              uint8_t (*ring)[kPairBytes], uint64_t* full,
+                                              uint64_t* empty, volatile int* abort_flag) {
   const int total_units = g.B * g.heads * g.nT;
-  long gp = 0, nk = 0, nv = 0;  // steps begun, K and V pairs issued
+  long gp = 0, issued = 0;
+  int nq = 0;  // query tiles loaded
   bool ok = true;
   for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
     const UnitInfo ui = unit_info(g, a, u);
+    if (ui.npairs == 0) continue;
+    if (kLoadQ) {
+      if (!mbar_wait(&s.q_empty, (uint32_t)((nq & 1) ^ 1), abort_flag)) {
+        ok = false;
+        break;
+      }
+      mbar_expect_tx(&s.q_full, kQBytes);
+      const int row0 = ui.b * g.Lp + ui.i * kTileElems;
+      for (int hh = 0; hh < kHalves; ++hh)
+        tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
+      ++nq;
+    }
     for (int n = 0; n < ui.npairs; ++n, ++gp) {
+      const int st = (int)(gp % kStages);
+      if (!mbar_wait(&empty[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag)) {
+        ok = false;
+        break;
+      }
       int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
       if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
       if (jb < 0) jb = ja;
-      const int za = ui.b * g.Lp + ja * kTileElems, zb = ui.b * g.Lp + jb * kTileElems;
-      const int ks = (int)(gp % kKStages), vs = (int)(gp % kVStages);
-      if (!mbar_wait(&s.k_empty[ks], (uint32_t)(((gp / kKStages) & 1) ^ 1), abort_flag)) {
-        ok = false;
-        break;
-      }
-      mbar_expect_tx(&s.k_full[ks], kPairBytes);
+      mbar_expect_tx(&full[st], kPairBytes);
       for (int hh = 0; hh < kHalves; ++hh) {
-        uint8_t* dst = s.k[ks] + hh * 2 * kTileBytes;
-        tma_load_3d(dst, &maps.k, &s.k_full[ks], 64 * hh, ui.h, za);
-        tma_load_3d(dst + kTileBytes, &maps.k, &s.k_full[ks], 64 * hh, ui.h, zb);
+        uint8_t* dst = ring[st] + hh * 2 * kTileBytes;
+        tma_load_3d(dst, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
+        tma_load_3d(dst + kTileBytes, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + jb * kTileElems);
       }
-      ++nk;
-      if (!mbar_wait(&s.v_empty[vs], (uint32_t)(((gp / kVStages) & 1) ^ 1), abort_flag)) {
-        ok = false;
-        break;
-      }
-      mbar_expect_tx(&s.v_full[vs], kPairBytes);
-      for (int hh = 0; hh < kHalves; ++hh) {
-        uint8_t* dst = s.v[vs] + hh * 2 * kTileBytes;
-        tma_load_3d(dst, &maps.v, &s.v_full[vs], 64 * hh, ui.h, za);
-        tma_load_3d(dst + kTileBytes, &maps.v, &s.v_full[vs], 64 * hh, ui.h, zb);
-      }
-      ++nv;
+      ++issued;
     }
   }
   if (!ok) fail(s, a.dev_status);
   // Drain: the last loads issued must land before the CTA can exit.
-  for (long t = nk - kKStages; t < nk; ++t)
-    if (t >= 0) mbar_wait(&s.k_full[t % kKStages], (uint32_t)((t / kKStages) & 1), nullptr);
-  for (long t = nv - kVStages; t < nv; ++t)
-    if (t >= 0) mbar_wait(&s.v_full[t % kVStages], (uint32_t)((t / kVStages) & 1), nullptr);
+  for (long t = issued - kStages; t < issued; ++t)
+    if (t >= 0) mbar_wait(&full[t % kStages], (uint32_t)((t / kStages) & 1), nullptr);
+  if (kLoadQ && nq > 0) mbar_wait(&s.q_full, (uint32_t)((nq - 1) & 1), nullptr);
 }
 
 
@@ -239,27 +245,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     regs_dec<kProducerRegs>();
     if (warp == 0) {
-      // ------------------------------------------------------------- K and V producer
-      if (lane == 0) produce_pairs(s, g, a, maps, abort_flag);
+      // ------------------------------------------------------------- K producer
+      if (lane == 0)
+        produce_pairs<kKStages, false>(s, g, a, maps, &maps.k, s.k, s.k_full, s.k_empty,
+                                       abort_flag);
     } else if (warp == 3) {
-      // ------------------------------------------------------------- Q producer
-      if (lane == 0) {
-        int active = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
-          const UnitInfo ui = unit_info(g, a, u);
-          if (ui.npairs == 0) continue;
-          if (!mbar_wait(&s.q_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&s.q_full, kQBytes);
-          const int row0 = ui.b * g.Lp + ui.i * kTileElems;
-          for (int hh = 0; hh < kHalves; ++hh)
-            tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
-          ++active;
-        }
-        if (!ok) fail(s, a.dev_status);
-        // Drain: the last query tile loaded must land before the CTA can exit.
-        if (active > 0) mbar_wait(&s.q_full, (uint32_t)((active - 1) & 1), nullptr);
-      }
+      // ------------------------------------------------------------- V and Q producer
+      if (lane == 0)
+        produce_pairs<kVStages, true>(s, g, a, maps, &maps.v, s.v, s.v_full, s.v_empty,
+                                      abort_flag);
     } else if (warp == 1) {
       // ------------------------------------------------------------- S issuer
       // A thread's tcgen05.mma issue proceeds at about the rate the tensor pipe retires MMAs, so a
@@ -425,24 +419,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        // Row maxima (the 4 threads of a row hold its 128 columns), as balanced trees.
+        // Row maxima (the 4 threads of a row hold its 128 columns), as trees of 3-input maxima.
         float x0, x1;
         {
-          float t0r[16], t1r[16];
+          float r0v[32], r1v[32];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
-            t0r[j] = fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]));
-            t1r[j] = fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+            r0v[2 * j] = __uint_as_float(v[4 * j]);
+            r0v[2 * j + 1] = __uint_as_float(v[4 * j + 1]);
+            r1v[2 * j] = __uint_as_float(v[4 * j + 2]);
+            r1v[2 * j + 1] = __uint_as_float(v[4 * j + 3]);
           }
-#pragma unroll
-          for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-            for (int j = 0; j < w; ++j) {
-              t0r[j] = fmaxf(t0r[j], t0r[j + w]);
-              t1r[j] = fmaxf(t1r[j], t1r[j + w]);
-            }
-          x0 = t0r[0];
-          x1 = t1r[0];
+          x0 = max_of_32(r0v);
+          x1 = max_of_32(r1v);
         }
         x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
         x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));

@@ -298,6 +298,22 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// Largest of three floats in one instruction (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// Largest of 32 floats as a tree of three-input maxima.
+__device__ __forceinline__ float max_of_32(const float (&x)[32]) {
+  float u[11];
+#pragma unroll
+  for (int k = 0; k < 10; ++k) u[k] = fmax3(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+  u[10] = fmaxf(x[30], x[31]);
+  const float w0 = fmax3(u[0], u[1], u[2]), w1 = fmax3(u[3], u[4], u[5]);
+  const float w2 = fmax3(u[6], u[7], u[8]), w3 = fmaxf(u[9], u[10]);
+  return fmaxf(fmax3(w0, w1, w2), w3);
+}
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
