@@ -16,14 +16,41 @@ namespace {
 constexpr int kSelThreads = 256;  // 8 warps
 constexpr int kKeyChunk = 128;    // pooled key rows staged in shared memory at a time (one per thread pair)
 constexpr int kPad = 4;           // key row padding (floats): consecutive rows 4 banks apart
+constexpr int kRegSelectMax = 512;  // rows up to this many tiles are selected in registers
 
-// Query tiles per CTA: 16 (two CTAs per SM for the common sizes), or 8 when 16 score rows would not
-// fit next to the staged operands (~200 KB of shared memory).
-__host__ __device__ inline size_t sel_smem_floats(int D, int nT, int R) {
-  return (size_t)R * D + (size_t)kKeyChunk * (D + kPad) + (size_t)R * nT + 8 * 256;
+// Shared memory of a selection CTA with R query tiles (floats): query rows, a key chunk, the score
+// rows and, when the selection uses them, the per-warp radix histograms (the mass selection always;
+// top-k for rows of more than kRegSelectMax tiles).
+inline size_t sel_smem_floats(int D, int nT, int R, bool hist) {
+  return (size_t)R * D + (size_t)kKeyChunk * (D + kPad) + (size_t)R * nT + (hist ? 8 * 256 : 0);
 }
-__host__ __device__ inline int sel_rows(int D, int nT) {
-  return sel_smem_floats(D, nT, 16) * 4 <= 200 * 1024 ? 16 : 8;
+// Query tiles per CTA of the cumulative-mass selection: 16 (two CTAs per SM for the common sizes),
+// or 8 when 16 score rows would not fit next to the staged operands (~200 KB of shared memory).
+inline int sel_rows(int D, int nT) {
+  return sel_smem_floats(D, nT, 16, true) * 4 <= 200 * 1024 ? 16 : 8;
+}
+// Query tiles per CTA of the top-k selection: the count (8 .. 24) with the fewest waves over the
+// machine, each wave weighted by its rows plus a fixed cost of streaming the head's pooled keys
+// (worth about 8 rows).
+int topk_rows(const Geo& g, int sms) {
+  constexpr size_t kSmPerSm = 233472, kSmPerCta = 232448, kReserve = 1024;
+  int best = 8;
+  long best_cost = -1;
+  for (int R = 8; R <= 24; R += 4) {
+    const size_t bytes = sel_smem_floats(g.D, g.nT, R, g.nT > kRegSelectMax) * sizeof(float);
+    if (bytes > kSmPerCta) continue;
+    long per_sm = (long)(kSmPerSm / (bytes + kReserve));
+    if (per_sm > 2048 / kSelThreads) per_sm = 2048 / kSelThreads;
+    if (per_sm < 1) continue;
+    const long blocks = (long)g.B * g.heads * ((g.nT + R - 1) / R);
+    const long waves = (blocks + per_sm * sms - 1) / (per_sm * sms);
+    const long cost = waves * (R + 8);
+    if (best_cost < 0 || cost < best_cost) {
+      best = R;
+      best_cost = cost;
+    }
+  }
+  return best;
 }
 
 // Scores S[i, j] = pq_i . pk_j in fp32 (fused multiply-adds over d in order) for the CTA's R query
@@ -83,10 +110,22 @@ __device__ void compute_scores(const Geo& g, const float* __restrict__ pq,
   __syncthreads();
 }
 
-__device__ void compute_scores_any(const Geo& g, const float* pq, const float* pk, long bh, int i0,
-                                   int R, float* sm) {
+// R = 8 or 16 (the cumulative-mass selection).
+__device__ void compute_scores_8_16(const Geo& g, const float* pq, const float* pk, long bh, int i0,
+                                    int R, float* sm) {
   if (R == 16) compute_scores<8>(g, pq, pk, bh, i0, sm);
   else compute_scores<4>(g, pq, pk, bh, i0, sm);
+}
+// R = 8, 12, 16, 20 or 24 (the top-k selection).
+__device__ void compute_scores_any(const Geo& g, const float* pq, const float* pk, long bh, int i0,
+                                   int R, float* sm) {
+  switch (R) {
+    case 24: compute_scores<12>(g, pq, pk, bh, i0, sm); break;
+    case 20: compute_scores<10>(g, pq, pk, bh, i0, sm); break;
+    case 16: compute_scores<8>(g, pq, pk, bh, i0, sm); break;
+    case 12: compute_scores<6>(g, pq, pk, bh, i0, sm); break;
+    default: compute_scores<4>(g, pq, pk, bh, i0, sm); break;
+  }
 }
 
 // Top-k of a row of at most 32 * KPL values held in registers (lane l owns entries l + 32 i):
@@ -255,7 +294,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(Geo g, const float* _
     int n;
     if (nT <= 128) n = select_topk_row_reg<4>(row, nT, kk, out);
     else if (nT <= 256) n = select_topk_row_reg<8>(row, nT, kk, out);
-    else if (nT <= 512) n = select_topk_row_reg<16>(row, nT, kk, out);
+    else if (nT <= kRegSelectMax) n = select_topk_row_reg<16>(row, nT, kk, out);
     else n = select_topk_row(row, nT, kk, out, hist);
     if (lane == 0) kv_cnt[bh * nT + i] = n;
   }
@@ -345,7 +384,7 @@ __global__ void __launch_bounds__(kSelThreads) mass_kernel(Geo g, const float* _
   const int blocks_per_head = (nT + R - 1) / R;
   const long bh = blockIdx.x / blocks_per_head;
   const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * R;
-  compute_scores_any(g, pq, pk, bh, i0, R, sm);
+  compute_scores_8_16(g, pq, pk, bh, i0, R, sm);
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* vals = sm + R * g.D + kKeyChunk * (g.D + kPad);
   int* hist = reinterpret_cast<int*>(vals + R * nT) + w * 256;
@@ -534,8 +573,11 @@ cudaError_t launch_select_topk(const Geo& g, const float* pq, const float* pk, i
                                int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
                                cudaStream_t s) {
   (void)dev_status;
-  const int R = sel_rows(g.D, g.nT);
-  const size_t smem = sel_smem_floats(g.D, g.nT, R) * sizeof(float);
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int R = topk_rows(g, sms > 0 ? sms : 148);
+  const size_t smem = sel_smem_floats(g.D, g.nT, R, g.nT > kRegSelectMax) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -548,7 +590,7 @@ cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, f
                                float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
                                int32_t* dev_status, cudaStream_t s) {
   const int R = sel_rows(g.D, g.nT);
-  const size_t smem = sel_smem_floats(g.D, g.nT, R) * sizeof(float);
+  const size_t smem = sel_smem_floats(g.D, g.nT, R, true) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(mass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
