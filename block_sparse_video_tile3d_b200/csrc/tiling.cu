@@ -75,10 +75,10 @@ __global__ void __launch_bounds__(kCopyThreads) gather_kernel(Geo g, const uint4
   }
 }
 
-// Grid (ceil(row_chunks / 32), nT, B); block (32, 8). Thread (lane, ry) sums one 16-byte column
-// chunk over the tile's valid rows ry, ry + 8, ...; the 8 partial sums are combined in shared
-// memory and divided by the valid count.
-constexpr int kPoolRows = 8;
+// Grid (ceil(row_chunks / 32), nT, B); block (32, kPoolRows). Thread (lane, ry) sums one 16-byte
+// column chunk over the tile's valid rows ry, ry + kPoolRows, ...; the kPoolRows partial sums are
+// combined in shared memory and divided by the valid count.
+constexpr int kPoolRows = 16;  // warps per CTA: 512 threads, four CTAs per SM
 
 __global__ void __launch_bounds__(32 * kPoolRows) pool_kernel(Geo g, const uint4* __restrict__ y,
                                                               float* __restrict__ pooled) {
@@ -109,12 +109,12 @@ __global__ void __launch_bounds__(32 * kPoolRows) pool_kernel(Geo g, const uint4
 #pragma unroll
   for (int e = 0; e < 8; ++e) part[ry][lane * 8 + e] = acc[e];
   __syncthreads();
-  // 256 threads finalise 32 chunks x 8 elements.
+  // The first 256 threads finalise 32 chunks x 8 elements.
   const int t = ry * 32 + lane;
   const int cc = t >> 3;
   const int e = t & 7;
   const int col_chunk = blockIdx.x * 32 + cc;
-  if (col_chunk < g.row_chunks) {
+  if (t < 32 * 8 && col_chunk < g.row_chunks) {
     float s = 0.f;
 #pragma unroll
     for (int q = 0; q < kPoolRows; ++q) s += part[q][cc * 8 + e];
@@ -125,10 +125,10 @@ __global__ void __launch_bounds__(32 * kPoolRows) pool_kernel(Geo g, const uint4
   }
 }
 
-// Fused scatter + pool: grid (ceil(row_chunks / 32), nT, B), block (32, 8). The CTA moves one
-// 512-byte column slab of one tile: thread (lane, ry) copies chunk column `lane` of the tile's
-// padded rows ry, ry + 8, ... from their raster rows (zeros for pad slots) and sums the valid ones;
-// the 8 partial sums are combined in shared memory and divided by the valid count.
+// Fused scatter + pool: grid (ceil(row_chunks / 32), nT, B), block (32, kPoolRows). The CTA moves
+// one 512-byte column slab of one tile: thread (lane, ry) copies chunk column `lane` of the tile's
+// padded rows ry, ry + kPoolRows, ... from their raster rows (zeros for pad slots) and sums the
+// valid ones; the partial sums are combined in shared memory and divided by the valid count.
 __global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_kernel(Geo g,
                                                                       const uint4* __restrict__ x,
                                                                       uint4* __restrict__ y,
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_kernel(Geo g,
   const int cc = t >> 3;
   const int e = t & 7;
   const int col_chunk = blockIdx.x * 32 + cc;
-  if (col_chunk < g.row_chunks) {
+  if (t < 32 * 8 && col_chunk < g.row_chunks) {  // the first 256 threads: 32 chunks x 8 elements
     float sum = 0.f;
 #pragma unroll
     for (int q = 0; q < kPoolRows; ++q) sum += part[q][cc * 8 + e];
