@@ -130,8 +130,9 @@ __device__ void compute_scores_any(const Geo& g, const float* pq, const float* p
 
 // Top-k of a row of at most 32 * KPL values held in registers (lane l owns entries l + 32 i):
 // the k-th largest order-preserving key is found bit by bit from the top (largest T with at least k
-// keys >= T), then every key above it and the first (by index) ties at it are emitted in
-// ascending index order. Same result as the radix select below; no shared-memory histograms.
+// keys >= T; the search stops early once exactly k keys are >= the candidate), then every key above
+// the threshold and the first (by index) ties at it are emitted in ascending index order. Same
+// result as the radix select below; no shared-memory histograms.
 template <int KPL>
 __device__ int select_topk_row_reg(const float* row, int n, int k, int32_t* out) {
   k = imin(k, n);
@@ -149,7 +150,11 @@ __device__ int select_topk_row_reg(const float* row, int n, int k, int32_t* out)
     int c = 0;
 #pragma unroll
     for (int i = 0; i < KPL; ++i) c += key[i] >= cand ? 1 : 0;
-    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) thr = cand;
+    const int total = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+    if (total >= k) thr = cand;
+    // Exactly k keys at or above the threshold: they are the top k (no tie crosses it), and the
+    // emission below keeps every key >= thr, so the remaining low bits change nothing.
+    if (total == k) break;
   }
   int gt = 0;
 #pragma unroll
