@@ -360,28 +360,61 @@ def run_ours(args, w):
     ms_step = total_ms / args.steps
     status = model.device_status()
 
-    # ---- end to end through the public API with pinned host buffers
+    # ---- end to end through the public API with pinned host buffers. Steps are pipelined the way a
+    # serving loop would run them: each step's inputs go host -> device on one copy stream and its
+    # output device -> host on another, into double-buffered device tensors, so step i + 1's upload
+    # overlaps step i's compute and download. Every step's copies lie inside the timed region.
     qh, kh, vh = (x.pin_memory() for x in (q, k, v))
-    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    ohs = [torch.empty(od.shape, dtype=od.dtype).pin_memory() for _ in range(2)]
+    ins = [(qd, kd, vd), tuple(torch.empty_like(x) for x in (qd, kd, vd))]
+    outs = [od, torch.empty_like(od)]
+    comp = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     e2e_steps = max(3, min(args.steps, 20))
-    for _ in range(2):
-        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True)  # noqa: E702
-        vd.copy_(vh, non_blocking=True); model.forward(qd, kd, vd, od)  # noqa: E702
-        oh.copy_(od, non_blocking=True)
+
+    def e2e_loop(n_steps):
+        in_free = [None, None]   # compute of the step that last read input buffer b has finished
+        out_free = [None, None]  # download of the step that last wrote output buffer b has finished
+        done = None
+        for i in range(n_steps):
+            b = i & 1
+            with torch.cuda.stream(up):
+                if in_free[b] is not None:
+                    up.wait_event(in_free[b])
+                for dst, src in zip(ins[b], (qh, kh, vh)):
+                    dst.copy_(src, non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(up)
+            comp.wait_event(ready)
+            if out_free[b] is not None:
+                comp.wait_event(out_free[b])
+            model.forward(*ins[b], outs[b])
+            computed = torch.cuda.Event()
+            computed.record(comp)
+            in_free[b] = computed
+            with torch.cuda.stream(down):
+                down.wait_event(computed)
+                ohs[b].copy_(outs[b], non_blocking=True)
+                done = torch.cuda.Event()
+                done.record(down)
+            out_free[b] = done
+        comp.wait_event(done)
+        for st in (up, down):  # the next region starts after every copy of this one
+            st.wait_stream(comp)
+
+    e2e_loop(2)
     barrier()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(e2e_steps):
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        model.forward(qd, kd, vd, od)
-        oh.copy_(od, non_blocking=True)
-    e1.record()
+    e0.record(comp)
+    up.wait_event(e0)
+    down.wait_event(e0)
+    e2e_loop(e2e_steps)
+    e1.record(comp)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
+    e2e_same = bool(torch.equal(ohs[(e2e_steps - 1) & 1], od.cpu()))  # same output as on device
 
     peaks = _peaks()
     attn_ms = stage_ms["attention"]
@@ -421,7 +454,10 @@ def run_ours(args, w):
                               "hbm_peak_gbs": peaks["hbm_gbs"]},
         "stages": stage_report,
         "e2e": {"value": whole_job_tflops(flops_all, e2e_ms), "unit": "TFLOPS",
-                "ms_per_step": e2e_ms,
+                "ms_per_step": e2e_ms, "steps": e2e_steps, "output_matches_device_run": e2e_same,
+                "pipelining": "host-to-device and device-to-host copies on their own streams, "
+                              "double-buffered device tensors: step i + 1's upload overlaps step "
+                              "i's compute and download",
                 "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                 "d2h_bytes_per_step": od.numel() * od.element_size()},
         "gpu_launches": args.steps * nst,
