@@ -12,9 +12,10 @@ Modules:
   select     tile-to-tile scores, top-k and cumulative-mass KV tile selection
   bsa        query pruning and reconstruction of the bidirectional sparse attention variant
   attention  softmax attention restricted to the kept (query tile, key tile) pairs
+  attention_bwd  its gradients with respect to Q, K and V (the backward pass)
   pipeline   the four stages chained, as the hot path runs them
 
 Every function is pinned by a CPU test against something other than itself (closed forms,
 brute force on tiny inputs, invariants, library routines for the dense special case).
 """
-from . import tiling, pool, select, bsa, attention, pipeline  # noqa: F401
+from . import tiling, pool, select, bsa, attention, attention_bwd, pipeline  # noqa: F401

@@ -10,11 +10,13 @@ import numpy as np
 import pytest
 
 import oracle.attention
+import oracle.attention_bwd
 import oracle.bsa
 import oracle.pool
 import oracle.select
 import oracle.tiling
 from tests import test_oracle_attention as ta
+from tests import test_oracle_attention_bwd as tb
 from tests import test_oracle_bsa_ratio as tr
 from tests import test_oracle_pool_select as tp
 from tests import test_oracle_tiling as tt
@@ -81,6 +83,41 @@ def _ratio_keep_most_similar(rows, ratio):
     return keep, oracle.bsa._sources(rows, keep), cmean
 
 
+def _bwd_no_delta(q_rows, k_rows, v_rows, do_rows, scale):
+    q, k, v, do = (np.asarray(a, dtype=np.float64) for a in (q_rows, k_rows, v_rows, do_rows))
+    logits = scale * (q @ k.T)
+    e = np.exp(logits - logits.max(axis=1, keepdims=True))
+    p = e / e.sum(axis=1, keepdims=True)
+    ds = p * (do @ v.T)  # the softmax Jacobian's "- dO . o" term dropped: wrong
+    return scale * (ds @ k), scale * (ds.T @ q), p.T @ do
+
+
+def _bwd_dk_unscaled(q_rows, k_rows, v_rows, do_rows, scale):
+    dq, dk, dv = _orig_rows_bwd(q_rows, k_rows, v_rows, do_rows, scale)
+    return dq, dk / scale, dv  # key gradient without the softmax scale: wrong
+
+
+_orig_rows_bwd = oracle.attention_bwd.attend_rows_bwd
+
+
+def _bwd_pruned_keep_own_grad(qt, kt, vt, vc, sets, scale, do, keep=None, src=None):
+    B, Lp, nh, D = qt.shape
+    dq, dk, dv = (np.zeros((B, Lp, nh, D)) for _ in range(3))
+    for b in range(B):
+        for h in range(nh):
+            for i in range(Lp // 64):
+                rows_k = oracle.attention._key_rows(sets[b][h][i], vc)
+                kk = np.nonzero(keep[b, h, i][:int(vc[i])])[0]
+                rows_q = 64 * i + kk
+                g_out = np.asarray(do)[b, rows_q, h]  # pruned rows' gradients dropped: wrong
+                gq, gk, gv = _orig_rows_bwd(qt[b, rows_q, h], kt[b, rows_k, h], vt[b, rows_k, h],
+                                            g_out, scale)
+                dq[b, rows_q, h] = gq
+                dk[b, rows_k, h] += gk
+                dv[b, rows_k, h] += gv
+    return dq, dk, dv
+
+
 @pytest.mark.parametrize("patch,pin", [
     ((oracle.tiling, "tile_partition_indices", _swapped_partition),
      lambda: tt.test_partition_matches_sort_by_tile_key((5, 9, 9))),
@@ -95,6 +132,10 @@ def _ratio_keep_most_similar(rows, ratio):
      tr.test_fan_keeps_the_widest_angles_and_copies_the_nearest_kept_row),
     ((oracle.bsa, "keep_size_for_ratio", lambda ratio, n=64: max(1, int(round(ratio * n)))),
      lambda: tr.test_keep_size(0.2, 12)),
+    ((oracle.attention_bwd, "attend_rows_bwd", _bwd_no_delta), tb.test_softmax_identities),
+    ((oracle.attention_bwd, "attend_rows_bwd", _bwd_dk_unscaled), tb.test_finite_differences_tiny),
+    ((oracle.attention_bwd, "block_sparse_attention_bwd", _bwd_pruned_keep_own_grad),
+     tb.test_pruned_rows_route_their_gradient_to_the_source_row),
 ])
 def test_planted_mistake_is_caught(monkeypatch, patch, pin):
     mod, name, fn = patch
