@@ -84,3 +84,22 @@ def test_ratio_mode_over_tiles_matches_per_block_calls():
                 k1, s1, c1 = bsa.prune_block_ratio(qt[b, 64 * i:64 * (i + 1), h], 0.5)
                 np.testing.assert_array_equal(keep[b, h, i], k1)
                 np.testing.assert_array_equal(src[b, h, i], s1)
+
+
+def test_pipeline_ratio_one_is_mass_selection_over_all_rows():
+    """Keep ratio 1 keeps every query row, so the BSA chain (pooled kept queries, mass selection,
+    attention with every row its own source) reduces to plain mass selection and attention."""
+    from oracle import pipeline
+
+    rng = np.random.default_rng(7)
+    T, H, W = 4, 8, 8  # no pads: the ratio mode needs L == 64 * nT
+    q, k, v = (rng.normal(size=(1, T * H * W, 2, 16)) for _ in range(3))
+    bsa_res = pipeline.forward(q, k, v, T, H, W, "bsa", scale=0.25, tau=0.8, keep_ratio=1.0)
+    mass_res = pipeline.forward(q, k, v, T, H, W, "mass", scale=0.25, tau=0.8)
+    assert bsa_res["keep"].all()
+    np.testing.assert_allclose(bsa_res["pq"], mass_res["pq"], rtol=1e-12, atol=1e-12)
+    for b in range(1):
+        for h in range(2):
+            for i in range(len(mass_res["sets"][b][h])):
+                np.testing.assert_array_equal(bsa_res["sets"][b][h][i], mass_res["sets"][b][h][i])
+    np.testing.assert_allclose(bsa_res["o"], mass_res["o"], rtol=1e-12, atol=1e-12)
