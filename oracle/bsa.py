@@ -141,8 +141,3 @@ def pooled_kept_queries(qt: np.ndarray, keep: np.ndarray) -> np.ndarray:
                 kk = keep[b, h, i]
                 out[b, h, i] = rows[kk].sum(axis=0) / int(kk.sum())
     return out
-
-
-def reconstruct_pruned(o_block: np.ndarray, src: np.ndarray) -> np.ndarray:
-    """Fill pruned rows of one block's output ``[64, D]`` from their source rows."""
-    return o_block[src]

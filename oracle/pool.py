@@ -24,11 +24,3 @@ def tile_mean_pool(y: np.ndarray, vc: np.ndarray) -> np.ndarray:
         rows = y[:, TILE_ELEMS * i:TILE_ELEMS * i + n].astype(np.float64)  # [B, n, heads, D]
         out[:, :, i, :] = rows.sum(axis=1) / n
     return out
-
-
-def block_mean_pool_rows(rows: np.ndarray, keep: np.ndarray) -> np.ndarray:
-    """Mean of the rows of one block selected by boolean ``keep`` (fp64). Empty selection -> 0."""
-    n = int(keep.sum())
-    if n == 0:
-        return np.zeros(rows.shape[-1], dtype=np.float64)
-    return rows[keep].astype(np.float64).sum(axis=0) / n

@@ -135,6 +135,33 @@ def test_topk_gap_and_margins():
     np.testing.assert_allclose(m["sum_margin"], 0.05, atol=1e-12)
 
 
+def test_mass_margins_hand_worked_row():
+    # Logits log(p) with p = (0.05, 0.45, 0.15, 0.35) at scale 1: the softmax gives p back. Ranked:
+    # 0.45 (tile 1), 0.35 (tile 3), 0.15 (tile 2), 0.05 (tile 0); running sums .45, .80, .95, 1.
+    row = np.log(np.array([0.05, 0.45, 0.15, 0.35]))
+    # tau = 0.65: the sum first reaches it at the second tile, so tiles {1, 3} are kept; the cut
+    # lies between p = 0.35 and p = 0.15, a gap of 0.2 relative to the largest p 0.45 (the gaps
+    # one place earlier or later would be 0.1 / 0.45); the sums on either side of the cut are
+    # 0.45 and 0.80, at distances 0.20 and 0.15 from tau.
+    np.testing.assert_array_equal(select.select_mass_row(row, 1.0, 0.65, 1), [1, 3])
+    m = select.mass_margins(row, 1.0, 0.65, 1)
+    assert m["count"] == 2
+    np.testing.assert_allclose(m["cut_gap"], 0.2 / 0.45, rtol=1e-12)
+    np.testing.assert_allclose(m["sum_margin"], 0.15, rtol=1e-9)
+    # a floor of 3 tiles moves the cut to between 0.15 and 0.05 and makes the sum irrelevant
+    m = select.mass_margins(row, 1.0, 0.65, 3)
+    assert m["count"] == 3
+    np.testing.assert_allclose(m["cut_gap"], 0.1 / 0.45, rtol=1e-12)
+    assert np.isinf(m["sum_margin"])
+    # tau = 0.97 needs every tile: no cut at all
+    m = select.mass_margins(row, 1.0, 0.97, 1)
+    assert m["count"] == 4 and np.isinf(m["cut_gap"])
+    # two equal probabilities at the cut: a zero gap flags the row as undecidable
+    tie = np.log(np.array([0.3, 0.3, 0.4]))
+    m = select.mass_margins(tie, 1.0, 0.5, 1)
+    assert m["count"] == 2 and m["cut_gap"] == 0.0
+
+
 def test_map_set_roundtrip():
     rng = np.random.default_rng(8)
     mask = (rng.random((2, 3, 5, 5)) < 0.4).astype(np.uint8)
