@@ -16,7 +16,10 @@ Readings taken where the pages are silent:
 * Mass mode: ``p = softmax(scale * S_i)`` over the row, with ``scale`` the attention softmax scale;
   tiles are taken in descending ``p`` (ties: lower index) until the running sum first reaches the
   threshold, the tile that reaches it included; at least ``min_k`` tiles are kept; if the running
-  sum never reaches the threshold (rounding at threshold 1) every tile is kept.
+  sum never reaches the threshold (rounding at threshold 1) every tile is kept. At a threshold of
+  1 every tile is kept outright: every softmax probability is positive, so the exact running sum
+  reaches 1 only with the last tile, while a rounded one can reach it earlier when the tail
+  probabilities are too small to change it.
 """
 from __future__ import annotations
 
@@ -71,7 +74,7 @@ def select_mass_row(row: np.ndarray, scale: float, tau: float, min_k: int) -> np
     order = _desc_order(row.astype(np.float64))
     csum = np.cumsum(p[order])
     hit = np.nonzero(csum >= tau)[0]
-    m = int(hit[0]) + 1 if hit.size else nT
+    m = int(hit[0]) + 1 if hit.size and tau < 1.0 else nT
     m = max(m, min(int(min_k), nT))
     return np.sort(order[:m])
 
@@ -93,7 +96,7 @@ def mass_margins(row: np.ndarray, scale: float, tau: float, min_k: int) -> dict:
     order = _desc_order(row.astype(np.float64))
     ps = p[order]
     csum = np.cumsum(ps)
-    hit = np.nonzero(csum >= tau)[0]
+    hit = np.nonzero(csum >= tau)[0] if tau < 1.0 else np.zeros(0, dtype=np.int64)
     m_tau = int(hit[0]) + 1 if hit.size else nT
     m = max(m_tau, min(int(min_k), nT))
     cut_gap = np.inf if m >= nT else (ps[m - 1] - ps[m]) / ps[0]

@@ -135,6 +135,17 @@ def test_topk_gap_and_margins():
     np.testing.assert_allclose(m["sum_margin"], 0.05, atol=1e-12)
 
 
+def test_mass_one_keeps_every_tile_even_when_the_tail_rounds_away():
+    # Scores spread so far that the tail probabilities (e^-60, e^-120 relative to the largest) are
+    # below fp64's resolution of 1: the rounded running sum reaches 1.0 before them, but each of
+    # them is positive, so the exact sum reaches 1 only with the last tile.
+    row = np.array([0.0, -60.0, 10.0, -120.0, 5.0])
+    assert np.cumsum(select.softmax_row(row)[[2, 4, 0, 1, 3]])[2] >= 1.0  # rounding reaches 1
+    np.testing.assert_array_equal(select.select_mass_row(row, 1.0, 1.0, 1), np.arange(5))
+    m = select.mass_margins(row, 1.0, 1.0, 1)
+    assert m["count"] == 5 and np.isinf(m["cut_gap"])
+
+
 def test_mass_margins_hand_worked_row():
     # Logits log(p) with p = (0.05, 0.45, 0.15, 0.35) at scale 1: the softmax gives p back. Ranked:
     # 0.45 (tile 1), 0.35 (tile 3), 0.15 (tile 2), 0.05 (tile 0); running sums .45, .80, .95, 1.
