@@ -278,19 +278,15 @@ def _source_sha() -> str:
 
 
 def _ncu_traffic(workload: str):
-    """Per-launch DRAM bytes of the attention kernel from the committed ncu summary, if it was
-    taken on the current kernel source; else None. The summary carries one line per workload:
-    ``traffic: workload=<name> source_sha=<sha> dram_bytes_per_launch=<bytes>``."""
-    p = os.path.join(ROOT, "profiles", "attn_sm100_small_topk56.md")
+    """Per-launch DRAM bytes of the attention kernel from ``profiles/attn_traffic.json`` (written
+    from an ncu capture), if that capture was taken on the current kernel source; else None. The
+    file maps a workload name to ``{"source_sha": ..., "dram_bytes_per_launch": ...}``."""
+    p = os.path.join(ROOT, "profiles", "attn_traffic.json")
     try:
         with open(p) as f:
-            for line in f:
-                line = line.strip().strip("`")
-                if not line.startswith("traffic:"):
-                    continue
-                kv = dict(t.split("=", 1) for t in line[len("traffic:"):].split())
-                if kv.get("workload") == workload and kv.get("source_sha") == _source_sha():
-                    return float(kv["dram_bytes_per_launch"])
+            rec = json.load(f).get(workload)
+        if rec and rec.get("source_sha") == _source_sha():
+            return float(rec["dram_bytes_per_launch"])
     except Exception:
         pass
     return None
@@ -337,8 +333,14 @@ def run_ours(args, w):
             launch()
     torch.cuda.synchronize()
     pairs = int(model.kv_cnt.sum().item())
-    flops = pairs * FLOPS_PER_PAIR(w.D)
-    flops_all = reduce_over_ranks(float(flops), "sum", world, dev)
+    flops = pairs * FLOPS_PER_PAIR(w.D)  # what the attention kernel computes: every row of a pair
+    if model.keep is not None:
+        # BSA: a pair's work counts the query rows that attend, 4 * kept_rows * 64 * D
+        kept_rows = model.keep.to(torch.int64).sum(-1)
+        flops_metric = int((model.kv_cnt.to(torch.int64) * kept_rows).sum().item()) * 4 * 64 * w.D
+    else:
+        flops_metric = flops
+    flops_all = reduce_over_ranks(float(flops_metric), "sum", world, dev)
 
     # ---- device-resident timed region, events between stages on the launching stream
     nst = len(stages)
@@ -364,13 +366,25 @@ def run_ours(args, w):
     # serving loop would run them: each step's inputs go host -> device on one copy stream and its
     # output device -> host on another, into double-buffered device tensors, so step i + 1's upload
     # overlaps step i's compute and download. Every step's copies lie inside the timed region.
-    qh, kh, vh = (x.pin_memory() for x in (q, k, v))
-    ohs = [torch.empty(od.shape, dtype=od.dtype).pin_memory() for _ in range(2)]
+    # Two different host inputs alternate (set i & 1 for step i, with buffer i & 1), each with its
+    # own reference output from the device-resident path, and every step's download is compared
+    # with its reference, so a race between an upload and the compute that reads it would show.
+    ref_out = [od.cpu()]
+    q2, k2, v2 = workloads.make_qkv(w, seed=w.seed + 7)
+    hosts = [tuple(x.pin_memory() for x in (q, k, v)), tuple(x.pin_memory() for x in (q2, k2, v2))]
     ins = [(qd, kd, vd), tuple(torch.empty_like(x) for x in (qd, kd, vd))]
     outs = [od, torch.empty_like(od)]
+    for dst, src in zip(ins[1], hosts[1]):
+        dst.copy_(src)
+    model.forward(*ins[1], outs[1])
+    torch.cuda.synchronize()
+    ref_out.append(outs[1].cpu())
+    out_bytes = od.numel() * od.element_size()
+    e2e_steps = max(4, min(args.steps, 20, int(2e9 // out_bytes)))
+    e2e_steps += e2e_steps & 1
+    ohs = [torch.empty(od.shape, dtype=od.dtype).pin_memory() for _ in range(e2e_steps)]
     comp = torch.cuda.current_stream()
     up, down = torch.cuda.Stream(), torch.cuda.Stream()
-    e2e_steps = max(3, min(args.steps, 20))
 
     def e2e_loop(n_steps):
         in_free = [None, None]   # compute of the step that last read input buffer b has finished
@@ -381,7 +395,7 @@ def run_ours(args, w):
             with torch.cuda.stream(up):
                 if in_free[b] is not None:
                     up.wait_event(in_free[b])
-                for dst, src in zip(ins[b], (qh, kh, vh)):
+                for dst, src in zip(ins[b], hosts[b]):
                     dst.copy_(src, non_blocking=True)
                 ready = torch.cuda.Event()
                 ready.record(up)
@@ -394,7 +408,7 @@ def run_ours(args, w):
             in_free[b] = computed
             with torch.cuda.stream(down):
                 down.wait_event(computed)
-                ohs[b].copy_(outs[b], non_blocking=True)
+                ohs[i].copy_(outs[b], non_blocking=True)
                 done = torch.cuda.Event()
                 done.record(down)
             out_free[b] = done
@@ -414,7 +428,7 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
-    e2e_same = bool(torch.equal(ohs[(e2e_steps - 1) & 1], od.cpu()))  # same output as on device
+    e2e_same = all(torch.equal(ohs[i], ref_out[i & 1]) for i in range(e2e_steps))
 
     peaks = _peaks()
     attn_ms = stage_ms["attention"]
@@ -438,6 +452,10 @@ def run_ours(args, w):
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": _describe(w), "kept_pairs": pairs,
                    "kept_block_gflop": flops / 1e9,
+                   "metric_gflop": flops_metric / 1e9,
+                   "metric_flops": ("4 * kept query rows * 64 * D per kept pair (pruned rows are "
+                                    "computed but not counted)") if model.keep is not None else
+                                   "4 * 64 * 64 * D per kept pair",
                    "density": pairs / (w.B * w.heads * w.nT * w.nT),
                    "l2": "no flush: raster Q/K/V inputs of "
                          f"{3 * w.B * w.L * w.heads * w.D * 2 / 1e6:.0f} MB exceed the 126 MB L2",

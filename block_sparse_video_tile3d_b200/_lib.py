@@ -31,7 +31,7 @@ _F = ctypes.c_float
 _S = ctypes.c_size_t
 _G = ctypes.POINTER(Geom)
 
-# name -> (restype, argtypes), in the order of include/tile3d.h
+# name -> (restype, argtypes), in the order of include/tile3d.h, then include/tile3d_testing.h
 SIGNATURES = {
     "t3d_last_error_string": (ctypes.c_char_p, []),
     "t3d_version": (ctypes.c_char_p, []),
@@ -48,6 +48,8 @@ SIGNATURES = {
     "block_sparse_attn_fwd": (_I, [_G, _P, _P, _P, _P, _P, _P, _I, _P, _P, _F, _I, _I, _P, _S,
                                    _P, _P]),
     "block_sparse_attn_workspace_size": (_S, [_G, _I]),
+    # include/tile3d_testing.h
+    "t3d_testing_set_wait_cycles": (_I, [ctypes.c_longlong]),
 }
 
 

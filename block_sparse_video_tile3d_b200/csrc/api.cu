@@ -5,10 +5,15 @@
 #include <stdio.h>
 
 #include "kernels.h"
+#include "tile3d_testing.h"
 
 namespace {
 
 thread_local char g_err[512] = "";
+
+// Limit of each pipeline wait of the attention kernel, in clock cycles (tile3d_testing.h).
+constexpr long long kDefaultWaitCycles = 4000000000LL;  // ~2 s at 2 GHz
+long long g_wait_cycles = kDefaultWaitCycles;
 
 t3d_status fail(t3d_status st, const char* fmt, ...) {
   va_list ap;
@@ -75,7 +80,13 @@ extern "C" {
 
 const char* t3d_last_error_string(void) { return g_err; }
 
-const char* t3d_version(void) { return "0.1.0"; }
+const char* t3d_version(void) { return "0.2.0"; }
+
+t3d_status t3d_testing_set_wait_cycles(long long cycles) {
+  if (cycles < 0) return fail(T3D_ERR_INVALID, "cycles=%lld must be >= 0", cycles);
+  g_wait_cycles = cycles == 0 ? kDefaultWaitCycles : cycles;
+  return ok();
+}
 
 t3d_status tile3d_geometry(const t3d_geom* g, int* nT, int* Lp, int32_t* vc_host) {
   t3d::Geo geo;
@@ -254,7 +265,7 @@ t3d_status block_sparse_attn_fwd(const t3d_geom* g, const void* q, const void* k
                 ws_bytes, need);
   if (need > 0) T3D_CHECK(check_ptr(workspace, "workspace"));
   t3d::AttnArgs a{q, k, v, o, kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale,
-                  workspace, ws_bytes, dev_status};
+                  workspace, ws_bytes, dev_status, g_wait_cycles};
   return cuda_status(t3d::launch_attn(geo, a, as_stream(stream)), "block_sparse_attn_fwd");
 }
 

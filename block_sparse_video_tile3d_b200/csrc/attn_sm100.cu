@@ -1,6 +1,6 @@
 // Fine stage on the sm_100a tensor cores: block-sparse softmax attention over the kept
 // (query tile, key tile) pairs with tcgen05 MMAs accumulating in tensor memory (TMEM) and the kept
-// key/value tiles fetched by TMA.
+// key/value tiles fetched by TMA. One kernel template for head dimensions 64 and 128.
 //
 // FastVideo API docs, bsa_attn page, BSAAttentionImpl.__init__ / forward: bidirectional attention,
 // one KV head per query head, softmax scale 1/sqrt(D), tile-ordered [B, L, heads, D] bf16 tensors,
@@ -12,24 +12,31 @@
 //     S[64 q, 128 keys]  = Q . K_pair^T      (A = Q, B = K pair: shared memory, K-major)
 //     O[64 q, D]        += P . V_pair         (A = P in TMEM, B = V pair in shared memory, MN-major)
 // fp32 accumulation in TMEM. P lives in TMEM, so the tensor core's shared-memory operands are the
-// query tile and the K and V pairs; its operand reads no longer compete with a P^T in shared memory.
+// query tile and the K and V pairs; its operand reads never compete with a P^T in shared memory.
 //
 // TMEM (512 columns; an M = 64 tile occupies lanes 0..15 of each 32-lane sub-partition):
-//   S buffer b: columns 128 b .. 128 b + 127 (fp32)    O: 256 .. 383 (fp32)
+//   S buffer b: columns 128 b .. 128 b + 127 (fp32)    O: 256 .. 255 + D (fp32)
 //   P buffer b: 384 + 64 b .. 447 + 64 b (bf16 pairs: column c holds keys 2c, 2c + 1)
 // Step n uses S and P buffer n & 1, so the softmax of step n + 1 never waits for the PV of step n.
 //
-// Roles (one persistent CTA per SM, 12 warps, units in static round robin, head-major):
-//   warp 0       TMA producer for the K pairs (3-stage ring)
+// Scheduling. One persistent CTA per SM takes units from a queue: an atomic counter in the
+// caller's workspace (zeroed on the stream before each launch), read by the K producer, which
+// publishes each unit through a small ring in shared memory to the other roles. Units come in
+// head-major order, so the CTAs working at one time share a head's K and V in L2; a CTA that drew
+// short units simply draws more, so lists of uneven length (cumulative-mass selection, block masks,
+// pruned queries) leave no CTA idle before the queue is empty.
+//
+// Roles (12 warps):
+//   warp 0       TMA producer for the K pairs (3-stage ring) and the unit queue
 //   warp 1       TMEM allocation; one thread issues the S MMAs and their commits
 //   warp 2       one thread issues the PV MMAs and their commits
 //   warp 3       TMA producer for the V pairs (3-stage ring) and for each unit's query tile (one
 //                buffer, refilled once the previous unit's last S has completed, so the next unit's
 //                scores start during the epilogue)
 //   warps 4..11  softmax and epilogue, two warpgroups: warpgroup X takes the steps n with n % 2 == X
-//                (S and P buffer X) and, in the epilogue, output columns 64 X .. 64 X + 63. Thread t
-//                of warp w owns query rows 16 (w % 4) + t/4 and that + 8, and the key columns
-//                8j + 2(t%4) + {0, 1} of its steps (tcgen05.ld 16x256b).
+//                (S and P buffer X) and, in the epilogue, output columns X D/2 .. X D/2 + D/2 - 1.
+//                Thread t of warp w owns query rows 16 (w % 4) + t/4 and that + 8, and the key
+//                columns 8j + 2(t%4) + {0, 1} of its steps (tcgen05.ld 16x256b).
 // S(n) is issued as soon as its K pair has landed and the softmax has read S(n - 2), so scores run
 // up to two steps ahead; PV(n) as soon as P(n) is in TMEM.
 //
@@ -43,9 +50,10 @@
 // warpgroup keeps the running sums of its own steps relative to the last shift it used; the
 // epilogue brings both to the final (largest) shift and adds them.
 //
-// Every mbarrier wait is bounded; on a timeout the CTA records T3D_DEV_TIMEOUT, stops issuing work,
-// waits (bounded) for its copies and MMAs in flight, frees TMEM and returns. The two warps of a pair
-// leave their loops together: a failure is carried to the pair's next barrier, which ORs it.
+// Every mbarrier wait of the pipeline is bounded (AttnArgs::wait_cycles); on a timeout the CTA
+// records T3D_DEV_TIMEOUT, stops issuing work, waits (bounded by the full limit) for its copies and
+// MMAs in flight, frees TMEM and returns. The two warps of a pair leave their loops together: a
+// failure is carried to the pair's next barrier, which ORs it.
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -54,10 +62,9 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kD = 128;             // head dimension handled by this kernel
-constexpr int kHalves = kD / 64;    // 64-element (128-byte) column blocks of a row
 constexpr int kKStages = 3;         // K-pair ring depth
 constexpr int kVStages = 3;         // V-pair ring depth
+constexpr int kUnitRing = 8;        // units published ahead by the queue reader
 constexpr int kThreads = 384;       // 12 warps: producers / MMA, two softmax halves
 constexpr int kSoftmaxThreads = 256;  // both softmax warpgroups
 constexpr int kWgThreads = 128;       // one softmax warpgroup
@@ -72,15 +79,25 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;       // S buffer b at 128 b
 constexpr uint32_t kColO = 256;
 constexpr uint32_t kColP = 384;     // P buffer b at 384 + 64 b
+constexpr uint32_t kTileBytes = 64 * 128;  // 64 rows x 128 B (one 64-element column block of a tile)
+// The unit queue's readers: the V/Q producer, the two MMA issuers and every softmax thread.
+constexpr uint32_t kUnitReaders = 3 + kSoftmaxThreads;
 
-constexpr uint32_t kTileBytes = 64 * 128;                  // 64 rows x 128 B (one half of a tile)
-constexpr uint32_t kPairBytes = kHalves * 2 * kTileBytes;  // 32 KB: two tiles, both halves
-constexpr uint32_t kQBytes = kHalves * kTileBytes;         // 16 KB
+template <int kD>
+struct Cfg {
+  static_assert(kD == 64 || kD == 128, "head dimension 64 or 128");
+  static constexpr int kHalves = kD / 64;                      // 128-byte column blocks of a row
+  static constexpr uint32_t kPairBytes = kHalves * 2 * kTileBytes;  // two tiles, every block
+  static constexpr uint32_t kQBytes = kHalves * kTileBytes;
+  static constexpr uint32_t idesc_s = idesc_bf16(64, 128, false, false);  // A = Q, B = K, K-major
+  static constexpr uint32_t idesc_o = idesc_bf16(64, kD, false, true);    // A = P (TMEM), B = V
+};
 
+template <int kD>
 struct alignas(1024) SmemLayout {
-  uint8_t k[kKStages][kPairBytes];
-  uint8_t v[kVStages][kPairBytes];
-  uint8_t q[kQBytes];
+  uint8_t k[kKStages][Cfg<kD>::kPairBytes];
+  uint8_t v[kVStages][Cfg<kD>::kPairBytes];
+  uint8_t q[Cfg<kD>::kQBytes];
   uint64_t k_full[kKStages], k_empty[kKStages];
   uint64_t v_full[kVStages], v_empty[kVStages];
   uint64_t s_full[2], s_empty[2];
@@ -92,6 +109,8 @@ struct alignas(1024) SmemLayout {
   uint64_t o_empty;   // O read by the epilogue (softmax -> MMA)
   uint64_t drain[2];  // all MMAs of the S issuer / the PV issuer complete
   uint64_t m_ready[2];      // shift of a step (parity b) published by warpgroup b
+  uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];  // the unit queue's ring
+  int unit[kUnitRing];      // unit index, or -1 once the queue is exhausted
   float mrow[2][64];        // [step & 1][row]: that shift
   float xsum[2][2][4][16];  // [unit & 1][warpgroup][warp % 4][row]: running sums, end of a unit
   float xm[2][2][4][16];    // [unit & 1][warpgroup][warp % 4][row]: the shift they are relative to
@@ -100,14 +119,12 @@ struct alignas(1024) SmemLayout {
   int abort;
 };
 
-static_assert(sizeof(SmemLayout) + 1024 <= 232448, "shared memory per CTA");
+static_assert(sizeof(SmemLayout<128>) + 1024 <= 232448, "shared memory per CTA");
 constexpr int kAbsent = -0x7fffffff - 1;  // list entry beyond kv_cnt
-
-constexpr uint32_t idesc_s = idesc_bf16(64, 128, false, false);  // A = Q, B = K, K-major
-constexpr uint32_t idesc_o = idesc_bf16(64, 128, false, true);   // A = P (TMEM), B = V, MN-major
 
 struct UnitInfo {
   int b, h, i, cnt, npairs;
+  bool over, under;  // kv_cnt above kmax (clamped) / negative (treated as 0)
   const int32_t* list;
 };
 
@@ -117,10 +134,11 @@ __device__ __forceinline__ UnitInfo unit_info(const Geo& g, const AttnArgs& a, i
   const int bh = u / g.nT;
   r.h = bh % g.heads;
   r.b = bh / g.heads;
-  int c = a.kv_cnt[(long)bh * g.nT + r.i];
-  c = c < 0 ? 0 : (c > a.kmax ? a.kmax : c);
-  r.cnt = c;
-  r.npairs = (c + 1) >> 1;
+  const int c = a.kv_cnt[(long)bh * g.nT + r.i];
+  r.over = c > a.kmax;
+  r.under = c < 0;
+  r.cnt = r.under ? 0 : (r.over ? a.kmax : c);
+  r.npairs = (r.cnt + 1) >> 1;
   r.list = a.kv_idx + ((long)bh * g.nT + r.i) * a.kmax;
   return r;
 }
@@ -132,76 +150,70 @@ __device__ __forceinline__ int list_tile(const Geo& g, const UnitInfo& u, int e)
   return (j >= 0 && j < g.nT) ? j : -1;
 }
 
-__device__ __forceinline__ void fail(SmemLayout& s, int32_t* status) {
+template <int kD>
+__device__ __forceinline__ void fail(SmemLayout<kD>& s, int32_t* status) {
   s.abort = 1;
   report(status, T3D_DEV_TIMEOUT);
+}
+
+// Next unit from the ring (every reader calls it once per unit, in the same order): the unit index,
+// or -1 when the queue is exhausted or the wait gave up (then `ok` is cleared).
+template <int kD>
+__device__ __forceinline__ int take_unit(SmemLayout<kD>& s, long& nu, volatile int* abort_flag,
+                                         long long lim, bool& ok) {
+  const int slot = (int)(nu % kUnitRing);
+  if (!mbar_wait(&s.unit_full[slot], (uint32_t)((nu / kUnitRing) & 1), abort_flag, lim)) {
+    ok = false;
+    return -1;
+  }
+  const int u = s.unit[slot];
+  mbar_arrive(&s.unit_empty[slot]);
+  ++nu;
+  return u;
 }
 
 struct Maps {
   CUtensorMap q, k, v;
 };
 
-// Streams one operand's kept tile pairs (K or V) of every unit of this CTA, in step order, into a
-// ring of kStages pair buffers (lane 0 of a producer warp): step gp's pair goes to stage
-// gp % kStages once the MMAs that read the stage's previous pair have completed. With kLoadQ the
-// thread also loads each unit's query tile, ahead of the unit's pairs, once the previous unit's last
-// S has completed (the V producer: its pairs are needed only after the unit's first scores).
-template <int kStages, bool kLoadQ>
-__device__ __forceinline__ void produce_pairs(SmemLayout& s, const Geo& g, const AttnArgs& a,
-                                              const Maps& maps, const CUtensorMap* map,
-                                              uint8_t (*ring)[kPairBytes], uint64_t* full,
-                                              uint64_t* empty, volatile int* abort_flag) {
-  const int total_units = g.B * g.heads * g.nT;
-  long gp = 0, issued = 0;
-  int nq = 0;  // query tiles loaded
-  bool ok = true;
-  for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
-    const UnitInfo ui = unit_info(g, a, u);
-    if (ui.npairs == 0) continue;
-    if (kLoadQ) {
-      if (!mbar_wait(&s.q_empty, (uint32_t)((nq & 1) ^ 1), abort_flag)) {
-        ok = false;
-        break;
-      }
-      mbar_expect_tx(&s.q_full, kQBytes);
-      const int row0 = ui.b * g.Lp + ui.i * kTileElems;
-      for (int hh = 0; hh < kHalves; ++hh)
-        tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
-      ++nq;
-    }
-    for (int n = 0; n < ui.npairs; ++n, ++gp) {
-      const int st = (int)(gp % kStages);
-      if (!mbar_wait(&empty[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag)) {
-        ok = false;
-        break;
-      }
-      int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
-      if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
-      if (jb < 0) jb = ja;
-      mbar_expect_tx(&full[st], kPairBytes);
-      for (int hh = 0; hh < kHalves; ++hh) {
-        uint8_t* dst = ring[st] + hh * 2 * kTileBytes;
-        tma_load_3d(dst, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
-        tma_load_3d(dst + kTileBytes, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + jb * kTileElems);
-      }
-      ++issued;
-    }
+// Loads the K or V pair of step gp of unit ui into stage gp % kStages of a ring once the MMAs that
+// read the stage's previous pair have completed (lane 0 of a producer warp). False on a timeout.
+template <int kD, int kStages>
+__device__ __forceinline__ bool load_pair(const Geo& g, const UnitInfo& ui, int n, long gp,
+                                          const CUtensorMap* map,
+                                          uint8_t (*ring)[Cfg<kD>::kPairBytes], uint64_t* full,
+                                          uint64_t* empty, volatile int* abort_flag, long long lim) {
+  const int st = (int)(gp % kStages);
+  if (!mbar_wait(&empty[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag, lim)) return false;
+  int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
+  if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
+  if (jb < 0) jb = ja;
+  mbar_expect_tx(&full[st], Cfg<kD>::kPairBytes);
+  for (int hh = 0; hh < Cfg<kD>::kHalves; ++hh) {
+    uint8_t* dst = ring[st] + hh * 2 * kTileBytes;
+    tma_load_3d(dst, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
+    tma_load_3d(dst + kTileBytes, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + jb * kTileElems);
   }
-  if (!ok) fail(s, a.dev_status);
-  // Drain: the last loads issued must land before the CTA can exit.
-  for (long t = issued - kStages; t < issued; ++t)
-    if (t >= 0) mbar_wait(&full[t % kStages], (uint32_t)((t / kStages) & 1), nullptr);
-  if (kLoadQ && nq > 0) mbar_wait(&s.q_full, (uint32_t)((nq - 1) & 1), nullptr);
+  return true;
 }
 
+// Before exit, the last loads issued to a ring must have landed (bounded by the full limit).
+template <int kStages>
+__device__ __forceinline__ void drain_ring(uint64_t* full, long issued) {
+  for (long t = issued - kStages; t < issued; ++t)
+    if (t >= 0) mbar_wait(&full[t % kStages], (uint32_t)((t / kStages) & 1), nullptr);
+}
 
+template <int kD>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_sm100_kernel(const __grid_constant__ Maps maps, Geo g, AttnArgs a, float sl2) {
+  using C = Cfg<kD>;
   extern __shared__ uint8_t smem_raw[];
-  SmemLayout& s = *reinterpret_cast<SmemLayout*>(
+  SmemLayout<kD>& s = *reinterpret_cast<SmemLayout<kD>*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int total_units = g.B * g.heads * g.nT;
+  const long long lim = a.wait_cycles;
   volatile int* abort_flag = &s.abort;
 
   if (threadIdx.x == 0) {
@@ -210,11 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.s_full[t], 1);
       mbar_init(&s.s_empty[t], kWgThreads);
-    }
-    for (int t = 0; t < 2; ++t) {
       mbar_init(&s.p_full[t], kWgThreads);
       mbar_init(&s.m_ready[t], kWgThreads);
       mbar_init(&s.pv_done[t], 1);
+    }
+    for (int t = 0; t < kUnitRing; ++t) {
+      mbar_init(&s.unit_full[t], 1);
+      mbar_init(&s.unit_empty[t], kUnitReaders);
     }
     mbar_init(&s.q_full, 1);
     mbar_init(&s.q_empty, 1);
@@ -245,15 +259,71 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < 4) {
     regs_dec<kProducerRegs>();
     if (warp == 0) {
-      // ------------------------------------------------------------- K producer
-      if (lane == 0)
-        produce_pairs<kKStages, false>(s, g, a, maps, &maps.k, s.k, s.k_full, s.k_empty,
-                                       abort_flag);
+      // ------------------------------------------------------------- queue reader and K producer
+      if (lane == 0) {
+        uint32_t* next_unit = static_cast<uint32_t*>(a.workspace);
+        long nu = 0, gp = 0;
+        bool ok = true;
+        int cur = (int)atomicAdd(next_unit, 1u);
+        while (ok) {
+          const int slot = (int)(nu % kUnitRing);
+          if (!mbar_wait(&s.unit_empty[slot], (uint32_t)(((nu / kUnitRing) & 1) ^ 1), abort_flag,
+                         lim)) {
+            ok = false;
+            break;
+          }
+          const int u = cur < total_units ? cur : -1;
+          s.unit[slot] = u;
+          mbar_arrive(&s.unit_full[slot]);
+          ++nu;
+          if (u < 0) break;
+          // The next index is fetched now and used after this unit's loads, hiding its latency.
+          const int nxt = (int)atomicAdd(next_unit, 1u);
+          const UnitInfo ui = unit_info(g, a, u);
+          for (int n = 0; n < ui.npairs; ++n, ++gp) {  // gp counts the loads issued
+            if (!load_pair<kD, kKStages>(g, ui, n, gp, &maps.k, s.k, s.k_full, s.k_empty,
+                                         abort_flag, lim)) {
+              ok = false;
+              break;
+            }
+          }
+          cur = nxt;
+        }
+        if (!ok) fail(s, a.dev_status);
+        drain_ring<kKStages>(s.k_full, gp);
+      }
     } else if (warp == 3) {
       // ------------------------------------------------------------- V and Q producer
-      if (lane == 0)
-        produce_pairs<kVStages, true>(s, g, a, maps, &maps.v, s.v, s.v_full, s.v_empty,
-                                      abort_flag);
+      if (lane == 0) {
+        long nu = 0, gp = 0;
+        int nq = 0;  // query tiles loaded
+        bool ok = true;
+        while (ok) {
+          const int u = take_unit(s, nu, abort_flag, lim, ok);
+          if (u < 0) break;
+          const UnitInfo ui = unit_info(g, a, u);
+          if (ui.npairs == 0) continue;
+          if (!mbar_wait(&s.q_empty, (uint32_t)((nq & 1) ^ 1), abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&s.q_full, C::kQBytes);
+          const int row0 = ui.b * g.Lp + ui.i * kTileElems;
+          for (int hh = 0; hh < C::kHalves; ++hh)
+            tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
+          ++nq;
+          for (int n = 0; n < ui.npairs; ++n, ++gp) {  // gp counts the loads issued
+            if (!load_pair<kD, kVStages>(g, ui, n, gp, &maps.v, s.v, s.v_full, s.v_empty,
+                                         abort_flag, lim)) {
+              ok = false;
+              break;
+            }
+          }
+        }
+        if (!ok) fail(s, a.dev_status);
+        drain_ring<kVStages>(s.v_full, gp);
+        if (nq > 0) mbar_wait(&s.q_full, (uint32_t)((nq - 1) & 1), nullptr);
+      }
     } else if (warp == 1) {
       // ------------------------------------------------------------- S issuer
       // A thread's tcgen05.mma issue proceeds at about the rate the tensor pipe retires MMAs, so a
@@ -262,34 +332,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       // of the committing thread only, which is what each barrier below needs.
       if (lane == 0) {
         int active = 0;  // units with at least one pair, in order
-        long gp = 0;     // global step index
+        long nu = 0, gp = 0;  // units taken, global step index
         bool ok = true;
         // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4 and
         // every buffer lies below 256 KB), so each MMA's operand is a base descriptor plus a constant.
         const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
         const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
-        for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
-          const UnitInfo ui = unit_info(g, a, u);
-          const int np = ui.npairs;
+        while (ok) {
+          const int u = take_unit(s, nu, abort_flag, lim, ok);
+          if (u < 0) break;
+          const int np = unit_info(g, a, u).npairs;
           if (np == 0) continue;
-          if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag, lim)) { ok = false; break; }
           for (int n = 0; n < np; ++n, ++gp) {
             // S(gp) = Q . K_pair^T into S buffer gp & 1, once the softmax has read S(gp - 2).
             const int ks = (int)(gp % kKStages);
             const int b = (int)(gp & 1);
-            if (!mbar_wait(&s.k_full[ks], (uint32_t)((gp / kKStages) & 1), abort_flag) ||
-                !mbar_wait(&s.s_empty[b], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag)) {
+            if (!mbar_wait(&s.k_full[ks], (uint32_t)((gp / kKStages) & 1), abort_flag, lim) ||
+                !mbar_wait(&s.s_empty[b], (uint32_t)(((gp >> 1) & 1) ^ 1), abort_flag, lim)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t db0 = dk + (uint64_t)(ks * (kPairBytes >> 4));
+            const uint64_t db0 = dk + (uint64_t)(ks * (C::kPairBytes >> 4));
             const uint32_t d_s = tmem + kColS + 128 * b;
   #pragma unroll
             for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
               const int hh = kk >> 2, st = kk & 3;
               mma_bf16(d_s, dq + ((hh * kTileBytes + st * 32) >> 4),
-                       db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), idesc_s, kk ? 1u : 0u);
+                       db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), C::idesc_s, kk ? 1u : 0u);
             }
             mma_commit(&s.s_full[b]);
             mma_commit(&s.k_empty[ks]);
@@ -306,29 +377,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------- PV issuer
       if (lane == 0) {
         int active = 0;
-        long gp = 0;
+        long nu = 0, gp = 0;
         bool ok = true;
         const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
-        for (int u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
-          const UnitInfo ui = unit_info(g, a, u);
-          const int np = ui.npairs;
+        while (ok) {
+          const int u = take_unit(s, nu, abort_flag, lim, ok);
+          if (u < 0) break;
+          const int np = unit_info(g, a, u).npairs;
           if (np == 0) continue;
           for (int n = 0; n < np; ++n, ++gp) {
             // O (+)= P . V_pair of step gp; the unit's first PV overwrites O once the epilogue of the
             // previous unit has read it.
             const int vs = (int)(gp % kVStages);
-            if ((n == 0 && !mbar_wait(&s.o_empty, (uint32_t)((active & 1) ^ 1), abort_flag)) ||
-                !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag) ||
-                !mbar_wait(&s.p_full[gp & 1], (uint32_t)((gp >> 1) & 1), abort_flag)) {
+            if ((n == 0 && !mbar_wait(&s.o_empty, (uint32_t)((active & 1) ^ 1), abort_flag, lim)) ||
+                !mbar_wait(&s.v_full[vs], (uint32_t)((gp / kVStages) & 1), abort_flag, lim) ||
+                !mbar_wait(&s.p_full[gp & 1], (uint32_t)((gp >> 1) & 1), abort_flag, lim)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint64_t db0 = dv + (uint64_t)(vs * (kPairBytes >> 4));
+            const uint64_t db0 = dv + (uint64_t)(vs * (C::kPairBytes >> 4));
   #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)  // 16 keys (2048 bytes of V) per MMA
+            for (int kk = 0; kk < 8; ++kk)  // 16 keys (16 rows x 128 B of each column block) per MMA
               mma_bf16_ts(tmem + kColO, tmem + kColP + 64 * (uint32_t)(gp & 1) + 8 * kk,
-                          db0 + kk * (2048 >> 4), idesc_o, (n == 0 && kk == 0) ? 0u : 1u);
+                          db0 + kk * (2048 >> 4), C::idesc_o, (n == 0 && kk == 0) ? 0u : 1u);
             mma_commit(&s.pv_done[gp & 1]);
             mma_commit(&s.v_empty[vs]);
             if (n == np - 1) mma_commit(&s.o_full);
@@ -343,10 +415,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     named_bar(kTeardownBar, kThreads);
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+    if (warp == 1) {
+      __syncwarp();
+      tmem_dealloc(tmem, kTmemCols);
+    }
   } else {
     regs_inc<kSoftmaxRegs>();
     // ------------------------------------------------------------- softmax + epilogue (warps 4..11)
+    constexpr int kCols = kD / 2;       // output columns of one warpgroup
     const int wg = (warp - 4) >> 2;     // this warpgroup takes the steps gp with gp & 1 == wg
     const int sp = warp & 3;            // TMEM sub-partition: lanes [32 sp, 32 sp + 32)
     const int bar_id = 1 + sp;          // named barrier of warps w and w + 4 (same TMEM lanes)
@@ -357,8 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t t_s = lane_base + kColS + 128 * (uint32_t)wg;  // this warpgroup's S buffer
     const uint32_t t_p = lane_base + kColP + 64 * (uint32_t)wg;   // and P buffer
     const long ld = (long)g.heads * kD;
-    const int col0 = 64 * wg;           // output columns this warpgroup writes
+    const int col0 = kCols * wg;        // output columns this warpgroup writes
+    const bool reporter = wg == 0 && sp == 0 && lane == 0;  // records list-size problems
     int active = 0;
+    long nu = 0;
     long gp = 0;  // global index of the unit's first step
     bool reported = false;
     bool failed = false;  // a bounded wait gave up; carried to the pair's next barrier
@@ -366,14 +444,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       failed = true;
       *abort_flag = 1;
     };
-    for (int u = blockIdx.x; u < total_units; u += gridDim.x) {
+    while (true) {
+      bool got = true;
+      const int u = take_unit(s, nu, abort_flag, lim, got);
+      if (!got) give_up();
+      // Both warps of a pair leave together (a failed wait in either ends both).
+      if (named_bar_or(bar_id, 64, failed)) {
+        failed = true;
+        break;
+      }
+      if (u < 0) break;
       const UnitInfo ui = unit_info(g, a, u);
+      if (reporter && (ui.over || ui.under))
+        report(a.dev_status, ui.over ? T3D_DEV_OVERFLOW : T3D_DEV_INDEX_RANGE);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
       const int vci = s.vc[ui.i];
       __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
       if (ui.npairs == 0) {
         // No kept key tile: this thread's two output rows are zero (this warpgroup's columns).
-        for (int c = col0 + 2 * t0; c < col0 + 64; c += 8) {
+        for (int c = col0 + 2 * t0; c < col0 + kCols; c += 8) {
           *reinterpret_cast<uint32_t*>(out + r0 * ld + c) = 0u;
           *reinterpret_cast<uint32_t*>(out + r1 * ld + c) = 0u;
         }
@@ -391,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ja = ea, jb = eb;
         ea = (2 * n + 4 < ui.cnt) ? ui.list[2 * n + 4] : kAbsent;
         eb = (2 * n + 5 < ui.cnt) ? ui.list[2 * n + 5] : kAbsent;
-        if (!mbar_wait(&s.s_full[wg], (uint32_t)((gs >> 1) & 1), abort_flag)) give_up();
+        if (!mbar_wait(&s.s_full[wg], (uint32_t)((gs >> 1) & 1), abort_flag, lim)) give_up();
         tc_fence_after();
         uint32_t v[64];
         tmem_ld_16x256b_x16(t_s, v);
@@ -443,7 +532,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Every step waits for its predecessor's, so the two barriers never run a phase apart.
         float mp0 = -INFINITY, mp1 = -INFINITY;
         if (gs > 0) {
-          if (!mbar_wait(&s.m_ready[wg ^ 1], (uint32_t)(((gs - 1) >> 1) & 1), abort_flag))
+          if (!mbar_wait(&s.m_ready[wg ^ 1], (uint32_t)(((gs - 1) >> 1) & 1), abort_flag, lim))
             give_up();
           if (n > 0) {
             mp0 = s.mrow[wg ^ 1][r0];
@@ -466,13 +555,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // O follows it too: rescale the warp's rows (factor 1 where the shift held) once the
         // previous step's PV has landed; our own PV of this step is issued only after our P.
         if (n > 0 && __any_sync(0xffffffffu, up0 || up1)) {
-          if (!mbar_wait(&s.pv_done[wg ^ 1], (uint32_t)(((gs - 1) >> 1) & 1), abort_flag))
+          if (!mbar_wait(&s.pv_done[wg ^ 1], (uint32_t)(((gs - 1) >> 1) & 1), abort_flag, lim))
             give_up();
           tc_fence_after();
           const float a0 = !up0 ? 1.f : (mp0 == -INFINITY ? 0.f : ex2(mp0 - n0));
           const float a1 = !up1 ? 1.f : (mp1 == -INFINITY ? 0.f : ex2(mp1 - n1));
 #pragma unroll
-          for (int hc = 0; hc < 2; ++hc) {
+          for (int hc = 0; hc < kD / 64; ++hc) {
             uint32_t o[32];
             tmem_ld_16x256b_x8(lane_base + kColO + 64 * hc, o);
             tmem_wait_ld();
@@ -489,7 +578,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // Our P buffer is free once the PV of our previous step (two steps back) has landed.
         if (gs >= 2) {
-          if (!mbar_wait(&s.pv_done[wg], (uint32_t)(((gs - 2) >> 1) & 1), abort_flag)) give_up();
+          if (!mbar_wait(&s.pv_done[wg], (uint32_t)(((gs - 2) >> 1) & 1), abort_flag, lim))
+            give_up();
           tc_fence_after();
         }
         // P = exp2(x * scale - shift) as bf16 pairs: keys 8j + 2 t0, + 1 go to P column 4j + t0
@@ -552,7 +642,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         i0 = s0 > 0.f ? 1.f / s0 : 0.f;
         i1 = s1 > 0.f ? 1.f / s1 : 0.f;
       }
-      if (!mbar_wait(&s.o_full, (uint32_t)(active & 1), abort_flag)) give_up();
+      // Pruned-query variant: the output rows that take this lane's row (row 16 sp + lane for
+      // lane < 16), as a bit mask over the tile's 64 rows: a kept row takes itself, a pruned row
+      // its source row (a source outside the tile falls back to the row itself).
+      uint64_t takers = 0;
+      const int rown = 16 * sp + (lane & 15);
+      if (a.keep != nullptr) {
+        const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
+        const uint4* kp = reinterpret_cast<const uint4*>(a.keep + blk * kTileElems);
+        const uint4* sr = reinterpret_cast<const uint4*>(a.src_row + blk * kTileElems);
+#pragma unroll
+        for (int w4 = 0; w4 < 4; ++w4) {
+          const uint4 kv = kp[w4], sv = sr[w4];
+          const uint32_t kw[4] = {kv.x, kv.y, kv.z, kv.w}, sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int rr = 16 * w4 + e;
+            const uint32_t kb = (kw[e >> 2] >> (8 * (e & 3))) & 0xffu;
+            uint32_t sb = (sw[e >> 2] >> (8 * (e & 3))) & 0xffu;
+            if (kb != 0u || sb >= (uint32_t)kTileElems) sb = (uint32_t)rr;
+            if (sb == (uint32_t)rown) takers |= 1ull << rr;
+          }
+        }
+      } else {
+        takers = 1ull << rown;
+      }
+      if (!mbar_wait(&s.o_full, (uint32_t)(active & 1), abort_flag, lim)) give_up();
       tc_fence_after();
       failed = __any_sync(0xffffffffu, failed);  // the TMEM loads below are warp-collective
       if (!failed) {
@@ -560,15 +675,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // (the M = 64 layout), 32 columns per load, so a row goes out in 16-byte stores. Its 1 / l
         // comes from the threads that own the row in the 16x256b layout (row r0 of lanes 4L.., or
         // r1).
-        const int rown = 16 * sp + (lane & 15);
         const float ia = __shfl_sync(0xffffffffu, i0, 4 * (lane & 7));
         const float ib = __shfl_sync(0xffffffffu, i1, 4 * (lane & 7));
         const float inv = (lane & 15) < 8 ? ia : ib;
-        const long blk = ((long)ui.b * g.heads + ui.h) * g.nT + ui.i;
-        const uint8_t* keep = a.keep ? a.keep + blk * kTileElems : nullptr;
-        const uint8_t* srcr = a.src_row ? a.src_row + blk * kTileElems : nullptr;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < kCols / 32; ++c) {
           const int cc = col0 + 32 * c;
           uint32_t o[32];
           tmem_ld32(lane_base + kColO + cc, o);
@@ -582,25 +693,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                        __uint_as_float(o[2 * e + 1]) * inv);
               w[e] = *reinterpret_cast<uint32_t*>(&y);
             }
-            // Row rr of the output takes the result of row src(rr): rr itself, or for a query row
-            // pruned by BSA its kept source row. Rows past the tile's valid count are zero.
-            auto put = [&](int rr) {
+            // Every output row that takes this row's result; rows past the tile's valid count
+            // are zero.
+            for (uint64_t m = takers; m != 0; m &= m - 1) {
+              const int rr = __ffsll((long long)m) - 1;
               uint4* dst = reinterpret_cast<uint4*>(out + rr * ld + cc);
               const bool zero = rr >= vci;
 #pragma unroll
               for (int k4 = 0; k4 < 4; ++k4) dst[k4] = zero ? make_uint4(0u, 0u, 0u, 0u) : w4[k4];
-            };
-            if (keep == nullptr) {
-              put(rown);
-            } else {
-              for (int rr = 0; rr < kTileElems; ++rr) {
-                int sr = rr;
-                if (!keep[rr]) {
-                  sr = srcr[rr];
-                  if (sr >= kTileElems) sr = rr;
-                }
-                if (sr == rown) put(rr);
-              }
             }
           }
         }
@@ -655,21 +755,42 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-}  // namespace
+// Dynamic shared memory of a CTA: the layout plus alignment slack, and never less than half of an
+// SM's 228 KB, so that no SM ever holds two CTAs (the second would wait for the first's TMEM).
+template <int kD>
+constexpr size_t smem_bytes() {
+  return sizeof(SmemLayout<kD>) + 1024 > 120 * 1024 ? sizeof(SmemLayout<kD>) + 1024 : 120 * 1024;
+}
 
-cudaError_t launch_attn_sm100(const Geo& g, const AttnArgs& a, cudaStream_t s) {
-  Maps maps;
-  if (!make_map(&maps.q, a.q, g) || !make_map(&maps.k, a.k, g) || !make_map(&maps.v, a.v, g))
-    return cudaErrorInvalidValue;
-  const size_t smem = sizeof(SmemLayout) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel,
+template <int kD>
+cudaError_t launch_d(const Maps& maps, const Geo& g, const AttnArgs& a, cudaStream_t s) {
+  const size_t smem = smem_bytes<kD>();
+  cudaError_t e = cudaFuncSetAttribute(attn_sm100_kernel<kD>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int units = g.B * g.heads * g.nT;
   const int grid = units < sm_count() ? units : sm_count();
   const float sl2 = a.scale * 1.4426950408889634f;
-  attn_sm100_kernel<<<grid, kThreads, smem, s>>>(maps, g, a, sl2);
+  attn_sm100_kernel<kD><<<grid, kThreads, smem, s>>>(maps, g, a, sl2);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t attn_workspace_bytes(const Geo& g, int kmax) {
+  (void)g;
+  (void)kmax;
+  return kAttnWorkspaceBytes;
+}
+
+cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s) {
+  Maps maps;
+  if (!make_map(&maps.q, a.q, g) || !make_map(&maps.k, a.k, g) || !make_map(&maps.v, a.v, g))
+    return cudaErrorInvalidValue;
+  // The unit queue starts at zero on every launch.
+  cudaError_t e = cudaMemsetAsync(a.workspace, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
+  return g.D == 128 ? launch_d<128>(maps, g, a, s) : launch_d<64>(maps, g, a, s);
 }
 
 }  // namespace t3d

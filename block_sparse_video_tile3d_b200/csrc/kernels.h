@@ -38,15 +38,16 @@ struct AttnArgs {
   const uint8_t* keep;
   const uint8_t* src_row;
   float scale;
-  void* workspace;
+  void* workspace;        // at least kAttnWorkspaceBytes: the unit queue's counter
   size_t ws_bytes;
   int32_t* dev_status;
+  long long wait_cycles;  // limit of each pipeline wait, in clock cycles
 };
 
+// Device scratch of the attention kernel: one 32-bit unit counter, padded to 256 bytes.
+constexpr size_t kAttnWorkspaceBytes = 256;
 size_t attn_workspace_bytes(const Geo& g, int kmax);
-// D = 128: tcgen05/TMEM/TMA kernel (attn_sm100.cu). D = 64: warp-MMA kernel (attn_mma.cu).
+// tcgen05/TMEM/TMA kernel (attn_sm100.cu), D = 64 or 128.
 cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s);
-cudaError_t launch_attn_sm100(const Geo& g, const AttnArgs& a, cudaStream_t s);
-cudaError_t launch_attn_mma(const Geo& g, const AttnArgs& a, cudaStream_t s);
 
 }  // namespace t3d

@@ -312,6 +312,17 @@ __global__ void __launch_bounds__(kSelThreads) topk_kernel(Geo g, const float* _
 __device__ int select_mass_row(float* row, int nT, float scale, float mass, int min_k, int kmax,
                                int32_t* out, int32_t* dev_status, int* hist) {
   const int lane = threadIdx.x & 31;
+  if (mass >= 1.f) {
+    // Every probability of a softmax is positive, so the running sum reaches 1 only with the last
+    // tile: all tiles are kept (the most probable kmax when they do not fit). Deciding this before
+    // the exponentials keeps tiles whose fp32 exponential underflows to 0.
+    if (nT <= kmax) {
+      for (int j = lane; j < nT; j += 32) out[j] = j;
+      return nT;
+    }
+    if (lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
+    return select_topk_row(row, nT, kmax, out, hist);
+  }
   float mx = -INFINITY;
   for (int j = lane; j < nT; j += 32) mx = fmaxf(mx, row[j]);
   mx = warp_max(mx);

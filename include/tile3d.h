@@ -11,8 +11,8 @@
  * Conventions shared by every call
  * --------------------------------
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library never frees or
- *    keeps them. The only device memory the library touches beyond its arguments is the
- *    caller-sized workspace of block_sparse_attn_fwd.
+ *    keeps them, and allocates no device memory. The only device memory it touches beyond its
+ *    arguments is the caller-sized workspace of block_sparse_attn_fwd.
  *  - Activations are bf16, layout [B, L, heads, D] with D fastest (raster order, L = T*H*W) or
  *    [B, Lp, heads, D] (tile order, Lp = 64 * nT). Tile i occupies rows [64 i, 64 i + 64); its
  *    vc_i valid tokens fill slots 0 .. vc_i - 1 in in-tile raster order, the rest are zero.
@@ -65,7 +65,7 @@ typedef struct {
 /* Human-readable description of the last error on this host thread ("" if none). */
 const char* t3d_last_error_string(void);
 
-/* Library version, e.g. "0.1.0". */
+/* Library version, e.g. "0.2.0". */
 const char* t3d_version(void);
 
 /*
@@ -204,12 +204,19 @@ t3d_status block_mask_to_index(const t3d_geom* g, const uint8_t* mask, int kmax,
  *   kv_idx:  in,  int32 [B, heads, nT, kmax], the first kv_cnt entries of each row used (any
  *            order; each index in [0, nT), duplicates not allowed). kv_cnt: in, int32 [B,heads,nT].
  *   keep, src_row: NULL, or the BSA outputs of tile_prune_queries (then L must equal Lp): only
- *            kept rows attend and pruned rows take the output of src_row.
+ *            kept rows attend and pruned rows take the output of src_row (which must name a kept
+ *            row of the same tile; an entry >= 64 makes the row take its own result).
  *   softmax_scale: must be 1/sqrt(D) (see above), else T3D_ERR_INVALID.
  *   causal != 0 or num_kv_heads != heads: T3D_ERR_UNSUPPORTED.
- *   workspace: device scratch of at least block_sparse_attn_workspace_size() bytes (may be NULL
- *            if that size is 0). Its contents on entry do not matter.
- *   dev_status: in/out device int32, or NULL. Out-of-range indices are skipped (T3D_DEV_INDEX_RANGE).
+ *   workspace: device scratch of at least block_sparse_attn_workspace_size() bytes (256: the
+ *            counter of the kernel's work queue, which the call zeroes on `stream` before its
+ *            launch). Its contents on entry do not matter; calls that may run at the same time
+ *            need workspaces of their own.
+ *   dev_status: in/out device int32, or NULL. Out-of-range indices are skipped and a negative
+ *            kv_cnt is read as 0 (T3D_DEV_INDEX_RANGE); a kv_cnt above kmax is read as kmax
+ *            (T3D_DEV_OVERFLOW); a pipeline wait that gave up sets T3D_DEV_TIMEOUT.
+ * The work units (batch, head, query tile) are handed out dynamically to one CTA per SM, so query
+ * tiles that keep different numbers of key tiles are balanced across the GPU.
  * fp32 accumulation and softmax; bf16 output rounded to nearest even.
  */
 t3d_status block_sparse_attn_fwd(const t3d_geom* g, const void* q, const void* k, const void* v,

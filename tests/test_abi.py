@@ -1,7 +1,8 @@
-"""The C ABI library loads, exports every call include/tile3d.h declares, computes the host-side
-geometry like the oracle, and rejects bad arguments on the host (no GPU needed: every call here
-fails validation before anything is enqueued)."""
+"""The C ABI library loads, exports every call the headers under include/ declare, computes the
+host-side geometry like the oracle, and rejects bad arguments on the host (no GPU needed: every
+call here fails validation before anything is enqueued)."""
 import ctypes
+import glob
 import math
 import os
 import re
@@ -13,13 +14,15 @@ from block_sparse_video_tile3d_b200 import _lib
 from block_sparse_video_tile3d_b200._lib import Geom, lib
 from oracle import tiling
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "tile3d.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include")
 
 
 def _declared():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(\w+)\s*\(", text, flags=re.M))
+    names = set()
+    for h in sorted(glob.glob(os.path.join(INCLUDE, "*.h"))):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names |= set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(\w+)\s*\(", text, flags=re.M))
+    return names
 
 
 def test_every_declared_symbol_is_exported_and_bound():
@@ -28,7 +31,7 @@ def test_every_declared_symbol_is_exported_and_bound():
             "tile3d_gather", "tile_select_mass", "tile_prune_queries", "tile_prune_queries_ratio",
             "block_mask_to_index",
             "tile3d_geometry", "block_sparse_attn_workspace_size", "t3d_last_error_string",
-            "t3d_version"} <= names
+            "t3d_version", "t3d_testing_set_wait_cycles"} <= names
     for n in names:
         assert hasattr(lib, n), n
         assert n in _lib.SIGNATURES, n
@@ -51,11 +54,12 @@ def _g(B=1, T=4, H=8, W=8, heads=2, D=64):
     return ctypes.byref(Geom(B, T, H, W, heads, D))
 
 
-def _attn(g=None, scale=None, causal=0, nkv=2, kmax=2, keep=None, src=None, q=FAKE, ws=0):
+def _attn(g=None, scale=None, causal=0, nkv=2, kmax=2, keep=None, src=None, q=FAKE, ws=256,
+          wsp=FAKE):
     g = g or _g()
     scale = 1.0 / math.sqrt(64) if scale is None else scale
     return lib.block_sparse_attn_fwd(g, q, FAKE, FAKE, FAKE, FAKE, FAKE, kmax, keep, src, scale,
-                                     causal, nkv, None, ws, None, None)
+                                     causal, nkv, wsp, ws, None, None)
 
 
 def test_attention_contract_rejections():
@@ -74,6 +78,18 @@ def test_attention_contract_rejections():
     assert _attn(g=_g(D=96)) == _lib.T3D_ERR_UNSUPPORTED
     assert _attn(g=_g(B=0)) == _lib.T3D_ERR_INVALID
     assert _attn(g=_g(T=4 * 17, H=4 * 16, W=4 * 16)) == _lib.T3D_ERR_UNSUPPORTED  # > 4096 tiles
+    # the work queue's counter lives in the caller's workspace: too small or missing is rejected
+    assert lib.block_sparse_attn_workspace_size(_g(), 2) == 256
+    assert _attn(ws=255) == _lib.T3D_ERR_INVALID
+    assert b"workspace" in lib.t3d_last_error_string()
+    assert _attn(wsp=None) == _lib.T3D_ERR_INVALID
+    assert _attn(wsp=ODD) == _lib.T3D_ERR_INVALID
+
+
+def test_testing_hook_validates_and_resets():
+    assert lib.t3d_testing_set_wait_cycles(-1) == _lib.T3D_ERR_INVALID
+    assert lib.t3d_testing_set_wait_cycles(1000) == _lib.T3D_OK
+    assert lib.t3d_testing_set_wait_cycles(0) == _lib.T3D_OK  # back to the default limit
 
 
 def test_scale_tolerance_matches_isclose():

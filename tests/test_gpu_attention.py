@@ -6,7 +6,8 @@ import pytest
 import torch
 
 from block_sparse_video_tile3d_b200 import block_sparse_attn_fwd, tile3d_scatter, workloads
-from block_sparse_video_tile3d_b200._lib import T3D_DEV_INDEX_RANGE
+from block_sparse_video_tile3d_b200._lib import (T3D_DEV_INDEX_RANGE, T3D_DEV_OVERFLOW,
+                                                  T3D_DEV_TIMEOUT, check, lib)
 from oracle import attention, bsa, select, tiling
 from tests.helpers import assert_attn_close, f64
 
@@ -106,8 +107,9 @@ def test_attention_empty_rows_and_large_magnitudes():
     assert_attn_close(got, want)
 
 
-def test_attention_out_of_range_index_is_skipped_and_reported():
-    B, T, H, W, heads, D = 1, 8, 8, 8, 1, 64
+@pytest.mark.parametrize("D", [64, 128])
+def test_attention_out_of_range_index_is_skipped_and_reported(D):
+    B, T, H, W, heads = 1, 8, 8, 8, 1
     q, k, v = _qkv(B, T, H, W, heads, D, seed=7)
     sets = _random_sets(B, heads, 8, 0.5, seed=8)
     kv_idx, kv_cnt = _lists(sets, B, heads, 8, 8)
@@ -120,6 +122,84 @@ def test_attention_out_of_range_index_is_skipped_and_reported():
     ot = block_sparse_attn_fwd(qt, kt, vt, idx.cuda(), kv_cnt, T, H, W, dev_status=status)
     assert int(status.item()) & T3D_DEV_INDEX_RANGE
     assert_attn_close(f64(ot), _oracle(q, k, v, T, H, W, sets))
+
+
+def test_attention_list_counts_outside_capacity():
+    """kv_cnt above kmax reads the first kmax entries (T3D_DEV_OVERFLOW); a negative kv_cnt reads as
+    an empty list (T3D_DEV_INDEX_RANGE, zero output rows)."""
+    B, T, H, W, heads, D = 1, 8, 8, 8, 2, 128
+    q, k, v = _qkv(B, T, H, W, heads, D, seed=12)
+    sets = _random_sets(B, heads, 8, 0.6, seed=13)
+    kmax = 8
+    kv_idx, kv_cnt = _lists(sets, B, heads, 8, kmax)
+    row = next(i for i in range(8) if len(sets[0][0][i]) >= 3)
+    cnt = kv_cnt.cpu()
+    cnt[0, 0, row] = kmax + 3          # claims more entries than a row holds
+    cnt[0, 1, 5] = -4                  # a negative count
+    want_sets = [[list(sets[0][0]), list(sets[0][1])]]
+    want_sets[0][0][row] = np.asarray(kv_idx[0, 0, row].cpu().numpy(), dtype=np.int64)
+    want_sets[0][1][5] = np.zeros(0, dtype=np.int64)
+    # the row's kmax entries: its own list followed by fill values, which are out of range and
+    # skipped (so the range bit is expected too)
+    want_sets[0][0][row] = want_sets[0][0][row][(want_sets[0][0][row] >= 0)
+                                                & (want_sets[0][0][row] < 8)]
+    qt, kt, vt = (tile3d_scatter(x.cuda(), T, H, W) for x in (q, k, v))
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ot = block_sparse_attn_fwd(qt, kt, vt, kv_idx, cnt.cuda(), T, H, W, dev_status=status)
+    st = int(status.item())
+    assert st & T3D_DEV_OVERFLOW and st & T3D_DEV_INDEX_RANGE
+    got = f64(ot)
+    assert np.all(got[0, 64 * 5:64 * 6, 1] == 0.0)
+    assert_attn_close(got, _oracle(q, k, v, T, H, W, want_sets))
+
+
+def test_attention_uneven_lists_balanced_queue():
+    """Units of very different lengths (every tile kept for one query tile in five, one to three
+    for the rest) over more units than SMs: the dynamic unit queue must cover every unit once."""
+    B, T, H, W, heads, D = 1, 9, 10, 13, 8, 128
+    nT = 36
+    q, k, v = _qkv(B, T, H, W, heads, D, seed=14)
+    rng = np.random.default_rng(15)
+    sets = [[[np.arange(nT) if (h * nT + i) % 5 == 0 else
+              np.sort(rng.choice(nT, int(rng.integers(1, 4)), replace=False))
+              for i in range(nT)] for h in range(heads)]]
+    got, st = _run(q, k, v, T, H, W, sets)
+    assert st == 0
+    assert_attn_close(got, _oracle(q, k, v, T, H, W, sets))
+
+
+def test_attention_repeated_calls_share_workspace():
+    """The queue counter in the workspace is reset by every call: two calls with one workspace
+    give the same output, bit for bit."""
+    B, T, H, W, heads, D = 1, 9, 10, 13, 6, 64
+    q, k, v = _qkv(B, T, H, W, heads, D, seed=16)
+    sets = _random_sets(B, heads, 36, 0.3, seed=17)
+    kv_idx, kv_cnt = _lists(sets, B, heads, 36, 36)
+    qt, kt, vt = (tile3d_scatter(x.cuda(), T, H, W) for x in (q, k, v))
+    ws = torch.full((256,), 0x7f, dtype=torch.uint8, device="cuda")  # not zero on entry
+    o1 = block_sparse_attn_fwd(qt, kt, vt, kv_idx, kv_cnt, T, H, W, workspace=ws)
+    o2 = block_sparse_attn_fwd(qt, kt, vt, kv_idx, kv_cnt, T, H, W, workspace=ws)
+    assert torch.equal(o1, o2)
+    assert_attn_close(f64(o1), _oracle(q, k, v, T, H, W, sets))
+
+
+def test_attention_bounded_wait_gives_up_cleanly():
+    """With the pipeline wait limit cut to 200 clock cycles the first wait that is not already
+    satisfied gives up: the kernel must record T3D_DEV_TIMEOUT, let its copies and MMAs in flight
+    finish, free its tensor memory and return; the next call at the normal limit must be exact."""
+    B, T, H, W, heads, D = 1, 8, 8, 8, 2, 128
+    q, k, v = _qkv(B, T, H, W, heads, D, seed=18)
+    sets = _random_sets(B, heads, 8, 0.5, seed=19)
+    try:
+        check(lib.t3d_testing_set_wait_cycles(200))
+        _, st = _run(q, k, v, T, H, W, sets)
+    finally:
+        check(lib.t3d_testing_set_wait_cycles(0))
+    torch.cuda.synchronize()  # the context is still usable
+    assert st & T3D_DEV_TIMEOUT
+    got, st2 = _run(q, k, v, T, H, W, sets)
+    assert st2 == 0
+    assert_attn_close(got, _oracle(q, k, v, T, H, W, sets))
 
 
 def test_attention_pruned_queries():

@@ -4,7 +4,8 @@ import numpy as np
 import pytest
 import torch
 
-from block_sparse_video_tile3d_b200 import TileSparseAttention, workloads
+from block_sparse_video_tile3d_b200 import (TileSparseAttention, block_sparse_attn_fwd,
+                                            workloads)
 from oracle import attention, pipeline, pool, select, tiling
 from tests.helpers import assert_attn_close, check_topk_sets, f64, gpu_sets
 
@@ -35,6 +36,12 @@ def test_ragged_topk_end_to_end():
                for a, b in zip(got_sets[bb][h], ref["sets"][bb][h]))
     if same:
         assert_attn_close(f64(out), ref["o"])
+    else:
+        # a near-tie row selected differently (within the gap rule): the fine stage is checked
+        # with the oracle's own lists fed in, on the pipeline's tiled tensors
+        idx, cnt = _lists(ref["sets"], w.B, w.heads, w.nT, w.k)
+        ot = block_sparse_attn_fwd(m.qt, m.kt, m.vt, idx, cnt, w.T, w.H, w.W)
+        assert_attn_close(f64(ot), ref["ot"])
 
 
 def test_mask_mode_end_to_end_sliding():
@@ -45,6 +52,19 @@ def test_mask_mode_end_to_end_sliding():
     out = m(q.cuda(), k.cuda(), v.cuda())
     ref = pipeline.forward(q, k, v, w.T, w.H, w.W, "mask", scale=w.scale, mask=mask.numpy())
     assert_attn_close(f64(out), ref["o"])
+
+
+def _lists(sets, B, heads, nT, kmax):
+    """Nested per-row index lists -> (kv_idx, kv_cnt) int32 CUDA tensors."""
+    idx = np.zeros((B, heads, nT, kmax), dtype=np.int32)
+    cnt = np.zeros((B, heads, nT), dtype=np.int32)
+    for b in range(B):
+        for h in range(heads):
+            for i in range(nT):
+                s_ = np.asarray(sets[b][h][i], dtype=np.int32)
+                idx[b, h, i, :len(s_)] = s_
+                cnt[b, h, i] = len(s_)
+    return torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda()
 
 
 def _exact_rows(got_sets, ref_sets, B, heads, nT):
@@ -111,3 +131,106 @@ def test_workload_topk_full_size(name, heads_checked):
         for i in tiles:
             rows = slice(64 * i, 64 * i + 64)
             assert_attn_close(got_t[0, rows, 0], want[0, rows, 0], what=f"{name} tile {(h, i)}")
+
+
+def _pruning_agrees(keep, src, okeep, osrc, ocos, oqt, thresh, b, h, i):
+    """Kept rows identical wherever the oracle's cosine to the block mean is decided (more than
+    1e-4 from the threshold), and every pruned row's source the oracle's wherever the best kept
+    row is decided (gap above 1e-4), else a kept row. True if the whole block agrees."""
+    decided = np.abs(ocos[b, h, i] - thresh) > 1e-4
+    np.testing.assert_array_equal(keep[b, h, i][decided], okeep[b, h, i][decided])
+    if not np.array_equal(keep[b, h, i], okeep[b, h, i]):
+        return False
+    rows = oqt[b, 64 * i:64 * i + 64, 0]
+    kept = np.nonzero(okeep[b, h, i])[0]
+    nrm = np.linalg.norm(rows, axis=1)
+    for r in np.nonzero(~okeep[b, h, i])[0]:
+        c = rows[kept] @ rows[r] / np.maximum(nrm[kept] * nrm[r], 1e-300)
+        top = np.sort(c)[::-1]
+        if len(top) < 2 or top[0] - top[1] > 1e-4:
+            assert src[b, h, i, r] == osrc[b, h, i, r]
+        else:
+            assert keep[b, h, i, src[b, h, i, r]]
+    return True
+
+
+@pytest.mark.parametrize("structured", [False, True])
+def test_bsa_full_size(structured):
+    """The BSA workload at full size (16x32x56, 12 heads, D = 128, prune at cosine 0.95, KV mass
+    0.9 at scale 1/sqrt(D), so kmax = nT = 448 and about 85% of the tiles kept), on the plain data
+    and on the structured-query variant. The oracle reruns three heads on single-head slices:
+    pruning must match where it is decided, kept sets exactly where the mass margins allow, and
+    the output element by element on sampled tiles; the fine stage is also run with the oracle's
+    own lists and pruning fed in, and compared on every sampled tile."""
+    w = workloads.WORKLOADS["bsa"]
+    q, k, v = workloads.make_qkv(w)
+    if structured:
+        q = workloads.make_structured_queries(w, q)
+    m = TileSparseAttention(w.B, w.T, w.H, w.W, w.heads, w.D, mode="bsa", mass=w.mass,
+                            min_k=w.min_kv, cos_thresh=w.cos_thresh)
+    out = f64(m(q.cuda(), k.cuda(), v.cuda()))
+    assert m.device_status() == 0
+    keep = m.keep.cpu().numpy().astype(bool)
+    src = m.src_row.cpu().numpy().astype(np.int64)
+    got_sets = gpu_sets(m.kv_idx, m.kv_cnt)
+    vc = tiling.variable_block_sizes(w.T, w.H, w.W)
+    pos = tiling.padded_positions(w.T, w.H, w.W)
+    rng = np.random.default_rng(21 + structured)
+    n_exact = n_rows = 0
+    for h in (0, 5, 11):
+        sl = lambda x: f64(x[:, :, h:h + 1])  # noqa: E731
+        qt, kt, vt = (tiling.tile_scatter(sl(x), w.T, w.H, w.W) for x in (q, k, v))
+        res = pipeline.coarse_select(qt, kt, vc, "bsa", scale=w.scale, tau=w.mass,
+                                     min_k=w.min_kv, cos_thresh=w.cos_thresh)
+        okeep, osrc, ocos, S = res["keep"], res["src"], res["cos"], res["S"]
+        if structured:
+            assert (~okeep).sum() > 1000  # the structured cells prune
+        agree = [_pruning_agrees(keep[:, h:h + 1], src[:, h:h + 1], okeep, osrc, ocos, qt,
+                                 w.cos_thresh, 0, 0, i) for i in range(w.nT)]
+        assert sum(agree) >= 0.99 * w.nT
+        for i in range(w.nT):
+            if not agree[i]:
+                continue
+            n_rows += 1
+            row = S[0, 0, i]
+            mm = select.mass_margins(row, w.scale, w.mass, w.min_kv)
+            g, want_i = got_sets[0][h][i], res["sets"][0][0][i]
+            assert np.all(np.diff(g) > 0)
+            if mm["cut_gap"] > 1e-3 and mm["sum_margin"] > 1e-4:
+                np.testing.assert_array_equal(g, want_i, err_msg=f"head {h} tile {i}")
+                n_exact += 1
+            else:  # near a decision boundary: a valid prefix of the ranking with mass ~ tau
+                p = select.softmax_row(w.scale * row)
+                dropped = np.setdiff1d(np.arange(w.nT), g)
+                if dropped.size:
+                    assert p[dropped].max() <= p[g].min() * (1 + 1e-3) + 1e-7
+                assert abs(len(g) - len(want_i)) <= 2
+                assert p[g].sum() >= w.mass - 1e-4
+                assert p[g].sum() - p[g].min() < w.mass + 1e-4
+        # sampled output tiles where pruning and sets agree, through the whole pipeline
+        tiles = [int(t) for t in rng.choice(w.nT, 5, replace=False)] + [w.nT - 1]
+        want = attention.block_sparse_attention(qt, kt, vt, vc, res["sets"], w.scale, keep=okeep,
+                                                src=osrc, q_tiles=[(0, 0, i) for i in tiles])
+        got_t = np.zeros_like(want)
+        got_t[:, pos, 0] = out[:, :, h]
+        for i in tiles:
+            if agree[i] and np.array_equal(got_sets[0][h][i], res["sets"][0][0][i]):
+                rows = slice(64 * i, 64 * i + 64)
+                assert_attn_close(got_t[0, rows, 0], want[0, rows, 0], what=f"bsa tile {(h, i)}")
+        # the fine stage with the oracle's lists and pruning fed in, on every sampled tile
+        full_sets = [[res["sets"][0][0] if hh == h else [np.arange(1)] * w.nT
+                      for hh in range(w.heads)]]
+        idx, cnt = _lists(full_sets, 1, w.heads, w.nT, w.nT)
+        kp = m.keep.clone()
+        sp = m.src_row.clone()
+        kp[0, h] = torch.from_numpy(okeep[0, 0].astype(np.uint8)).cuda()
+        sp[0, h] = torch.from_numpy(osrc[0, 0].astype(np.uint8)).cuda()
+        ot = f64(block_sparse_attn_fwd(m.qt, m.kt, m.vt, idx, cnt, w.T, w.H, w.W, keep=kp,
+                                       src_row=sp))
+        for i in tiles:
+            rows = slice(64 * i, 64 * i + 64)
+            assert_attn_close(ot[0, rows, h], want[0, rows, 0], what=f"bsa fed tile {(h, i)}")
+    # 26% (plain) and 21% (structured) of these rows are decided by the mass margins in the
+    # oracle's own fp64 scores: the pooled softmax is near uniform, so neighbouring tiles at the cut
+    # often differ by less than the 1e-3 relative gap
+    assert n_exact >= 0.15 * n_rows

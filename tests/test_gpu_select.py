@@ -109,6 +109,32 @@ def test_mass_overflow_truncates_to_most_probable():
                 np.testing.assert_array_equal(got[0][h][i], select.select_topk_row(S[0, h, i], 5))
 
 
+@pytest.mark.parametrize("kmax", [None, 20])
+def test_mass_one_keeps_every_tile_with_underflowing_scores(kmax):
+    """At mass 1 every tile is kept (the most probable kmax when they do not fit), even where the
+    scaled scores are spread so widely that fp32 exponentials of the tail underflow to 0."""
+    T, H, W, D = 9, 10, 13, 64
+    nT = 36
+    pq, pk = _pooled(1, 2, nT, D, seed=23)
+    pq = (pq * 40.0).contiguous()
+    S = select.tile_scores(f64(pq), f64(pk))
+    spread = S.max(axis=-1, keepdims=True) - S
+    assert (spread > 104.0).any()  # exp(-104) is below fp32's smallest subnormal
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    kv_idx, kv_cnt = tile_select_mass(pq.cuda(), pk.cuda(), T, H, W, 1.0, 1.0, 1, kmax=kmax,
+                                      dev_status=status)
+    got = gpu_sets(kv_idx, kv_cnt)
+    want = select.select_mass(S, 1.0, 1.0, 1)
+    for h in range(2):
+        for i in range(nT):
+            np.testing.assert_array_equal(want[0][h][i], np.arange(nT))
+            if kmax is None:
+                np.testing.assert_array_equal(got[0][h][i], np.arange(nT))
+            elif select.topk_gap(S[0, h, i][None], kmax)[0] > 1e-3:
+                np.testing.assert_array_equal(got[0][h][i], select.select_topk_row(S[0, h, i], kmax))
+    assert bool(int(status.item()) & T3D_DEV_OVERFLOW) == (kmax is not None)
+
+
 @pytest.mark.parametrize("kmax", [None, 4])
 def test_mask_to_index_bit_exact(kmax):
     T, H, W, D = 21, 30, 52, 128
