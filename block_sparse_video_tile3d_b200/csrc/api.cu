@@ -269,4 +269,49 @@ t3d_status block_sparse_attn_fwd(const t3d_geom* g, const void* q, const void* k
   return cuda_status(t3d::launch_attn(geo, a, as_stream(stream)), "block_sparse_attn_fwd");
 }
 
+t3d_status block_sparse_attn_fwd_noalloc(const t3d_geom* g, const void* q, const void* k,
+                                         const void* v, void* o, const int32_t* kv_idx,
+                                         const int32_t* kv_cnt, int kmax, const uint8_t* keep,
+                                         const uint8_t* src_row, float softmax_scale, int causal,
+                                         int num_kv_heads, int32_t* dev_status,
+                                         t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  if (causal != 0)
+    return fail(T3D_ERR_UNSUPPORTED, "the attention is bidirectional; causal=1 is unsupported");
+  if (num_kv_heads != g->heads)
+    return fail(T3D_ERR_UNSUPPORTED,
+                "grouped-query attention is unsupported (num_kv_heads=%d, heads=%d)", num_kv_heads,
+                g->heads);
+  const double expected = 1.0 / sqrt((double)g->D);
+  const double diff = fabs((double)softmax_scale - expected);
+  if (!(diff <= fmax(1e-4 * fmax(fabs((double)softmax_scale), expected), 1e-5)))
+    return fail(T3D_ERR_INVALID, "softmax_scale=%.8g must be 1/sqrt(D)=%.8g", (double)softmax_scale,
+                expected);
+  T3D_CHECK(check_ptr(q, "q"));
+  T3D_CHECK(check_ptr(k, "k"));
+  T3D_CHECK(check_ptr(v, "v"));
+  T3D_CHECK(check_ptr(o, "o"));
+  T3D_CHECK(check_ptr4(kv_idx, "kv_idx"));
+  T3D_CHECK(check_ptr4(kv_cnt, "kv_cnt"));
+  if (kmax < 1 || kmax > geo.nT)
+    return fail(T3D_ERR_INVALID, "kmax=%d must lie in [1, nT=%d]", kmax, geo.nT);
+  if ((keep == nullptr) != (src_row == nullptr))
+    return fail(T3D_ERR_INVALID, "keep and src_row must both be given or both be NULL");
+  if (keep != nullptr && geo.L != geo.Lp)
+    return fail(T3D_ERR_INVALID, "pruned-query attention needs every tile full (L=%d, Lp=%d)",
+                geo.L, geo.Lp);
+  const size_t need = t3d::attn_workspace_bytes(geo, kmax);
+  if (need > t3d::kNoAllocScratchBytes)
+    return fail(T3D_ERR_UNSUPPORTED,
+                "this problem needs %zu bytes of scratch, more than the library's fixed %zu bytes",
+                need, t3d::kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  cudaError_t e = t3d::noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return cuda_status(e, "block_sparse_attn_fwd_noalloc: scratch address");
+  t3d::AttnArgs a{q, k, v, o, kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale,
+                  scratch, t3d::kNoAllocScratchBytes, dev_status, g_wait_cycles};
+  return cuda_status(t3d::launch_attn(geo, a, as_stream(stream)), "block_sparse_attn_fwd_noalloc");
+}
+
 }  // extern "C"

@@ -50,4 +50,9 @@ size_t attn_workspace_bytes(const Geo& g, int kmax);
 // tcgen05/TMEM/TMA kernel (attn_sm100.cu), D = 64 or 128.
 cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s);
 
+// Size of the library's own attention scratch (attn_noalloc.cu) and its device address on the
+// current device (looked up on the first call per device).
+constexpr size_t kNoAllocScratchBytes = 256;
+cudaError_t noalloc_scratch(void** ptr);
+
 }  // namespace t3d

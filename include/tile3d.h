@@ -228,6 +228,31 @@ t3d_status block_sparse_attn_fwd(const t3d_geom* g, const void* q, const void* k
 /* Bytes of device workspace block_sparse_attn_fwd needs for this geometry and list capacity. */
 size_t block_sparse_attn_workspace_size(const t3d_geom* g, int kmax);
 
+/*
+ * block_sparse_attn_fwd_noalloc — block_sparse_attn_fwd for callers that cannot allocate device
+ * memory. The paper has no counterpart: this is a library service, not a step of the method.
+ * Some callers own no allocator of their own: a plugin inside a host framework whose allocator
+ * manages all device memory, a runtime that fixes its memory budget at start-up and forbids later
+ * allocations, or a latency-bound loop that cannot afford cudaMalloc's implicit synchronisation.
+ * Such a caller cannot provide the workspace, so this call takes none: the kernel's scratch (the
+ * counter of its work queue) lives in a fixed 256-byte array inside the library, which every GPU
+ * that loads the library holds until the process exits. The call allocates and frees nothing.
+ *   Arguments, results and errors: as block_sparse_attn_fwd without `workspace` / `ws_bytes`. A
+ *   problem whose scratch would exceed the fixed 256 bytes is rejected with T3D_ERR_UNSUPPORTED
+ *   (the kernel's scratch does not depend on the problem size today, so none is).
+ *   The first call on a device looks up the array's device address on that device (with it
+ *   current) and caches it; make that first call before any stream capture.
+ *   Every call on a device shares the one array (the call zeroes the counter on `stream` before
+ *   its launch): calls that may overlap on the GPU race and give undefined results, so calls on
+ *   one device must be ordered (one stream, or events between streams).
+ */
+t3d_status block_sparse_attn_fwd_noalloc(const t3d_geom* g, const void* q, const void* k,
+                                         const void* v, void* o, const int32_t* kv_idx,
+                                         const int32_t* kv_cnt, int kmax, const uint8_t* keep,
+                                         const uint8_t* src_row, float softmax_scale, int causal,
+                                         int num_kv_heads, int32_t* dev_status,
+                                         t3d_stream stream);
+
 #ifdef __cplusplus
 }
 #endif
