@@ -12,7 +12,7 @@ _API = (
     "Geom", "Tile3dError", "TileSparseAttention", "block_mask_to_index", "block_sparse_attn_fwd",
     "block_sparse_attn_workspace_size", "geometry", "tile3d_gather", "tile3d_scatter",
     "tile3d_scatter_pool", "tile_pool", "tile_prune_queries", "tile_prune_queries_ratio",
-    "tile_select_mass", "tile_select_topk",
+    "tile_select_mass", "tile_select_topk", "tile_select_workspace_size",
 )
 __all__ = list(_API)
 

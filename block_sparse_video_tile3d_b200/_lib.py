@@ -40,8 +40,9 @@ SIGNATURES = {
     "tile3d_gather": (_I, [_G, _P, _P, _P]),
     "tile_pool": (_I, [_G, _P, _P, _P]),
     "tile3d_scatter_pool": (_I, [_G, _P, _P, _P, _P]),
-    "tile_select_topk": (_I, [_G, _P, _P, _I, _P, _P, _P, _P]),
-    "tile_select_mass": (_I, [_G, _P, _P, _F, _F, _I, _I, _P, _P, _P, _P]),
+    "tile_select_topk": (_I, [_G, _P, _P, _I, _P, _P, _P, _S, _P, _P]),
+    "tile_select_mass": (_I, [_G, _P, _P, _F, _F, _I, _I, _P, _P, _P, _S, _P, _P]),
+    "tile_select_workspace_size": (_S, [_G]),
     "tile_prune_queries": (_I, [_G, _P, _F, _P, _P, _P, _P]),
     "tile_prune_queries_ratio": (_I, [_G, _P, _F, _P, _P, _P, _P]),
     "block_mask_to_index": (_I, [_G, _P, _I, _P, _P, _P, _P]),

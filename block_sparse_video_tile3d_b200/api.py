@@ -18,7 +18,8 @@ from ._lib import Geom, Tile3dError, check, lib
 __all__ = [
     "Geom", "Tile3dError", "geometry", "tile3d_scatter", "tile3d_gather", "tile_pool",
     "tile3d_scatter_pool",
-    "tile_select_topk", "tile_select_mass", "tile_prune_queries", "tile_prune_queries_ratio",
+    "tile_select_topk", "tile_select_mass", "tile_select_workspace_size", "tile_prune_queries",
+    "tile_prune_queries_ratio",
     "block_mask_to_index",
     "block_sparse_attn_fwd", "block_sparse_attn_workspace_size", "TileSparseAttention",
 ]
@@ -132,7 +133,21 @@ def _sel_out(B, nh, nT, kcap, device, kv_idx, kv_cnt):
     return kv_idx, kv_cnt
 
 
-def tile_select_topk(pq, pk, T, H, W, k, kv_idx=None, kv_cnt=None, dev_status=None):
+def tile_select_workspace_size(B, T, H, W, heads, D) -> int:
+    """Bytes of device workspace the selection calls need (the fp32 score rows)."""
+    g = _geom(B, T, H, W, heads, D)
+    return int(lib.tile_select_workspace_size(ctypes.byref(g)))
+
+
+def _sel_workspace(g, device, workspace):
+    need = int(lib.tile_select_workspace_size(ctypes.byref(g)))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def tile_select_topk(pq, pk, T, H, W, k, kv_idx=None, kv_cnt=None, dev_status=None,
+                     workspace=None):
     """Top-k key tiles per query tile from pooled ``[B, heads, nT, D]`` fp32 Q and K.
     Returns ``(kv_idx [B, heads, nT, min(k, nT)], kv_cnt [B, heads, nT])`` int32, ascending."""
     B, nh, nT, D = pq.shape
@@ -141,13 +156,14 @@ def tile_select_topk(pq, pk, T, H, W, k, kv_idx=None, kv_cnt=None, dev_status=No
     kcap = min(int(k), nT)
     kv_idx, kv_cnt = _sel_out(B, nh, nT, kcap, pq.device, kv_idx, kv_cnt)
     g = _geom(B, T, H, W, nh, D)
+    ws, ws_bytes = _sel_workspace(g, pq.device, workspace)
     check(lib.tile_select_topk(ctypes.byref(g), _ptr(pq), _ptr(pk), int(k), _ptr(kv_idx),
-                               _ptr(kv_cnt), _ptr(dev_status), _stream()))
+                               _ptr(kv_cnt), _ptr(ws), ws_bytes, _ptr(dev_status), _stream()))
     return kv_idx, kv_cnt
 
 
 def tile_select_mass(pq, pk, T, H, W, scale, mass, min_k=1, kmax=None, kv_idx=None, kv_cnt=None,
-                     dev_status=None):
+                     dev_status=None, workspace=None):
     """Key tiles by cumulative softmax mass per query tile. Returns ``(kv_idx, kv_cnt)``."""
     B, nh, nT, D = pq.shape
     _need(pq, "pq", torch.float32)
@@ -155,9 +171,10 @@ def tile_select_mass(pq, pk, T, H, W, scale, mass, min_k=1, kmax=None, kv_idx=No
     kmax = nT if kmax is None else int(kmax)
     kv_idx, kv_cnt = _sel_out(B, nh, nT, kmax, pq.device, kv_idx, kv_cnt)
     g = _geom(B, T, H, W, nh, D)
+    ws, ws_bytes = _sel_workspace(g, pq.device, workspace)
     check(lib.tile_select_mass(ctypes.byref(g), _ptr(pq), _ptr(pk), float(scale), float(mass),
-                               int(min_k), kmax, _ptr(kv_idx), _ptr(kv_cnt), _ptr(dev_status),
-                               _stream()))
+                               int(min_k), kmax, _ptr(kv_idx), _ptr(kv_cnt), _ptr(ws), ws_bytes,
+                               _ptr(dev_status), _stream()))
     return kv_idx, kv_cnt
 
 
@@ -303,6 +320,10 @@ class TileSparseAttention:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         ws = block_sparse_attn_workspace_size(B, T, H, W, heads, D, self.kmax)
         self.workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+        self.sel_workspace = None
+        if mode != "mask":
+            ws = tile_select_workspace_size(B, T, H, W, heads, D)
+            self.sel_workspace = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
 
     def stages(self, q, k, v, out=None):
         """The hot path as an ordered list of ``(name, launch)`` pairs; each ``launch()`` enqueues
@@ -340,11 +361,12 @@ class TileSparseAttention:
                     self.qt, T, H, W, self.cos_thresh, self.keep, self.src_row, self.pq)))
             if self.mode == "topk":
                 st.append(("select_topk", lambda: tile_select_topk(
-                    self.pq, self.pk, T, H, W, self.topk, self.kv_idx, self.kv_cnt, self.status)))
+                    self.pq, self.pk, T, H, W, self.topk, self.kv_idx, self.kv_cnt, self.status,
+                    self.sel_workspace)))
             else:
                 st.append(("select_mass", lambda: tile_select_mass(
                     self.pq, self.pk, T, H, W, self.scale, self.mass, self.min_k, self.kmax,
-                    self.kv_idx, self.kv_cnt, self.status)))
+                    self.kv_idx, self.kv_cnt, self.status, self.sel_workspace)))
         st.append(("attention", lambda: block_sparse_attn_fwd(
             self.qt, self.kt, self.vt, self.kv_idx, self.kv_cnt, T, H, W, keep=self.keep,
             src_row=self.src_row, softmax_scale=self.scale, out=self.ot,

@@ -133,9 +133,24 @@ t3d_status tile3d_scatter_pool(const t3d_geom* g, const void* x, void* y, float*
                      "tile3d_scatter_pool");
 }
 
+size_t tile_select_workspace_size(const t3d_geom* g) {
+  t3d::Geo geo;
+  if (check_geom(g, &geo) != T3D_OK) return 0;
+  return t3d::select_workspace_bytes(geo);
+}
+
+static t3d_status check_select_workspace(const t3d::Geo& geo, const void* workspace,
+                                         size_t ws_bytes) {
+  const size_t need = t3d::select_workspace_bytes(geo);
+  if (ws_bytes < need)
+    return fail(T3D_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
+                ws_bytes, need);
+  return check_ptr(workspace, "workspace");
+}
+
 t3d_status tile_select_topk(const t3d_geom* g, const float* pq, const float* pk, int k,
-                            int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
-                            t3d_stream stream) {
+                            int32_t* kv_idx, int32_t* kv_cnt, void* workspace, size_t ws_bytes,
+                            int32_t* dev_status, t3d_stream stream) {
   t3d::Geo geo;
   T3D_CHECK(check_geom(g, &geo));
   T3D_CHECK(check_ptr(pq, "pq"));
@@ -143,14 +158,16 @@ t3d_status tile_select_topk(const t3d_geom* g, const float* pq, const float* pk,
   T3D_CHECK(check_ptr4(kv_idx, "kv_idx"));
   T3D_CHECK(check_ptr4(kv_cnt, "kv_cnt"));
   if (k < 1) return fail(T3D_ERR_INVALID, "k=%d must be >= 1", k);
-  return cuda_status(
-      t3d::launch_select_topk(geo, pq, pk, k, kv_idx, kv_cnt, dev_status, as_stream(stream)),
-      "tile_select_topk");
+  T3D_CHECK(check_select_workspace(geo, workspace, ws_bytes));
+  return cuda_status(t3d::launch_select_topk(geo, pq, pk, k, kv_idx, kv_cnt, workspace, dev_status,
+                                             as_stream(stream)),
+                     "tile_select_topk");
 }
 
 t3d_status tile_select_mass(const t3d_geom* g, const float* pq, const float* pk, float scale,
                             float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
-                            int32_t* dev_status, t3d_stream stream) {
+                            void* workspace, size_t ws_bytes, int32_t* dev_status,
+                            t3d_stream stream) {
   t3d::Geo geo;
   T3D_CHECK(check_geom(g, &geo));
   T3D_CHECK(check_ptr(pq, "pq"));
@@ -164,8 +181,9 @@ t3d_status tile_select_mass(const t3d_geom* g, const float* pq, const float* pk,
   if (min_k < 1) return fail(T3D_ERR_INVALID, "min_k=%d must be >= 1", min_k);
   if (kmax < 1 || kmax > geo.nT)
     return fail(T3D_ERR_INVALID, "kmax=%d must lie in [1, nT=%d]", kmax, geo.nT);
+  T3D_CHECK(check_select_workspace(geo, workspace, ws_bytes));
   return cuda_status(t3d::launch_select_mass(geo, pq, pk, scale, mass, min_k, kmax, kv_idx, kv_cnt,
-                                             dev_status, as_stream(stream)),
+                                             workspace, dev_status, as_stream(stream)),
                      "tile_select_mass");
 }
 

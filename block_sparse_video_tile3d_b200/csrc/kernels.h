@@ -2,6 +2,7 @@
 // api.cu before any of these is called; each returns the CUDA launch error.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -16,16 +17,24 @@ cudaError_t launch_pool(const Geo& g, const void* y, float* pooled, cudaStream_t
 cudaError_t launch_scatter_pool(const Geo& g, const void* x, void* y, float* pooled,
                                 cudaStream_t s);
 
+// Selection: tensor-core score product into `workspace` (select_workspace_bytes), then one warp
+// per query tile.
+size_t select_workspace_bytes(const Geo& g);
 cudaError_t launch_select_topk(const Geo& g, const float* pq, const float* pk, int k,
-                               int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
-                               cudaStream_t s);
+                               int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
+                               int32_t* dev_status, cudaStream_t s);
 cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, float scale,
                                float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
-                               int32_t* dev_status, cudaStream_t s);
+                               void* workspace, int32_t* dev_status, cudaStream_t s);
 cudaError_t launch_mask_to_index(const Geo& g, const uint8_t* mask, int kmax, int32_t* kv_idx,
                                  int32_t* kv_cnt, int32_t* dev_status, cudaStream_t s);
 cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, int keep_size, uint8_t* keep,
                          uint8_t* src_row, float* pq_kept, cudaStream_t s);
+
+// Tensor map over a bf16 tensor of `rank` (2 or 3) dimensions, innermost first, strides in bytes
+// of every dimension but the innermost; 128-byte swizzle, out-of-range elements read as zero.
+bool encode_bf16_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                     const cuuint64_t* strides, const cuuint32_t* box);
 
 struct AttnArgs {
   const void* q;

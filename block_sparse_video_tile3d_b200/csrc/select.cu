@@ -4,129 +4,25 @@
 // K transposed, top-k per row, block map and LUT forms); bsa_attn page, BSAAttentionImpl.forward
 // (query pruning per block, KV blocks by cumulative threshold with a floor).
 //
-// Selection is exact on the fp32 scores: the k-th largest value of a row is found by a radix
-// select (four 8-bit passes) over an order-preserving uint32 image of the floats (no sort), ties at
-// the boundary go to the lower index, and kept indices are emitted in ascending order with warp
-// ballots.
+// Selection runs in two kernels. The score product S = pq . pk^T of every head runs on the tcgen05
+// tensor cores (scores_tc_kernel) and lands in fp32 in the caller's workspace; then one warp per
+// query tile selects its key tiles from its score row (topk_rows_kernel, mass_rows_kernel), so the
+// selection, which costs far more instructions than the product, spreads over every SM.
+//
+// Selection is exact on the fp32 scores: the k-th largest value of a row is found by a bit-by-bit
+// search over an order-preserving uint32 image of the floats held in registers (a radix select over
+// shared-memory histograms for rows too long for registers), with no sort; ties at the boundary go
+// to the lower index, and kept indices are emitted in ascending order with warp ballots.
+#include <math.h>
+
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace t3d {
 namespace {
 
-constexpr int kSelThreads = 256;  // 8 warps
-constexpr int kKeyChunk = 128;    // pooled key rows staged in shared memory at a time (one per thread pair)
-constexpr int kPad = 4;           // key row padding (floats): consecutive rows 4 banks apart
-constexpr int kRegSelectMax = 512;  // rows up to this many tiles are selected in registers
-
-// Shared memory of a selection CTA with R query tiles (floats): query rows, a key chunk, the score
-// rows and, when the selection uses them, the per-warp radix histograms (the mass selection always;
-// top-k for rows of more than kRegSelectMax tiles).
-inline size_t sel_smem_floats(int D, int nT, int R, bool hist) {
-  return (size_t)R * D + (size_t)kKeyChunk * (D + kPad) + (size_t)R * nT + (hist ? 8 * 256 : 0);
-}
-// Query tiles per CTA of the cumulative-mass selection: 16 (two CTAs per SM for the common sizes),
-// or 8 when 16 score rows would not fit next to the staged operands (~200 KB of shared memory).
-inline int sel_rows(int D, int nT) {
-  return sel_smem_floats(D, nT, 16, true) * 4 <= 200 * 1024 ? 16 : 8;
-}
-// Query tiles per CTA of the top-k selection: the count (8 .. 24) with the fewest waves over the
-// machine, each wave weighted by its rows plus a fixed cost of streaming the head's pooled keys
-// (worth about 8 rows).
-int topk_rows(const Geo& g, int sms) {
-  constexpr size_t kSmPerSm = 233472, kSmPerCta = 232448, kReserve = 1024;
-  int best = 8;
-  long best_cost = -1;
-  for (int R = 8; R <= 24; R += 4) {
-    const size_t bytes = sel_smem_floats(g.D, g.nT, R, g.nT > kRegSelectMax) * sizeof(float);
-    if (bytes > kSmPerCta) continue;
-    long per_sm = (long)(kSmPerSm / (bytes + kReserve));
-    if (per_sm > 2048 / kSelThreads) per_sm = 2048 / kSelThreads;
-    if (per_sm < 1) continue;
-    const long blocks = (long)g.B * g.heads * ((g.nT + R - 1) / R);
-    const long waves = (blocks + per_sm * sms - 1) / (per_sm * sms);
-    const long cost = waves * (R + 8);
-    if (best_cost < 0 || cost < best_cost) {
-      best = R;
-      best_cost = cost;
-    }
-  }
-  return best;
-}
-
-// Scores S[i, j] = pq_i . pk_j in fp32 (fused multiply-adds over d in order) for the CTA's R query
-// tiles i0 .. i0 + R - 1; row r lands in vals[r * nT + j]. Shared memory (floats): pq rows [R][D],
-// a key chunk [128][D + 4], the score rows [R][nT], then the per-warp histograms of the radix
-// select. Thread t owns key j0 + (t mod 128) of each chunk and the R / 2 rows of half t / 128: its
-// key row is one conflict-free 16-byte load per four d, the query rows are warp-wide broadcasts.
-template <int RH>
-__device__ void compute_scores(const Geo& g, const float* __restrict__ pq,
-                               const float* __restrict__ pk, long bh, int i0, float* sm) {
-  constexpr int R = 2 * RH;
-  const int D = g.D, nT = g.nT, ldk = D + kPad, d4 = D / 4;
-  float* pq_s = sm;
-  float* pk_s = pq_s + R * D;
-  float* vals = pk_s + kKeyChunk * ldk;
-  const int tid = threadIdx.x;
-  for (int e = tid; e < R * d4; e += kSelThreads) {
-    const int r = e / d4, c = e - r * d4;
-    const int i = i0 + r;
-    const float4 v = (i < nT) ? reinterpret_cast<const float4*>(pq + (bh * nT + i) * D)[c]
-                              : make_float4(0.f, 0.f, 0.f, 0.f);
-    *reinterpret_cast<float4*>(pq_s + r * D + 4 * c) = v;
-  }
-  const float* pkh = pk + bh * nT * D;
-  const int kc = tid & (kKeyChunk - 1), rh = tid / kKeyChunk;
-  const float* qrow = pq_s + rh * RH * D;
-  for (int j0 = 0; j0 < nT; j0 += kKeyChunk) {
-    __syncthreads();
-    const int rows = imin(kKeyChunk, nT - j0);
-    for (int e = tid; e < kKeyChunk * d4; e += kSelThreads) {
-      const int r = e / d4, c = e - r * d4;
-      const float4 v = (r < rows) ? reinterpret_cast<const float4*>(pkh + (long)(j0 + r) * D)[c]
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-      *reinterpret_cast<float4*>(pk_s + r * ldk + 4 * c) = v;
-    }
-    __syncthreads();
-    float acc[RH];
-#pragma unroll
-    for (int a = 0; a < RH; ++a) acc[a] = 0.f;
-    const float* krow = pk_s + kc * ldk;
-    for (int d = 0; d < D; d += 4) {
-      const float4 kb = *reinterpret_cast<const float4*>(krow + d);
-#pragma unroll
-      for (int a = 0; a < RH; ++a) {
-        const float4 qa = *reinterpret_cast<const float4*>(qrow + a * D + d);
-        acc[a] = fmaf(qa.x, kb.x, acc[a]);
-        acc[a] = fmaf(qa.y, kb.y, acc[a]);
-        acc[a] = fmaf(qa.z, kb.z, acc[a]);
-        acc[a] = fmaf(qa.w, kb.w, acc[a]);
-      }
-    }
-    if (kc < rows) {
-#pragma unroll
-      for (int a = 0; a < RH; ++a) vals[(rh * RH + a) * nT + j0 + kc] = acc[a];
-    }
-  }
-  __syncthreads();
-}
-
-// R = 8 or 16 (the cumulative-mass selection).
-__device__ void compute_scores_8_16(const Geo& g, const float* pq, const float* pk, long bh, int i0,
-                                    int R, float* sm) {
-  if (R == 16) compute_scores<8>(g, pq, pk, bh, i0, sm);
-  else compute_scores<4>(g, pq, pk, bh, i0, sm);
-}
-// R = 8, 12, 16, 20 or 24 (the top-k selection).
-__device__ void compute_scores_any(const Geo& g, const float* pq, const float* pk, long bh, int i0,
-                                   int R, float* sm) {
-  switch (R) {
-    case 24: compute_scores<12>(g, pq, pk, bh, i0, sm); break;
-    case 20: compute_scores<10>(g, pq, pk, bh, i0, sm); break;
-    case 16: compute_scores<8>(g, pq, pk, bh, i0, sm); break;
-    case 12: compute_scores<6>(g, pq, pk, bh, i0, sm); break;
-    default: compute_scores<4>(g, pq, pk, bh, i0, sm); break;
-  }
-}
+constexpr int kSelThreads = 256;     // 8 warps: one score row each at a time
+constexpr int kRegSelectMax = 1536;  // rows up to this many tiles are selected in registers
 
 // Top-k of a row of at most 32 * KPL values held in registers (lane l owns entries l + 32 i):
 // the k-th largest order-preserving key is found bit by bit from the top (largest T with at least k
@@ -276,34 +172,17 @@ __device__ int select_topk_row(const float* row, int n, int k, int32_t* out, int
   return k;
 }
 
-__global__ void __launch_bounds__(kSelThreads) topk_kernel(Geo g, const float* __restrict__ pq,
-                                                           const float* __restrict__ pk, int k,
-                                                           int R, int32_t* __restrict__ kv_idx,
-                                                           int32_t* __restrict__ kv_cnt) {
-  extern __shared__ float4 sm4[];
-  float* sm = reinterpret_cast<float*>(sm4);
-  const int nT = g.nT;
-  const int blocks_per_head = (nT + R - 1) / R;
-  const long bh = blockIdx.x / blocks_per_head;
-  const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * R;
-  compute_scores_any(g, pq, pk, bh, i0, R, sm);
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float* vals = sm + R * g.D + kKeyChunk * (g.D + kPad);
-  int* hist = reinterpret_cast<int*>(const_cast<float*>(vals) + R * nT) + w * 256;
-  const int kk = imin(k, nT);
-  for (int r = w; r < R; r += kSelThreads / 32) {
-    const int i = i0 + r;
-    if (i >= nT) break;
-    const float* row = vals + r * nT;
-    int32_t* out = kv_idx + (bh * nT + i) * kk;
-    int n;
-    if (nT <= 128) n = select_topk_row_reg<4>(row, nT, kk, out);
-    else if (nT <= 256) n = select_topk_row_reg<8>(row, nT, kk, out);
-    else if (nT <= kRegSelectMax) n = select_topk_row_reg<16>(row, nT, kk, out);
-    else n = select_topk_row(row, nT, kk, out, hist);
-    if (lane == 0) kv_cnt[bh * nT + i] = n;
-  }
+// Top-k of row[0..n) with the register search when the row fits (n <= kRegSelectMax), else the
+// radix select over the per-warp histogram `hist` (256 ints).
+__device__ int select_topk_any(const float* row, int n, int k, int32_t* out, int* hist) {
+  if (n <= 128) return select_topk_row_reg<4>(row, n, k, out);
+  if (n <= 256) return select_topk_row_reg<8>(row, n, k, out);
+  if (n <= 512) return select_topk_row_reg<16>(row, n, k, out);
+  if (n <= 1024) return select_topk_row_reg<32>(row, n, k, out);
+  if (n <= kRegSelectMax) return select_topk_row_reg<48>(row, n, k, out);
+  return select_topk_row(row, n, k, out, hist);
 }
+
 
 // Cumulative-mass selection of one row (one warp). The scores in row[0..nT) are replaced by
 // e_j = exp(scale * (S_j - max S)); tiles are ranked by e (ties: lower index) and the smallest
@@ -321,7 +200,7 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
       return nT;
     }
     if (lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
-    return select_topk_row(row, nT, kmax, out, hist);
+    return select_topk_any(row, nT, kmax, out, hist);
   }
   float mx = -INFINITY;
   for (int j = lane; j < nT; j += 32) mx = fmaxf(mx, row[j]);
@@ -380,36 +259,337 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
   if (count < floor_k || count > kmax) {
     const int kk = count < floor_k ? floor_k : kmax;
     if (count > kmax && lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
-    count = select_topk_row(row, nT, imin(kk, kmax), out, hist);
+    count = select_topk_any(row, nT, imin(kk, kmax), out, hist);
   } else {
     emit_threshold(row, nT, prefix, need_eq, out, kmax);
   }
   return count;
 }
 
-__global__ void __launch_bounds__(kSelThreads) mass_kernel(Geo g, const float* __restrict__ pq,
-                                                           const float* __restrict__ pk,
-                                                           float scale, float mass, int min_k,
-                                                           int kmax, int R,
-                                                           int32_t* __restrict__ kv_idx,
-                                                           int32_t* __restrict__ kv_cnt,
-                                                           int32_t* dev_status) {
-  extern __shared__ float4 sm4[];
-  float* sm = reinterpret_cast<float*>(sm4);
-  const int nT = g.nT;
-  const int blocks_per_head = (nT + R - 1) / R;
-  const long bh = blockIdx.x / blocks_per_head;
-  const int i0 = (int)(blockIdx.x - bh * blocks_per_head) * R;
-  compute_scores_8_16(g, pq, pk, bh, i0, R, sm);
+// ------------------------------------------------------------ score product on the tensor cores
+//
+// S = pq . pk^T per head runs on the tcgen05 tensor cores in two kernels. split_kernel turns the
+// fp32 operands into bf16 pairs x = hi + lo (hi = bf16(x), lo = bf16(x - hi)), stored row-major in
+// the workspace; scores_tc_kernel then computes S = hi.hi + hi.lo + lo.hi for 128 query tiles
+// (MMA M = 128, one TMEM lane per query tile) against 256 key tiles (two MMAs of N = 128, TMEM
+// columns 0..255), K = D, fp32 in TMEM, with every operand fetched by TMA into 128-byte-swizzled
+// K-major tiles. The dropped lo.lo term and the rounding of lo leave a relative error of about
+// 2^-16 of sum_d |q_d k_d|, near fp32 accuracy, where a single bf16 product would err by 2^-8.
+// TMEM then goes to the score rows in the workspace, one 128-byte run of 32 key tiles per thread
+// and load.
+constexpr int kSplitThreads = 256;
+constexpr int kScThreads = 256;   // 8 warps: two per TMEM sub-partition for the read-out
+constexpr int kScRows = 128;      // query tiles per CTA (MMA M)
+constexpr int kScChunk = 128;     // key tiles per MMA (MMA N)
+constexpr int kScCols = 256;      // key tiles per CTA (two chunks; TMEM columns allocated)
+
+// Workspace of the selection calls: the score rows, then the four split operands.
+struct SelLayout {
+  size_t s_bytes, part_elems;  // score rows; elements of one split operand (B * heads * nT * D)
+  int ldS;                     // score row stride (floats): nT rounded up to 4
+};
+inline SelLayout sel_layout(const Geo& g) {
+  SelLayout l;
+  l.ldS = (g.nT + 3) & ~3;
+  l.s_bytes = (((size_t)g.B * g.heads * g.nT * l.ldS * sizeof(float)) + 255) & ~(size_t)255;
+  l.part_elems = (size_t)g.B * g.heads * g.nT * g.D;
+  return l;
+}
+
+// pq, pk -> their hi and lo bf16 parts (8 elements per thread; n8 = elements / 8 of one operand).
+__global__ void __launch_bounds__(kSplitThreads) split_kernel(const float4* __restrict__ pq,
+                                                              const float4* __restrict__ pk,
+                                                              long n8, uint4* __restrict__ qhi,
+                                                              uint4* __restrict__ qlo,
+                                                              uint4* __restrict__ khi,
+                                                              uint4* __restrict__ klo) {
+  for (long e = (long)blockIdx.x * kSplitThreads + threadIdx.x; e < 2 * n8;
+       e += (long)gridDim.x * kSplitThreads) {
+    const bool isk = e >= n8;
+    const long i = isk ? e - n8 : e;
+    const float4* src = isk ? pk : pq;
+    const float4 a = __ldg(src + 2 * i), b = __ldg(src + 2 * i + 1);
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(v[2 * t]);
+      const __nv_bfloat16 h1 = __float2bfloat16_rn(v[2 * t + 1]);
+      const __nv_bfloat162 hp = __halves2bfloat162(h0, h1);
+      const __nv_bfloat162 lp = __floats2bfloat162_rn(v[2 * t] - __bfloat162float(h0),
+                                                      v[2 * t + 1] - __bfloat162float(h1));
+      h[t] = *reinterpret_cast<const uint32_t*>(&hp);
+      l[t] = *reinterpret_cast<const uint32_t*>(&lp);
+    }
+    (isk ? khi : qhi)[i] = make_uint4(h[0], h[1], h[2], h[3]);
+    (isk ? klo : qlo)[i] = make_uint4(l[0], l[1], l[2], l[3]);
+  }
+}
+
+template <int kD>
+struct ScSmem {
+  static constexpr int kHalves = kD / 64;
+  uint8_t a[2][kHalves][kScRows * 128];                      // query block: hi, lo
+  uint8_t b[kScCols / kScChunk][2][kHalves][kScChunk * 128];  // key chunks: hi, lo
+  uint64_t full[2];  // the query block and key chunk c landed
+  uint64_t mma_done;
+  uint32_t tmem_base;
+};
+
+struct ScMaps {
+  CUtensorMap qhi, qlo, khi, klo;  // [B * heads * nT rows, D] bf16, box 128 rows x 64 elements
+};
+
+// Grid: (query blocks of 128) x (key blocks of 256) x (B * heads). S row i of head bh lands at
+// S + (bh * nT + i) * ldS. Rows of a box past the head's last tile read the next head's (or zero
+// past the tensor); their scores are never stored.
+template <int kD>
+__global__ void __launch_bounds__(kScThreads, 1)
+    scores_tc_kernel(const __grid_constant__ ScMaps maps, Geo g, float* __restrict__ S, int ldS) {
+  using namespace sm100;
+  constexpr int kHalves = kD / 64;
+  extern __shared__ uint8_t smem_raw[];
+  ScSmem<kD>& sm = *reinterpret_cast<ScSmem<kD>*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  constexpr uint32_t idesc = idesc_bf16(kScRows, kScChunk, false, false);
+  constexpr uint32_t kBox = kScRows * 128;  // bytes of one 128-row x 64-element box
+  const int nT = g.nT, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int i0 = blockIdx.x * kScRows, j0 = blockIdx.y * kScCols;
+  const long bh = blockIdx.z;
+  const int nchunks = imin(kScCols, nT - j0 + kScChunk - 1) / kScChunk;  // 1 or 2
+  if (threadIdx.x == 0) {
+    mbar_init(&sm.full[0], 1);
+    mbar_init(&sm.full[1], 1);
+    mbar_init(&sm.mma_done, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&sm.tmem_base, (uint32_t)kScCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  if (threadIdx.x == 0) {
+    const int qrow = (int)(bh * nT + i0);
+    mbar_expect_tx(&sm.full[0], 2 * kHalves * kBox * 2);  // query block + key chunk 0
+    if (nchunks > 1) mbar_expect_tx(&sm.full[1], 2 * kHalves * kBox);
+    for (int hh = 0; hh < kHalves; ++hh) {
+      tma_load_2d(sm.a[0][hh], &maps.qhi, &sm.full[0], 64 * hh, qrow);
+      tma_load_2d(sm.a[1][hh], &maps.qlo, &sm.full[0], 64 * hh, qrow);
+    }
+    for (int c = 0; c < nchunks; ++c) {
+      const int krow = (int)(bh * nT + j0 + c * kScChunk);
+      for (int hh = 0; hh < kHalves; ++hh) {
+        tma_load_2d(sm.b[c][0][hh], &maps.khi, &sm.full[c], 64 * hh, krow);
+        tma_load_2d(sm.b[c][1][hh], &maps.klo, &sm.full[c], 64 * hh, krow);
+      }
+    }
+    const uint64_t ah = sdesc_sw128(smem_u32(sm.a[0][0]), 16, 1024);
+    const uint64_t al = sdesc_sw128(smem_u32(sm.a[1][0]), 16, 1024);
+    for (int c = 0; c < nchunks; ++c) {
+      mbar_wait(&sm.full[c], 0, nullptr);
+      tc_fence_after();
+      const uint64_t bhd = sdesc_sw128(smem_u32(sm.b[c][0][0]), 16, 1024);
+      const uint64_t bld = sdesc_sw128(smem_u32(sm.b[c][1][0]), 16, 1024);
+      const uint32_t d = tmem + (uint32_t)(c * kScChunk);
+#pragma unroll
+      for (int kk = 0; kk < kD / 16; ++kk) {  // 16 elements of D per MMA
+        const int hh = kk >> 2, st = kk & 3;
+        const uint64_t o = (uint64_t)((hh * kBox + st * 32) >> 4);
+        mma_bf16(d, ah + o, bhd + o, idesc, kk ? 1u : 0u);
+        mma_bf16(d, ah + o, bld + o, idesc, 1u);
+        mma_bf16(d, al + o, bhd + o, idesc, 1u);
+      }
+    }
+    mma_commit(&sm.mma_done);
+  }
+  __syncwarp();
+  mbar_wait(&sm.mma_done, 0, nullptr);
+  tc_fence_after();
+  // TMEM -> S: warp w reads lanes 32 (w % 4) .. + 31 (query tiles i0 + 32 (w % 4) + lane) and the
+  // key tiles j0 + 128 (w / 4) .. + 127 in four loads of 32 columns.
+  {
+    const int sp = warp & 3, part = warp >> 2;
+    const int i = i0 + 32 * sp + lane;
+    float* srow = S + (bh * nT + i) * (long)ldS;
+#pragma unroll
+    for (int c32 = 0; c32 < 4; ++c32) {
+      const int col = kScChunk * part + 32 * c32;
+      if (col >= nchunks * kScChunk) break;  // warp-uniform
+      uint32_t v[32];
+      tmem_ld32(tmem + ((uint32_t)(32 * sp) << 16) + (uint32_t)col, v);
+      tmem_wait_ld();
+      const int j = j0 + col;
+      if (i < nT && j < nT) {
+        if (j + 32 <= nT) {
+          float4* dst = reinterpret_cast<float4*>(srow + j);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4)
+            dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                  __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (j + e < nT) srow[j + e] = __uint_as_float(v[e]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, (uint32_t)kScCols);
+  }
+}
+
+template <int kD>
+constexpr size_t sc_smem_bytes() {
+  return sizeof(ScSmem<kD>) + 1024;
+}
+
+// Top-k of a row of at most 32 * KPL values (lane l holds entries l + 32 i) by an exact threshold
+// search on the values: c(t) = #{x >= t} is driven to k, and when c(t) == k the set {x >= t} is
+// exactly the k largest values (no tie can straddle t). The first guess is the row's mean plus z
+// standard deviations, z the standard normal quantile of 1 - k/n (computed on the host): the
+// pooled scores are sums of many products and close to normal, so c lands near k. Then a bracket
+// lo (c > k) / hi (c < k) is narrowed by interpolating the count linearly between its ends, with
+// the Illinois rule (an end kept twice in a row has its weight halved) so one end cannot stall;
+// about 4 counting passes per row on the pooled scores. Rows where no such t exists (ties at the
+// boundary) or that do not converge in kMaxSteps go to the bit-by-bit key search, which breaks
+// ties toward the lower index.
+template <int KPL>
+__device__ int select_topk_row_fast(const float* row, int n, int k, float z, int32_t* out) {
+  constexpr int kMaxSteps = 24;
+  k = imin(k, n);
+  if (k <= 0) return 0;
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = lanemask_lt();
+  float x[KPL];
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int j = lane + 32 * i;
+    x[i] = j < n ? row[j] : -INFINITY;
+  }
+  if (k == n) {
+    for (int j = lane; j < n; j += 32) out[j] = j;
+    return n;
+  }
+  float mx = -INFINITY, mn = INFINITY, s1 = 0.f, s2 = 0.f;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    if (lane + 32 * i < n) {
+      mx = fmaxf(mx, x[i]);
+      mn = fminf(mn, x[i]);
+      s1 += x[i];
+      s2 = fmaf(x[i], x[i], s2);
+    }
+  }
+  mx = sm100::redux_max(mx);
+  mn = -sm100::redux_max(-mn);
+  s1 = warp_sum(s1);
+  s2 = warp_sum(s2);
+  auto count_ge = [&](float t) {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) c += x[i] >= t ? 1 : 0;
+    return (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+  };
+  float lo = mn, hi = mx;
+  int clo = n, chi = count_ge(mx);
+  float thr = 0.f;
+  bool found = false;
+  if (chi < k && lo < hi) {
+    const float mean = s1 / (float)n;
+    const float sd = sqrtf(fmaxf(s2 / (float)n - mean * mean, 0.f));
+    float t = fmaf(z, sd, mean);
+    float wlo = 1.f, whi = 1.f;
+    int side = 0;  // end moved at the previous step: 1 = lo, -1 = hi
+    for (int step = 0; step < kMaxSteps; ++step) {
+      if (step > 0) {
+        const float a = wlo * (float)(clo - k), b = whi * (float)(k - chi);
+        t = fmaf(hi - lo, __fdividef(a, a + b), lo);
+      }
+      if (!(t > lo && t < hi)) t = 0.5f * (lo + hi);
+      if (!(t > lo && t < hi)) break;  // the bracket is down to adjacent floats
+      const int c = count_ge(t);
+      if (c == k) {
+        thr = t;
+        found = true;
+        break;
+      }
+      if (c > k) {
+        lo = t;
+        clo = c;
+        whi = side == 1 ? 0.5f * whi : 1.f;
+        wlo = 1.f;
+        side = 1;
+      } else {
+        hi = t;
+        chi = c;
+        wlo = side == -1 ? 0.5f * wlo : 1.f;
+        whi = 1.f;
+        side = -1;
+      }
+    }
+  }
+  if (!found) return select_topk_row_reg<KPL>(row, n, k, out);
+  int written = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const bool sel = x[i] >= thr;  // pads are -inf
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    if (sel) out[written + __popc(sb & lt)] = lane + 32 * i;
+    written += __popc(sb);
+  }
+  return k;
+}
+
+// One warp per query tile: its top-k key tiles from its score row. KPL = 0: the radix select for
+// rows too long for registers.
+template <int KPL>
+__global__ void __launch_bounds__(kSelThreads) topk_rows_kernel(Geo g, const float* __restrict__ S,
+                                                                int ldS, int k, float z,
+                                                                int32_t* __restrict__ kv_idx,
+                                                                int32_t* __restrict__ kv_cnt) {
+  __shared__ int hist[KPL == 0 ? kSelThreads / 32 : 1][256];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* vals = sm + R * g.D + kKeyChunk * (g.D + kPad);
-  int* hist = reinterpret_cast<int*>(vals + R * nT) + w * 256;
-  for (int r = w; r < R; r += kSelThreads / 32) {
-    const int i = i0 + r;
-    if (i >= nT) break;
-    const int count = select_mass_row(vals + r * nT, nT, scale, mass, min_k, kmax,
-                                      kv_idx + (bh * nT + i) * kmax, dev_status, hist);
-    if (lane == 0) kv_cnt[bh * nT + i] = count;
+  const long rows = (long)g.B * g.heads * g.nT;
+  const int kk = imin(k, g.nT);
+  for (long r = (long)blockIdx.x * (kSelThreads / 32) + w; r < rows;
+       r += (long)gridDim.x * (kSelThreads / 32)) {
+    int n;
+    if constexpr (KPL == 0) n = select_topk_row(S + r * ldS, g.nT, kk, kv_idx + r * kk, hist[w]);
+    else n = select_topk_row_fast<KPL>(S + r * ldS, g.nT, kk, z, kv_idx + r * kk);
+    if (lane == 0) kv_cnt[r] = n;
+  }
+}
+
+// One warp per query tile: cumulative-mass selection from its score row, staged in the warp's
+// shared-memory row buffer (the search reads it many times).
+__global__ void __launch_bounds__(kSelThreads) mass_rows_kernel(Geo g, const float* __restrict__ S,
+                                                                int ldS, float scale, float mass,
+                                                                int min_k, int kmax,
+                                                                int32_t* __restrict__ kv_idx,
+                                                                int32_t* __restrict__ kv_cnt,
+                                                                int32_t* dev_status) {
+  extern __shared__ float rowbuf[];  // [8 warps][nT], then [8 warps][256] histogram ints
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nT = g.nT;
+  float* row = rowbuf + (long)w * nT;
+  int* hist = reinterpret_cast<int*>(rowbuf + (long)(kSelThreads / 32) * nT) + w * 256;
+  const long rows = (long)g.B * g.heads * nT;
+  for (long r = (long)blockIdx.x * (kSelThreads / 32) + w; r < rows;
+       r += (long)gridDim.x * (kSelThreads / 32)) {
+    const float* src = S + r * ldS;
+    for (int j = lane; j < nT; j += 32) row[j] = src[j];
+    __syncwarp();
+    const int count = select_mass_row(row, nT, scale, mass, min_k, kmax, kv_idx + r * kmax,
+                                      dev_status, hist);
+    if (lane == 0) kv_cnt[r] = count;
+    __syncwarp();
   }
 }
 
@@ -585,33 +765,117 @@ __global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_
 
 }  // namespace
 
-cudaError_t launch_select_topk(const Geo& g, const float* pq, const float* pk, int k,
-                               int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
-                               cudaStream_t s) {
-  (void)dev_status;
+size_t select_workspace_bytes(const Geo& g) {
+  const SelLayout l = sel_layout(g);
+  return l.s_bytes + 4 * l.part_elems * sizeof(__nv_bfloat16);
+}
+
+namespace {
+
+// z with P(N(0, 1) > z) = p, by bisection on the host's erfc (a starting guess only: accuracy
+// beyond a few digits does not matter). p = 1 gives the lower end of the search range.
+float upper_normal_quantile(double p) {
+  double lo = -8.0, hi = 8.0;
+  for (int it = 0; it < 60; ++it) {
+    const double mid = 0.5 * (lo + hi);
+    if (0.5 * erfc(mid / sqrt(2.0)) > p) lo = mid;
+    else hi = mid;
+  }
+  return (float)(0.5 * (lo + hi));
+}
+
+int sel_grid(const Geo& g) {
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int R = topk_rows(g, sms > 0 ? sms : 148);
-  const size_t smem = sel_smem_floats(g.D, g.nT, R, g.nT > kRegSelectMax) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  const long rows = (long)g.B * g.heads * g.nT;
+  long blocks = (rows + (kSelThreads / 32) - 1) / (kSelThreads / 32);
+  const long cap = (long)(sms > 0 ? sms : 148) * 8;
+  return (int)(blocks < cap ? blocks : cap);
+}
+
+template <int kD>
+cudaError_t launch_scores_d(const Geo& g, const ScMaps& maps, float* S, int ldS, cudaStream_t s) {
+  const size_t smem = sc_smem_bytes<kD>();
+  cudaError_t e = cudaFuncSetAttribute(scores_tc_kernel<kD>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const long blocks = (long)g.B * g.heads * ((g.nT + R - 1) / R);
-  topk_kernel<<<(unsigned)blocks, kSelThreads, smem, s>>>(g, pq, pk, k, R, kv_idx, kv_cnt);
+  dim3 grid((g.nT + kScRows - 1) / kScRows, (g.nT + kScCols - 1) / kScCols, g.B * g.heads);
+  scores_tc_kernel<kD><<<grid, kScThreads, smem, s>>>(maps, g, S, ldS);
+  return cudaGetLastError();
+}
+
+// Split the operands into the workspace, then the score rows into its head.
+cudaError_t launch_scores(const Geo& g, const float* pq, const float* pk, void* workspace,
+                          float** S, int* ldS, cudaStream_t s) {
+  const SelLayout l = sel_layout(g);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* part = reinterpret_cast<__nv_bfloat16*>(ws + l.s_bytes);
+  __nv_bfloat16 *qhi = part, *qlo = part + l.part_elems, *khi = part + 2 * l.part_elems,
+                *klo = part + 3 * l.part_elems;
+  const long n8 = (long)(l.part_elems / 8);
+  long blocks = (2 * n8 + kSplitThreads - 1) / kSplitThreads;
+  if (blocks > 148L * 16) blocks = 148L * 16;
+  split_kernel<<<(unsigned)blocks, kSplitThreads, 0, s>>>(
+      reinterpret_cast<const float4*>(pq), reinterpret_cast<const float4*>(pk), n8,
+      reinterpret_cast<uint4*>(qhi), reinterpret_cast<uint4*>(qlo), reinterpret_cast<uint4*>(khi),
+      reinterpret_cast<uint4*>(klo));
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  ScMaps maps;
+  const cuuint64_t dims[2] = {(cuuint64_t)g.D, (cuuint64_t)g.B * g.heads * g.nT};
+  const cuuint64_t strides[1] = {(cuuint64_t)g.D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kScRows};
+  if (!encode_bf16_map(&maps.qhi, qhi, 2, dims, strides, box) ||
+      !encode_bf16_map(&maps.qlo, qlo, 2, dims, strides, box) ||
+      !encode_bf16_map(&maps.khi, khi, 2, dims, strides, box) ||
+      !encode_bf16_map(&maps.klo, klo, 2, dims, strides, box))
+    return cudaErrorInvalidValue;
+  *S = reinterpret_cast<float*>(ws);
+  *ldS = l.ldS;
+  return g.D == 128 ? launch_scores_d<128>(g, maps, *S, l.ldS, s)
+                    : launch_scores_d<64>(g, maps, *S, l.ldS, s);
+}
+
+}  // namespace
+
+cudaError_t launch_select_topk(const Geo& g, const float* pq, const float* pk, int k,
+                               int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
+                               int32_t* dev_status, cudaStream_t s) {
+  (void)dev_status;
+  float* S = nullptr;
+  int ldS = 0;
+  cudaError_t e = launch_scores(g, pq, pk, workspace, &S, &ldS, s);
+  if (e != cudaSuccess) return e;
+  const int grid = sel_grid(g);
+  const float z = upper_normal_quantile((double)imin(k, g.nT) / g.nT);
+  if (g.nT <= 128)
+    topk_rows_kernel<4><<<grid, kSelThreads, 0, s>>>(g, S, ldS, k, z, kv_idx, kv_cnt);
+  else if (g.nT <= 256)
+    topk_rows_kernel<8><<<grid, kSelThreads, 0, s>>>(g, S, ldS, k, z, kv_idx, kv_cnt);
+  else if (g.nT <= 512)
+    topk_rows_kernel<16><<<grid, kSelThreads, 0, s>>>(g, S, ldS, k, z, kv_idx, kv_cnt);
+  else if (g.nT <= 1024)
+    topk_rows_kernel<32><<<grid, kSelThreads, 0, s>>>(g, S, ldS, k, z, kv_idx, kv_cnt);
+  else if (g.nT <= kRegSelectMax)
+    topk_rows_kernel<48><<<grid, kSelThreads, 0, s>>>(g, S, ldS, k, z, kv_idx, kv_cnt);
+  else
+    topk_rows_kernel<0><<<grid, kSelThreads, 0, s>>>(g, S, ldS, k, z, kv_idx, kv_cnt);
   return cudaGetLastError();
 }
 
 cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, float scale,
                                float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
-                               int32_t* dev_status, cudaStream_t s) {
-  const int R = sel_rows(g.D, g.nT);
-  const size_t smem = sel_smem_floats(g.D, g.nT, R, true) * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(mass_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+                               void* workspace, int32_t* dev_status, cudaStream_t s) {
+  float* S = nullptr;
+  int ldS = 0;
+  cudaError_t e = launch_scores(g, pq, pk, workspace, &S, &ldS, s);
   if (e != cudaSuccess) return e;
-  const long blocks = (long)g.B * g.heads * ((g.nT + R - 1) / R);
-  mass_kernel<<<(unsigned)blocks, kSelThreads, smem, s>>>(g, pq, pk, scale, mass, min_k, kmax, R,
+  const size_t smem = (size_t)(kSelThreads / 32) * ((size_t)g.nT * sizeof(float) + 256 * sizeof(int));
+  e = cudaFuncSetAttribute(mass_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+  if (e != cudaSuccess) return e;
+  mass_rows_kernel<<<sel_grid(g), kSelThreads, smem, s>>>(g, S, ldS, scale, mass, min_k, kmax,
                                                           kv_idx, kv_cnt, dev_status);
   return cudaGetLastError();
 }

@@ -147,23 +147,27 @@ __global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_kernel(Geo g,
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   if (c < g.row_chunks) {
+    // All four of this thread's rows are loaded before any is used, so the four loads are in
+    // flight together; pad slots read as zero and add nothing to the sums.
+    constexpr int kPer = kTileElems / kPoolRows;
     const long dst0 = ((long)b * g.Lp + (long)i * kTileElems) * g.row_chunks + c;
     const long src_b = (long)b * g.L;
-#pragma unroll 4
-    for (int r = ry; r < kTileElems; r += kPoolRows) {
-      const int sr = src_row[r];
-      uint4 u = make_uint4(0u, 0u, 0u, 0u);
-      if (sr >= 0) {
-        u = ld_nc(x + (src_b + sr) * g.row_chunks + c);
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+    uint4 u[kPer];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(h2[e]);
-          acc[2 * e] += f.x;
-          acc[2 * e + 1] += f.y;
-        }
+    for (int t = 0; t < kPer; ++t) {
+      const int sr = src_row[ry + kPoolRows * t];
+      u[t] = sr >= 0 ? ld_nc(x + (src_b + sr) * g.row_chunks + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[t]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
       }
-      y[dst0 + (long)r * g.row_chunks] = u;
+      y[dst0 + (long)(ry + kPoolRows * t) * g.row_chunks] = u[t];
     }
   }
 #pragma unroll

@@ -123,15 +123,19 @@ t3d_status tile3d_scatter_pool(const t3d_geom* g, const void* x, void* y, float*
  * FastVideo API docs, fastvideo.attention.backends page, sla.get_block_map:
  * S = pooled_q @ pooled_k^T (no softmax scale), top-k per row, recorded as an index list (LUT).
  * Ties at the k-th score go to the lower key-tile index; indices are written in ascending order.
- * Scores are fp32 dot products over D.
+ * Scores are computed on the tensor cores from fp32 operands split into bf16 pairs
+ * (hi.hi + hi.lo + lo.hi, fp32 accumulation): within about 2^-16 of sum_d |pq_d pk_d| of the exact
+ * dot product, so kept sets are exact wherever the k-th and (k+1)-th scores are further apart.
  *   pq, pk: in,  fp32 [B, heads, nT, D].
  *   k:      1 <= k; k > nT is clamped to nT (every tile kept).
  *   kv_idx: out, int32 [B, heads, nT, min(k, nT)].  kv_cnt: out, int32 [B, heads, nT].
+ *   workspace: device scratch of at least tile_select_workspace_size() bytes (the fp32 score
+ *           rows, B * heads * nT * ceil4(nT) floats); contents on entry do not matter.
  *   dev_status: in/out device int32, or NULL.
  */
 t3d_status tile_select_topk(const t3d_geom* g, const float* pq, const float* pk, int k,
-                            int32_t* kv_idx, int32_t* kv_cnt, int32_t* dev_status,
-                            t3d_stream stream);
+                            int32_t* kv_idx, int32_t* kv_cnt, void* workspace, size_t ws_bytes,
+                            int32_t* dev_status, t3d_stream stream);
 
 /*
  * tile_select_mass — keep key tiles by cumulative softmax mass per query tile.
@@ -144,10 +148,15 @@ t3d_status tile_select_topk(const t3d_geom* g, const float* pq, const float* pk,
  *   kmax:   capacity of each row of kv_idx (1 <= kmax <= nT); longer sets are truncated to their
  *           kmax highest-probability tiles and T3D_DEV_OVERFLOW is set.
  *   kv_idx: out, int32 [B, heads, nT, kmax].  kv_cnt: out, int32 [B, heads, nT].
+ *   workspace: as tile_select_topk. Scores as tile_select_topk. mass = 1 keeps every tile.
  */
 t3d_status tile_select_mass(const t3d_geom* g, const float* pq, const float* pk, float scale,
                             float mass, int min_k, int kmax, int32_t* kv_idx, int32_t* kv_cnt,
-                            int32_t* dev_status, t3d_stream stream);
+                            void* workspace, size_t ws_bytes, int32_t* dev_status,
+                            t3d_stream stream);
+
+/* Bytes of device workspace tile_select_topk / tile_select_mass need for this geometry. */
+size_t tile_select_workspace_size(const t3d_geom* g);
 
 /*
  * tile_prune_queries — BSA query pruning per 64-token block.

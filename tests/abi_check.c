@@ -34,7 +34,7 @@ int main(int argc, char** argv) {
   free(vc);
   /* Validation failures, all caught on the host before anything touches a device. */
   printf("scatter_null %d\n", (int)tile3d_scatter(&g, NULL, NULL, NULL));
-  printf("topk_k0 %d\n", (int)tile_select_topk(&g, NULL, NULL, 0, NULL, NULL, NULL, NULL));
+  printf("topk_k0 %d\n", (int)tile_select_topk(&g, NULL, NULL, 0, NULL, NULL, NULL, 0, NULL, NULL));
   printf("ws_null_geom %zu\n", block_sparse_attn_workspace_size(NULL, 4));
   return 0;
 }

@@ -103,15 +103,26 @@ def test_other_calls_reject_bad_arguments():
     assert lib.tile3d_scatter(g, ODD, FAKE, None) == _lib.T3D_ERR_INVALID
     assert lib.tile3d_gather(g, FAKE, None, None) == _lib.T3D_ERR_INVALID
     assert lib.tile_pool(None, FAKE, FAKE, None) == _lib.T3D_ERR_INVALID
-    assert lib.tile_select_topk(g, FAKE, FAKE, 0, FAKE, FAKE, None, None) == _lib.T3D_ERR_INVALID
-    assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 1.5, 1, 4, FAKE, FAKE, None, None) == \
+    ws = lib.tile_select_workspace_size(g)
+    # fp32 score rows (B * heads * nT * ceil4(nT) floats = 128 bytes, rounded up to 256) and the
+    # bf16 hi and lo parts of pq and pk (4 * B * heads * nT * D * 2 bytes)
+    assert ws == 256 + 4 * (1 * 2 * 4 * 64) * 2
+    assert lib.tile_select_topk(g, FAKE, FAKE, 0, FAKE, FAKE, FAKE, ws, None, None) == \
         _lib.T3D_ERR_INVALID
-    assert lib.tile_select_mass(g, FAKE, FAKE, -1.0, 0.9, 1, 4, FAKE, FAKE, None, None) == \
-        _lib.T3D_ERR_INVALID
-    assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 0.9, 0, 4, FAKE, FAKE, None, None) == \
-        _lib.T3D_ERR_INVALID
-    assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 0.9, 1, 9, FAKE, FAKE, None, None) == \
-        _lib.T3D_ERR_INVALID
+    assert lib.tile_select_topk(g, FAKE, FAKE, 2, FAKE, FAKE, FAKE, ws - 1, None, None) == \
+        _lib.T3D_ERR_INVALID  # workspace too small
+    assert lib.tile_select_topk(g, FAKE, FAKE, 2, FAKE, FAKE, None, ws, None, None) == \
+        _lib.T3D_ERR_INVALID  # workspace missing
+    assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 1.5, 1, 4, FAKE, FAKE, FAKE, ws, None,
+                                None) == _lib.T3D_ERR_INVALID
+    assert lib.tile_select_mass(g, FAKE, FAKE, -1.0, 0.9, 1, 4, FAKE, FAKE, FAKE, ws, None,
+                                None) == _lib.T3D_ERR_INVALID
+    assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 0.9, 0, 4, FAKE, FAKE, FAKE, ws, None,
+                                None) == _lib.T3D_ERR_INVALID
+    assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 0.9, 1, 9, FAKE, FAKE, FAKE, ws, None,
+                                None) == _lib.T3D_ERR_INVALID
+    assert lib.tile_select_mass(g, FAKE, FAKE, 0.1, 0.9, 1, 4, FAKE, FAKE, FAKE, 0, None,
+                                None) == _lib.T3D_ERR_INVALID
     assert lib.tile_prune_queries(_g(T=5), FAKE, 0.95, FAKE, FAKE, FAKE, None) == \
         _lib.T3D_ERR_INVALID
     for ratio in (0.0, -0.5, 1.5, float("nan")):  # the keep ratio must lie in (0, 1]

@@ -26,6 +26,7 @@ def _pooled(B, heads, nT, D, seed, ties=False):
     ((9, 10, 13), 64, 1, False), ((9, 10, 13), 128, 5, False), ((9, 10, 13), 64, 36, False),
     ((9, 10, 13), 64, 50, False), ((9, 10, 13), 128, 7, True), ((4, 8, 8), 64, 2, False),
     ((1, 1, 1), 64, 3, False), ((40, 40, 40), 128, 100, False),
+    ((48, 48, 48), 64, 200, False),  # 1,728 tiles: past the register search, the radix select
 ])
 def test_topk_matches_oracle(grid, D, k, ties):
     T, H, W = grid
@@ -42,8 +43,9 @@ def test_topk_matches_oracle(grid, D, k, ties):
             for h in range(heads):
                 for i in range(nT):
                     np.testing.assert_array_equal(got[b][h][i], want[b][h][i])
-    # random scores leave a data-dependent share of rows within the gap; keep the check non-vacuous
-    assert stats["exact"] >= 0.3 * B * heads * nT
+    # random scores leave a data-dependent share of rows within the gap (28% of the 1,728-tile rows
+    # are decided, more at fewer tiles); keep the check non-vacuous
+    assert stats["exact"] >= (0.25 if nT > 1024 else 0.3) * B * heads * nT
 
 
 def _check_mass(got, S, scale, tau, min_k):
