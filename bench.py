@@ -14,7 +14,9 @@ key-tile pair) per step, with ms per call, and the fraction of the roofline of t
 API with host buffers: every step copies Q, K, V from pinned host memory and the output back.
 
 With N > 1 (torchrun), every rank runs its own replica of the workload (independent batches, no
-data exchange); ``value`` is the kept-block FLOPs of all ranks over the max-over-ranks time.
+data exchange; weak scaling), or with ``--shard heads`` the ranks share one layer by head, each
+taking a contiguous head range of the same full-width rows (strong scaling, still no exchange);
+``value`` is the kept-block FLOPs of all ranks over the max-over-ranks time.
 
 ``--impl reference`` times the CPU oracle (fp64 numpy) on a bounded sample of the same workload
 on the host cores; it is the reported CPU baseline, not a target.
@@ -298,8 +300,15 @@ def run_ours(args, w):
 
     from block_sparse_video_tile3d_b200 import TileSparseAttention, workloads
 
+    from block_sparse_video_tile3d_b200.sharding import head_partition
+
     world, rank, local = rank_env()
-    w = rank_workload(w, rank)
+    shard_heads = args.shard == "heads" and world > 1
+    if shard_heads and world > w.heads:
+        raise SystemExit(f"--shard heads needs at most {w.heads} ranks for {w.name}")
+    if not shard_heads:
+        w = rank_workload(w, rank)
+    h0, nh = head_partition(w.heads, world, rank) if shard_heads else (0, w.heads)
     if world > 1:
         torch.cuda.set_device(local)
         import datetime
@@ -308,15 +317,15 @@ def run_ours(args, w):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
 
-    q, k, v = workloads.make_qkv(w)
-    mask = workloads.block_mask(w) if w.mode == "mask" else None
+    q, k, v = workloads.make_qkv(w)  # in head mode every rank holds the same full-width layer
+    mask = workloads.block_mask(w)[:, h0:h0 + nh].contiguous() if w.mode == "mask" else None
     if w.mode == "bsa":
         pass  # the benchmark runs the workload's own data; query pruning drops what it finds
     qd, kd, vd = (x.to(dev) for x in (q, k, v))
     od = torch.empty_like(qd)
-    model = TileSparseAttention(w.B, w.T, w.H, w.W, w.heads, w.D, mode=w.mode, topk=w.k or None,
+    model = TileSparseAttention(w.B, w.T, w.H, w.W, nh, w.D, mode=w.mode, topk=w.k or None,
                                 mass=w.mass, min_k=w.min_kv, cos_thresh=w.cos_thresh, mask=mask,
-                                device=dev)
+                                device=dev, head0=h0, heads_total=w.heads)
     stages = model.stages(qd, kd, vd, od)
     names = [n for n, _ in stages]
 
@@ -428,27 +437,30 @@ def run_ours(args, w):
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / e2e_steps
-    e2e_same = all(torch.equal(ohs[i], ref_out[i & 1]) for i in range(e2e_steps))
+    e2e_same = all(torch.equal(ohs[i][:, :, h0:h0 + nh], ref_out[i & 1][:, :, h0:h0 + nh])
+                   for i in range(e2e_steps))  # this rank's heads
 
     peaks = _peaks()
+    wb = w.with_(heads=nh)  # this rank's share of the bytes
     attn_ms = stage_ms["attention"]
     achieved = flops / (attn_ms * 1e-3) / 1e12
     kmax = model.kmax
     stage_report = {}
     for n in names:
-        byt = _stage_bytes(w, n, pairs, kmax)
+        byt = _stage_bytes(wb, n, pairs, kmax)
         stage_report[n] = {"ms": round(stage_ms[n], 4),
                            "gbs": round(byt / (stage_ms[n] * 1e-3) / 1e9, 1) if byt else None,
                            "bytes": byt}
     coarse_ms = sum(stage_ms[n] for n in names if n != "attention")
-    coarse_bytes = sum(_stage_bytes(w, n, pairs, kmax) for n in names if n != "attention")
+    coarse_bytes = sum(_stage_bytes(wb, n, pairs, kmax) for n in names if n != "attention")
     line = {
         "metric": METRIC,
         "value": whole_job_tflops(flops_all, ms_step),
         "unit": "TFLOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_step, "ms_per_call": ms_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "higher_is_better": True, "scaling": "strong" if shard_heads else "weak",
+        "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": _describe(w), "kept_pairs": pairs,
                    "kept_block_gflop": flops / 1e9,
@@ -459,7 +471,10 @@ def run_ours(args, w):
                    "density": pairs / (w.B * w.heads * w.nT * w.nT),
                    "l2": "no flush: raster Q/K/V inputs of "
                          f"{3 * w.B * w.L * w.heads * w.D * 2 / 1e6:.0f} MB exceed the 126 MB L2",
-                   "parallelism": f"{world} independent replica(s), one per GPU, each with its "
+                   "parallelism": (f"one layer shared out by head over {world} GPUs (this rank: "
+                                   f"heads {h0}..{h0 + nh - 1}), no data exchange")
+                                  if shard_heads else
+                                  f"{world} independent replica(s), one per GPU, each with its "
                                   "own seed of the workload"},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
@@ -500,6 +515,9 @@ def main():
                     help="workload: tiny, small, large, bsa, ragged_sliding, ragged_random")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas (weak scaling) or one layer shared out by "
+                         "head (strong scaling)")
     ap.add_argument("--cpu-budget", type=float, default=20.0,
                     help="seconds of oracle work for the cpu_baseline sample")
     args = ap.parse_args()

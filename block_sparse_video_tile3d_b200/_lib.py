@@ -20,9 +20,10 @@ STATUS_NAMES = {0: "T3D_OK", 1: "T3D_ERR_INVALID", 2: "T3D_ERR_UNSUPPORTED", 3: 
 
 
 class Geom(ctypes.Structure):
-    """``t3d_geom``: B, T, H, W, heads, D."""
+    """``t3d_geom``: B, T, H, W, heads, D, heads_total (0: = heads), head0."""
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int),
-                ("heads", ctypes.c_int), ("D", ctypes.c_int)]
+                ("heads", ctypes.c_int), ("D", ctypes.c_int), ("heads_total", ctypes.c_int),
+                ("head0", ctypes.c_int)]
 
 
 _P = ctypes.c_void_p

@@ -25,8 +25,18 @@ __all__ = [
 ]
 
 
-def _geom(B, T, H, W, heads, D) -> Geom:
-    return Geom(int(B), int(T), int(H), int(W), int(heads), int(D))
+def _geom(B, T, H, W, heads, D, heads_total=0, head0=0) -> Geom:
+    return Geom(int(B), int(T), int(H), int(W), int(heads), int(D), int(heads_total), int(head0))
+
+
+def _slice(nh: int, head0: int, heads):
+    """(heads, heads_total, head0) of a call on heads head0 .. head0 + heads - 1 of rows of nh
+    heads (every head when ``heads`` is None)."""
+    head0 = int(head0)
+    heads = nh - head0 if heads is None else int(heads)
+    if head0 < 0 or heads < 1 or head0 + heads > nh:
+        raise ValueError(f"heads {head0} .. {head0 + heads - 1} lie outside the {nh} heads of a row")
+    return heads, nh, head0
 
 
 def _stream() -> ctypes.c_void_p:
@@ -66,59 +76,71 @@ def _geometry(T, H, W, B, heads, D):
     return nT.value, Lp.value, tuple(vc)
 
 
-def tile3d_scatter(x: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None):
-    """Raster ``[B, L, heads, D]`` bf16 -> padded tile order ``[B, Lp, heads, D]`` (zero pads)."""
+def tile3d_scatter(x: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None,
+                   head0: int = 0, heads: int | None = None):
+    """Raster ``[B, L, heads, D]`` bf16 -> padded tile order ``[B, Lp, heads, D]`` (zero pads).
+    ``head0``/``heads`` restrict the call to those heads of each row (the rest of ``out`` is left
+    as it is)."""
     B, L, nh, D = x.shape
     _need(x, "x", torch.bfloat16, (B, T * H * W, nh, D))
     _, Lp, _ = _geometry(int(T), int(H), int(W), B, nh, D)
     if out is None:
         out = torch.empty((B, Lp, nh, D), dtype=torch.bfloat16, device=x.device)
     _need(out, "out", torch.bfloat16, (B, Lp, nh, D))
-    g = _geom(B, T, H, W, nh, D)
+    hs = _slice(nh, head0, heads)
+    g = _geom(B, T, H, W, hs[0], D, hs[1], hs[2])
     check(lib.tile3d_scatter(ctypes.byref(g), _ptr(x), _ptr(out), _stream()))
     return out
 
 
-def tile3d_gather(y: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None):
-    """Padded tile order ``[B, Lp, heads, D]`` bf16 -> raster ``[B, L, heads, D]``."""
+def tile3d_gather(y: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None,
+                  head0: int = 0, heads: int | None = None):
+    """Padded tile order ``[B, Lp, heads, D]`` bf16 -> raster ``[B, L, heads, D]`` (the heads
+    ``head0 .. head0 + heads - 1`` only, when given)."""
     B, Lp, nh, D = y.shape
     _, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh, D)
     _need(y, "y", torch.bfloat16, (B, Lp2, nh, D))
     if out is None:
         out = torch.empty((B, T * H * W, nh, D), dtype=torch.bfloat16, device=y.device)
     _need(out, "out", torch.bfloat16, (B, T * H * W, nh, D))
-    g = _geom(B, T, H, W, nh, D)
+    hs = _slice(nh, head0, heads)
+    g = _geom(B, T, H, W, hs[0], D, hs[1], hs[2])
     check(lib.tile3d_gather(ctypes.byref(g), _ptr(y), _ptr(out), _stream()))
     return out
 
 
-def tile_pool(y: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None):
-    """Tile order ``[B, Lp, heads, D]`` bf16 -> per-tile mean ``[B, heads, nT, D]`` fp32."""
+def tile_pool(y: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None,
+              head0: int = 0, heads: int | None = None):
+    """Tile order ``[B, Lp, heads, D]`` bf16 -> per-tile mean ``[B, heads, nT, D]`` fp32 (of the
+    heads ``head0 .. head0 + heads - 1`` when given)."""
     B, Lp, nh, D = y.shape
     nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh, D)
     _need(y, "y", torch.bfloat16, (B, Lp2, nh, D))
+    hs = _slice(nh, head0, heads)
     if out is None:
-        out = torch.empty((B, nh, nT, D), dtype=torch.float32, device=y.device)
-    _need(out, "out", torch.float32, (B, nh, nT, D))
-    g = _geom(B, T, H, W, nh, D)
+        out = torch.empty((B, hs[0], nT, D), dtype=torch.float32, device=y.device)
+    _need(out, "out", torch.float32, (B, hs[0], nT, D))
+    g = _geom(B, T, H, W, hs[0], D, hs[1], hs[2])
     check(lib.tile_pool(ctypes.byref(g), _ptr(y), _ptr(out), _stream()))
     return out
 
 
 def tile3d_scatter_pool(x: torch.Tensor, T: int, H: int, W: int, out: torch.Tensor | None = None,
-                        pooled: torch.Tensor | None = None):
+                        pooled: torch.Tensor | None = None, head0: int = 0,
+                        heads: int | None = None):
     """Scatter and pool in one pass: returns ``(y [B, Lp, heads, D] bf16, pooled [B, heads, nT, D]
     fp32)``, the same as :func:`tile3d_scatter` then :func:`tile_pool`."""
     B, L, nh, D = x.shape
     _need(x, "x", torch.bfloat16, (B, T * H * W, nh, D))
     nT, Lp, _ = _geometry(int(T), int(H), int(W), B, nh, D)
+    hs = _slice(nh, head0, heads)
     if out is None:
         out = torch.empty((B, Lp, nh, D), dtype=torch.bfloat16, device=x.device)
     if pooled is None:
-        pooled = torch.empty((B, nh, nT, D), dtype=torch.float32, device=x.device)
+        pooled = torch.empty((B, hs[0], nT, D), dtype=torch.float32, device=x.device)
     _need(out, "out", torch.bfloat16, (B, Lp, nh, D))
-    _need(pooled, "pooled", torch.float32, (B, nh, nT, D))
-    g = _geom(B, T, H, W, nh, D)
+    _need(pooled, "pooled", torch.float32, (B, hs[0], nT, D))
+    g = _geom(B, T, H, W, hs[0], D, hs[1], hs[2])
     check(lib.tile3d_scatter_pool(ctypes.byref(g), _ptr(x), _ptr(out), _ptr(pooled), _stream()))
     return out, pooled
 
@@ -178,12 +200,14 @@ def tile_select_mass(pq, pk, T, H, W, scale, mass, min_k=1, kmax=None, kv_idx=No
     return kv_idx, kv_cnt
 
 
-def tile_prune_queries(qt, T, H, W, cos_thresh, keep=None, src_row=None, pq_kept=None):
+def tile_prune_queries(qt, T, H, W, cos_thresh, keep=None, src_row=None, pq_kept=None, head0=0,
+                       heads=None):
     """BSA query pruning on tile-ordered ``[B, Lp, heads, D]`` bf16 queries (no pad tiles).
     Returns ``(keep u8 [B, heads, nT, 64], src_row u8 [B, heads, nT, 64], pq_kept f32)``."""
-    B, Lp, nh, D = qt.shape
-    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh, D)
-    _need(qt, "q", torch.bfloat16, (B, Lp2, nh, D))
+    B, Lp, nh_row, D = qt.shape
+    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh_row, D)
+    _need(qt, "q", torch.bfloat16, (B, Lp2, nh_row, D))
+    nh, ht, h0 = _slice(nh_row, head0, heads)
     dev = qt.device
     keep = torch.empty((B, nh, nT, 64), dtype=torch.uint8, device=dev) if keep is None else keep
     src_row = torch.empty((B, nh, nT, 64), dtype=torch.uint8, device=dev) if src_row is None \
@@ -193,18 +217,20 @@ def tile_prune_queries(qt, T, H, W, cos_thresh, keep=None, src_row=None, pq_kept
     _need(keep, "keep", torch.uint8, (B, nh, nT, 64))
     _need(src_row, "src_row", torch.uint8, (B, nh, nT, 64))
     _need(pq_kept, "pq_kept", torch.float32, (B, nh, nT, D))
-    g = _geom(B, T, H, W, nh, D)
+    g = _geom(B, T, H, W, nh, D, ht, h0)
     check(lib.tile_prune_queries(ctypes.byref(g), _ptr(qt), float(cos_thresh), _ptr(keep),
                                  _ptr(src_row), _ptr(pq_kept), _stream()))
     return keep, src_row, pq_kept
 
 
-def tile_prune_queries_ratio(qt, T, H, W, keep_ratio, keep=None, src_row=None, pq_kept=None):
+def tile_prune_queries_ratio(qt, T, H, W, keep_ratio, keep=None, src_row=None, pq_kept=None,
+                             head0=0, heads=None):
     """BSA query pruning keeping ``max(1, floor(64 * keep_ratio))`` rows per block (the rows least
     similar to the block mean). Same inputs and outputs as ``tile_prune_queries``."""
-    B, Lp, nh, D = qt.shape
-    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh, D)
-    _need(qt, "q", torch.bfloat16, (B, Lp2, nh, D))
+    B, Lp, nh_row, D = qt.shape
+    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh_row, D)
+    _need(qt, "q", torch.bfloat16, (B, Lp2, nh_row, D))
+    nh, ht, h0 = _slice(nh_row, head0, heads)
     dev = qt.device
     keep = torch.empty((B, nh, nT, 64), dtype=torch.uint8, device=dev) if keep is None else keep
     src_row = torch.empty((B, nh, nT, 64), dtype=torch.uint8, device=dev) if src_row is None \
@@ -214,7 +240,7 @@ def tile_prune_queries_ratio(qt, T, H, W, keep_ratio, keep=None, src_row=None, p
     _need(keep, "keep", torch.uint8, (B, nh, nT, 64))
     _need(src_row, "src_row", torch.uint8, (B, nh, nT, 64))
     _need(pq_kept, "pq_kept", torch.float32, (B, nh, nT, D))
-    g = _geom(B, T, H, W, nh, D)
+    g = _geom(B, T, H, W, nh, D, ht, h0)
     check(lib.tile_prune_queries_ratio(ctypes.byref(g), _ptr(qt), float(keep_ratio), _ptr(keep),
                                        _ptr(src_row), _ptr(pq_kept), _stream()))
     return keep, src_row, pq_kept
@@ -239,13 +265,15 @@ def block_sparse_attn_workspace_size(B, T, H, W, heads, D, kmax) -> int:
 
 def block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, T, H, W, keep=None, src_row=None,
                           softmax_scale=None, causal=False, num_kv_heads=None, out=None,
-                          workspace=None, dev_status=None):
+                          workspace=None, dev_status=None, head0=0, heads=None):
     """Block-sparse attention on tile-ordered ``[B, Lp, heads, D]`` bf16 Q, K, V over the kept
-    pairs listed in ``kv_idx``/``kv_cnt``. Returns the tile-ordered output."""
-    B, Lp, nh, D = q.shape
-    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh, D)
+    pairs listed in ``kv_idx``/``kv_cnt`` (of the heads ``head0 .. head0 + heads - 1`` when given;
+    the other heads of ``out`` are left as they are). Returns the tile-ordered output."""
+    B, Lp, nh_row, D = q.shape
+    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh_row, D)
     for name, t in (("q", q), ("k", k), ("v", v)):
-        _need(t, name, torch.bfloat16, (B, Lp2, nh, D))
+        _need(t, name, torch.bfloat16, (B, Lp2, nh_row, D))
+    nh, ht, h0 = _slice(nh_row, head0, heads)
     _need(kv_cnt, "kv_cnt", torch.int32, (B, nh, nT))
     _need(kv_idx, "kv_idx", torch.int32)
     if kv_idx.dim() != 4 or tuple(kv_idx.shape[:3]) != (B, nh, nT):
@@ -256,10 +284,10 @@ def block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, T, H, W, keep=None, src_row=N
         _need(src_row, "src_row", torch.uint8, (B, nh, nT, 64))
     if out is None:
         out = torch.empty_like(q)
-    _need(out, "out", torch.bfloat16, (B, Lp2, nh, D))
+    _need(out, "out", torch.bfloat16, (B, Lp2, nh_row, D))
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
     nkv = nh if num_kv_heads is None else int(num_kv_heads)
-    g = _geom(B, T, H, W, nh, D)
+    g = _geom(B, T, H, W, nh, D, ht, h0)
     need = int(lib.block_sparse_attn_workspace_size(ctypes.byref(g), kmax))
     if need > 0 and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -280,20 +308,27 @@ class TileSparseAttention:
     per block — then mass selection from the kept queries) or ``"mask"`` (a fixed uint8 block map
     ``[B, heads, nT, nT]``).
 
-    ``forward(q, k, v)`` takes raster ``[B, L, heads, D]`` bf16 CUDA tensors and returns the raster
-    output; one call = scatter Q, K, V -> coarse selection -> block-sparse attention -> gather.
+    ``forward(q, k, v)`` takes raster ``[B, L, heads_total, D]`` bf16 CUDA tensors and returns the
+    raster output; one call = scatter Q, K, V -> coarse selection -> block-sparse attention ->
+    gather. With ``head0`` and ``heads_total`` given, the instance works on heads
+    ``head0 .. head0 + heads - 1`` of rows of ``heads_total`` heads and writes only those heads'
+    columns of the output: one layer's heads shared out over GPUs, each rank with its own range.
     """
 
     def __init__(self, B, T, H, W, heads, D, mode="topk", topk=None, mass=0.9, min_k=1,
-                 cos_thresh=0.95, mask=None, keep_ratio=None, device="cuda"):
+                 cos_thresh=0.95, mask=None, keep_ratio=None, device="cuda", head0=0,
+                 heads_total=None):
         self.B, self.T, self.H, self.W, self.heads, self.D = B, T, H, W, heads, D
+        self.heads_total = heads if heads_total is None else int(heads_total)
+        self.head0 = int(head0)
+        _slice(self.heads_total, self.head0, heads)
         self.mode = mode
         self.nT, self.Lp, self.vc = geometry(T, H, W, B, heads, D)
         self.scale = 1.0 / math.sqrt(D)
         self.topk, self.mass, self.min_k, self.cos_thresh = topk, mass, min_k, cos_thresh
         self.keep_ratio = keep_ratio
         dev = torch.device(device)
-        shp = (B, self.Lp, heads, D)
+        shp = (B, self.Lp, self.heads_total, D)
         self.qt = torch.empty(shp, dtype=torch.bfloat16, device=dev)
         self.kt = torch.empty(shp, dtype=torch.bfloat16, device=dev)
         self.vt = torch.empty(shp, dtype=torch.bfloat16, device=dev)
@@ -330,35 +365,37 @@ class TileSparseAttention:
         one library call on the current stream. ``forward`` runs them in order; a profiler or a
         benchmark can interleave its own events between them."""
         T, H, W = self.T, self.H, self.W
+        hr = {"head0": self.head0, "heads": self.heads}  # this instance's heads of a row
         if out is None:
-            out = torch.empty((self.B, T * H * W, self.heads, self.D), dtype=torch.bfloat16,
+            out = torch.empty((self.B, T * H * W, self.heads_total, self.D), dtype=torch.bfloat16,
                               device=q.device)
         self._out = out
         if self.mode == "mask":
             st = [
-                ("scatter_q", lambda: tile3d_scatter(q, T, H, W, self.qt)),
-                ("scatter_k", lambda: tile3d_scatter(k, T, H, W, self.kt)),
-                ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt)),
+                ("scatter_q", lambda: tile3d_scatter(q, T, H, W, self.qt, **hr)),
+                ("scatter_k", lambda: tile3d_scatter(k, T, H, W, self.kt, **hr)),
+                ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt, **hr)),
                 ("mask_to_index", lambda: block_mask_to_index(
                     self.mask, T, H, W, self.D, self.kmax, self.kv_idx, self.kv_cnt,
                     self.status)),
             ]
         else:
             if self.mode == "bsa":  # queries are pooled over kept rows, by the pruning kernel
-                st = [("scatter_q", lambda: tile3d_scatter(q, T, H, W, self.qt))]
+                st = [("scatter_q", lambda: tile3d_scatter(q, T, H, W, self.qt, **hr))]
             else:
                 st = [("scatter_pool_q",
-                       lambda: tile3d_scatter_pool(q, T, H, W, self.qt, self.pq))]
+                       lambda: tile3d_scatter_pool(q, T, H, W, self.qt, self.pq, **hr))]
             st += [
-                ("scatter_pool_k", lambda: tile3d_scatter_pool(k, T, H, W, self.kt, self.pk)),
-                ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt)),
+                ("scatter_pool_k", lambda: tile3d_scatter_pool(k, T, H, W, self.kt, self.pk,
+                                                               **hr)),
+                ("scatter_v", lambda: tile3d_scatter(v, T, H, W, self.vt, **hr)),
             ]
             if self.mode == "bsa" and self.keep_ratio is not None:
                 st.append(("prune_q", lambda: tile_prune_queries_ratio(
-                    self.qt, T, H, W, self.keep_ratio, self.keep, self.src_row, self.pq)))
+                    self.qt, T, H, W, self.keep_ratio, self.keep, self.src_row, self.pq, **hr)))
             elif self.mode == "bsa":
                 st.append(("prune_q", lambda: tile_prune_queries(
-                    self.qt, T, H, W, self.cos_thresh, self.keep, self.src_row, self.pq)))
+                    self.qt, T, H, W, self.cos_thresh, self.keep, self.src_row, self.pq, **hr)))
             if self.mode == "topk":
                 st.append(("select_topk", lambda: tile_select_topk(
                     self.pq, self.pk, T, H, W, self.topk, self.kv_idx, self.kv_cnt, self.status,
@@ -370,8 +407,8 @@ class TileSparseAttention:
         st.append(("attention", lambda: block_sparse_attn_fwd(
             self.qt, self.kt, self.vt, self.kv_idx, self.kv_cnt, T, H, W, keep=self.keep,
             src_row=self.src_row, softmax_scale=self.scale, out=self.ot,
-            workspace=self.workspace, dev_status=self.status)))
-        st.append(("gather", lambda: tile3d_gather(self.ot, T, H, W, out)))
+            workspace=self.workspace, dev_status=self.status, **hr)))
+        st.append(("gather", lambda: tile3d_gather(self.ot, T, H, W, out, **hr)))
         return st
 
     def forward(self, q, k, v, out=None):

@@ -42,13 +42,22 @@ t3d_status check_geom(const t3d_geom* g, t3d::Geo* out) {
                 g->T, g->H, g->W, g->heads);
   if (g->D != 64 && g->D != 128)
     return fail(T3D_ERR_UNSUPPORTED, "head dimension D=%d is not supported (64 or 128)", g->D);
+  if (g->head0 < 0 || g->heads_total < 0)
+    return fail(T3D_ERR_INVALID, "head0=%d and heads_total=%d must be >= 0", g->head0,
+                g->heads_total);
+  if (g->heads_total == 0 && g->head0 != 0)
+    return fail(T3D_ERR_INVALID, "head0=%d needs heads_total (0 means heads_total = heads)",
+                g->head0);
+  if (g->heads_total > 0 && g->head0 + g->heads > g->heads_total)
+    return fail(T3D_ERR_INVALID, "heads %d .. %d lie outside the %d heads of a row", g->head0,
+                g->head0 + g->heads - 1, g->heads_total);
   const t3d::Geo geo = t3d::make_geo(*g);
   if (geo.nT > t3d::kMaxTiles)
     return fail(T3D_ERR_UNSUPPORTED, "%d tiles exceed the supported maximum %d", geo.nT,
                 t3d::kMaxTiles);
-  if ((long long)g->B * geo.Lp * g->heads > (1LL << 31))
-    return fail(T3D_ERR_UNSUPPORTED, "B * Lp * heads = %lld token-head rows exceeds 2^31",
-                (long long)g->B * geo.Lp * g->heads);
+  if ((long long)g->B * geo.Lp * geo.heads_total > (1LL << 31))
+    return fail(T3D_ERR_UNSUPPORTED, "B * Lp * heads_total = %lld token-head rows exceeds 2^31",
+                (long long)g->B * geo.Lp * geo.heads_total);
   *out = geo;
   return T3D_OK;
 }

@@ -191,8 +191,9 @@ __device__ __forceinline__ bool load_pair(const Geo& g, const UnitInfo& ui, int 
   mbar_expect_tx(&full[st], Cfg<kD>::kPairBytes);
   for (int hh = 0; hh < Cfg<kD>::kHalves; ++hh) {
     uint8_t* dst = ring[st] + hh * 2 * kTileBytes;
-    tma_load_3d(dst, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + ja * kTileElems);
-    tma_load_3d(dst + kTileBytes, map, &full[st], 64 * hh, ui.h, ui.b * g.Lp + jb * kTileElems);
+    tma_load_3d(dst, map, &full[st], 64 * hh, g.head0 + ui.h, ui.b * g.Lp + ja * kTileElems);
+    tma_load_3d(dst + kTileBytes, map, &full[st], 64 * hh, g.head0 + ui.h,
+                ui.b * g.Lp + jb * kTileElems);
   }
   return true;
 }
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_expect_tx(&s.q_full, C::kQBytes);
           const int row0 = ui.b * g.Lp + ui.i * kTileElems;
           for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, ui.h, row0);
+            tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, g.head0 + ui.h, row0);
           ++nq;
           for (int n = 0; n < ui.npairs; ++n, ++gp) {  // gp counts the loads issued
             if (!load_pair<kD, kVStages>(g, ui, n, gp, &maps.v, s.v, s.v_full, s.v_empty,
@@ -432,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = tmem + ((uint32_t)(sp * 32) << 16);
     const uint32_t t_s = lane_base + kColS + 128 * (uint32_t)wg;  // this warpgroup's S buffer
     const uint32_t t_p = lane_base + kColP + 64 * (uint32_t)wg;   // and P buffer
-    const long ld = (long)g.heads * kD;
+    const long ld = (long)g.heads_total * kD;
     const int col0 = kCols * wg;        // output columns this warpgroup writes
     const bool reporter = wg == 0 && sp == 0 && lane == 0;  // records list-size problems
     int active = 0;
@@ -459,7 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         report(a.dev_status, ui.over ? T3D_DEV_OVERFLOW : T3D_DEV_INDEX_RANGE);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
       const int vci = s.vc[ui.i];
-      __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)ui.h * kD;
+      __nv_bfloat16* out =
+          static_cast<__nv_bfloat16*>(a.o) + row0 * ld + (long)(g.head0 + ui.h) * kD;
       if (ui.npairs == 0) {
         // No kept key tile: this thread's two output rows are zero (this warpgroup's columns).
         for (int c = col0 + 2 * t0; c < col0 + kCols; c += 8) {
@@ -717,10 +719,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---------------------------------------------------------------------------------- host side
 
-// 3D map over a [B * Lp, heads, D] bf16 tensor; box = 64 rows x 1 head x 64 elements, 128B swizzle.
+// 3D map over a [B * Lp, heads_total, D] bf16 tensor; box = 64 rows x 1 head x 64 elements, 128B
+// swizzle (a unit of head h reads head coordinate head0 + h).
 bool make_map(CUtensorMap* m, const void* base, const Geo& g) {
-  const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.heads, (cuuint64_t)g.B * g.Lp};
-  const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.heads * g.D * 2};
+  const cuuint64_t dims[3] = {(cuuint64_t)g.D, (cuuint64_t)g.heads_total, (cuuint64_t)g.B * g.Lp};
+  const cuuint64_t strides[2] = {(cuuint64_t)g.D * 2, (cuuint64_t)g.heads_total * g.D * 2};
   const cuuint32_t box[3] = {64, 1, 64};
   return encode_bf16_map(m, base, 3, dims, strides, box);
 }

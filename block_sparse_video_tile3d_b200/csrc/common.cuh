@@ -19,17 +19,24 @@ constexpr int kTile = 4;
 constexpr int kTileElems = 64;
 constexpr int kMaxTiles = 4096;
 
+// Activations are [B, L or Lp, heads_total, D]; a call works on heads head0 .. head0 + heads - 1
+// (per-head outputs such as pooled tiles and kept lists are [B, heads, ...] for those heads only).
 struct Geo {
   int B, T, H, W, heads, D;
+  int heads_total, head0;
   int nt, nh, nw;  // tiles along t, h, w
   int nT;          // nt * nh * nw
   int L, Lp;       // raster length, padded tile-order length (64 * nT)
-  int row_chunks;  // 16-byte chunks in one token row of heads * D bf16
+  int row_chunks;  // 16-byte chunks of this call's heads in one token row (heads * D bf16)
+  int row_stride;  // 16-byte chunks in one whole token row (heads_total * D bf16)
+  int row_off;     // 16-byte chunks before this call's first head (head0 * D bf16)
 };
 
 inline Geo make_geo(const t3d_geom& g) {
   Geo r;
   r.B = g.B; r.T = g.T; r.H = g.H; r.W = g.W; r.heads = g.heads; r.D = g.D;
+  r.heads_total = g.heads_total > 0 ? g.heads_total : g.heads;
+  r.head0 = g.head0;
   r.nt = (g.T + kTile - 1) / kTile;
   r.nh = (g.H + kTile - 1) / kTile;
   r.nw = (g.W + kTile - 1) / kTile;
@@ -37,6 +44,8 @@ inline Geo make_geo(const t3d_geom& g) {
   r.L = g.T * g.H * g.W;
   r.Lp = kTileElems * r.nT;
   r.row_chunks = g.heads * g.D / 8;
+  r.row_stride = r.heads_total * g.D / 8;
+  r.row_off = r.head0 * g.D / 8;
   return r;
 }
 

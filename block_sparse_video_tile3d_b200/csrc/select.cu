@@ -644,8 +644,9 @@ __global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_
   __shared__ int n_keep;
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const long row_stride = (long)g.heads * D;
-  const __nv_bfloat16* base = q + ((long)b * g.Lp + (long)i * kTileElems) * row_stride + (long)h * D;
+  const long row_stride = (long)g.heads_total * D;
+  const __nv_bfloat16* base =
+      q + ((long)b * g.Lp + (long)i * kTileElems) * row_stride + (long)(g.head0 + h) * D;
   for (int e = tid; e < kTileElems * D / 8; e += kPruneThreads) {
     const int r = e / (D / 8), c = e - r * (D / 8);
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + r * row_stride) + c);

@@ -4,10 +4,10 @@
 // postprocess_output), video_sparse_attn_h3 page (tile(): padded tile buffer, zero pads) and the
 // fastvideo.attention.backends page (sla.mean_pool).
 //
-// All three kernels are HBM-bound streams over [*, heads * D] bf16 token rows. A row is
-// heads * D * 2 bytes (3 KB for 12 heads x 128), so one warp moves one row with 16-byte vector
-// accesses; the source/destination row is computed arithmetically from the geometry (no index
-// tensor is read).
+// All of them are HBM-bound streams over the [*, heads * D] bf16 slice of token rows that a call
+// covers (heads head0 .. head0 + heads - 1 of rows of heads_total heads). A slice is heads * D * 2
+// bytes (3 KB for 12 heads x 128), so one warp moves one row with 16-byte vector accesses; the
+// source/destination row is computed arithmetically from the geometry (no index tensor is read).
 #include "kernels.h"
 
 namespace t3d {
@@ -50,11 +50,11 @@ __global__ void __launch_bounds__(kCopyThreads) scatter_kernel(Geo g, const uint
     const int b = (int)(row / g.Lp);
     const int p = (int)(row - (long)b * g.Lp);
     const int src = padded_to_raster(g, p);
-    uint4* dst = y + row * cpr;
+    uint4* dst = y + row * g.row_stride + g.row_off;
     if (src < 0) {
       zero_row(dst, cpr, lane);
     } else {
-      copy_row(x + ((long)b * g.L + src) * cpr, dst, cpr, lane);
+      copy_row(x + ((long)b * g.L + src) * g.row_stride + g.row_off, dst, cpr, lane);
     }
   }
 }
@@ -71,7 +71,8 @@ __global__ void __launch_bounds__(kCopyThreads) gather_kernel(Geo g, const uint4
     const int b = (int)(row / g.L);
     const int tok = (int)(row - (long)b * g.L);
     const int p = raster_to_padded(g, tok);
-    copy_row(y + ((long)b * g.Lp + p) * cpr, x + row * cpr, cpr, lane);
+    copy_row(y + ((long)b * g.Lp + p) * g.row_stride + g.row_off,
+             x + row * g.row_stride + g.row_off, cpr, lane);
   }
 }
 
@@ -93,10 +94,10 @@ __global__ void __launch_bounds__(32 * kPoolRows) pool_kernel(Geo g, const uint4
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = 0.f;
   if (c < g.row_chunks) {
-    const uint4* base = y + ((long)b * g.Lp + (long)i * kTileElems) * g.row_chunks + c;
+    const uint4* base = y + ((long)b * g.Lp + (long)i * kTileElems) * g.row_stride + g.row_off + c;
 #pragma unroll 4
     for (int r = ry; r < vc; r += kPoolRows) {
-      const uint4 u = ld_nc(base + (long)r * g.row_chunks);
+      const uint4 u = ld_nc(base + (long)r * g.row_stride);
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -150,13 +151,14 @@ __global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_kernel(Geo g,
     // All four of this thread's rows are loaded before any is used, so the four loads are in
     // flight together; pad slots read as zero and add nothing to the sums.
     constexpr int kPer = kTileElems / kPoolRows;
-    const long dst0 = ((long)b * g.Lp + (long)i * kTileElems) * g.row_chunks + c;
+    const long dst0 = ((long)b * g.Lp + (long)i * kTileElems) * g.row_stride + g.row_off + c;
     const long src_b = (long)b * g.L;
     uint4 u[kPer];
 #pragma unroll
     for (int t = 0; t < kPer; ++t) {
       const int sr = src_row[ry + kPoolRows * t];
-      u[t] = sr >= 0 ? ld_nc(x + (src_b + sr) * g.row_chunks + c) : make_uint4(0u, 0u, 0u, 0u);
+      u[t] = sr >= 0 ? ld_nc(x + (src_b + sr) * g.row_stride + g.row_off + c)
+                     : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int t = 0; t < kPer; ++t) {
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_kernel(Geo g,
         acc[2 * e] += f.x;
         acc[2 * e + 1] += f.y;
       }
-      y[dst0 + (long)(ry + kPoolRows * t) * g.row_chunks] = u[t];
+      y[dst0 + (long)(ry + kPoolRows * t) * g.row_stride] = u[t];
     }
   }
 #pragma unroll

@@ -13,9 +13,14 @@
  *  - All tensor pointers are DEVICE pointers owned by the caller; the library never frees or
  *    keeps them, and allocates no device memory. The only device memory it touches beyond its
  *    arguments is the caller-sized workspace of block_sparse_attn_fwd.
- *  - Activations are bf16, layout [B, L, heads, D] with D fastest (raster order, L = T*H*W) or
- *    [B, Lp, heads, D] (tile order, Lp = 64 * nT). Tile i occupies rows [64 i, 64 i + 64); its
- *    vc_i valid tokens fill slots 0 .. vc_i - 1 in in-tile raster order, the rest are zero.
+ *  - Activations are bf16, layout [B, L, heads_total, D] with D fastest (raster order,
+ *    L = T*H*W) or [B, Lp, heads_total, D] (tile order, Lp = 64 * nT). Tile i occupies rows
+ *    [64 i, 64 i + 64); its vc_i valid tokens fill slots 0 .. vc_i - 1 in in-tile raster order,
+ *    the rest are zero. A call works on heads head0 .. head0 + heads - 1 of those rows (all of
+ *    them by default: heads_total = 0 means heads_total = heads, head0 = 0) and leaves the other
+ *    heads' columns untouched; per-head arrays (pooled tiles, kept lists, pruning masks) cover
+ *    the call's heads only: [B, heads, ...]. This is how one layer's heads are shared out over
+ *    GPUs with no data exchange: each rank passes its own head range of the same full rows.
  *  - Tiles are numbered t-tile major, then h-tile, then w-tile; nT = ceil(T/4)*ceil(H/4)*ceil(W/4).
  *  - Every call is asynchronous on `stream` (0 = legacy default stream), never synchronises, and
  *    returns a t3d_status. Argument errors are detected on the host before anything is enqueued.
@@ -54,12 +59,14 @@ typedef enum {
 
 /* Problem geometry. The tile is fixed at 4 x 4 x 4 = 64 tokens. */
 typedef struct {
-  int B;     /* batch */
-  int T;     /* latent frames */
-  int H;     /* latent height */
-  int W;     /* latent width */
-  int heads; /* attention heads (query heads == key/value heads) */
-  int D;     /* head dimension */
+  int B;           /* batch */
+  int T;           /* latent frames */
+  int H;           /* latent height */
+  int W;           /* latent width */
+  int heads;       /* attention heads this call works on (query heads == key/value heads) */
+  int D;           /* head dimension */
+  int heads_total; /* heads in one activation row; 0: equal to `heads` */
+  int head0;       /* first head of this call within a row; 0 when heads_total is 0 */
 } t3d_geom;
 
 /* Human-readable description of the last error on this host thread ("" if none). */

@@ -18,6 +18,8 @@ int main(int argc, char** argv) {
   g.W = atoi(argv[4]);
   g.heads = atoi(argv[5]);
   g.D = atoi(argv[6]);
+  g.heads_total = 0; /* every head of the row */
+  g.head0 = 0;
   int nT = 0, Lp = 0;
   t3d_status st = tile3d_geometry(&g, &nT, &Lp, NULL);
   if (st != T3D_OK) {

@@ -86,6 +86,35 @@ def test_attention_contract_rejections():
     assert _attn(wsp=ODD) == _lib.T3D_ERR_INVALID
 
 
+def test_head_ranges_are_validated():
+    def geom(heads, heads_total, head0):
+        return ctypes.byref(Geom(1, 4, 8, 8, heads, 64, heads_total, head0))
+    nT, Lp = ctypes.c_int(), ctypes.c_int()
+    ok = lambda g: lib.tile3d_geometry(g, ctypes.byref(nT), ctypes.byref(Lp), None)  # noqa: E731
+    assert ok(geom(3, 8, 5)) == _lib.T3D_OK                # heads 5, 6, 7 of 8
+    assert ok(geom(3, 0, 0)) == _lib.T3D_OK                # every head of the row
+    assert ok(geom(3, 8, 6)) == _lib.T3D_ERR_INVALID       # would reach head 8 of 8
+    assert b"outside" in lib.t3d_last_error_string()
+    assert ok(geom(3, 0, 1)) == _lib.T3D_ERR_INVALID       # an offset needs the row's head count
+    assert ok(geom(3, 8, -1)) == _lib.T3D_ERR_INVALID
+    assert ok(geom(3, -2, 0)) == _lib.T3D_ERR_INVALID
+
+
+def test_head_partition_tiles_the_heads():
+    from block_sparse_video_tile3d_b200.sharding import head_partition
+    for heads in (1, 2, 12, 24, 40):
+        for world in (1, 2, 3, 4, 8):
+            parts = [head_partition(heads, world, r) for r in range(world)]
+            covered = [h for h0, n in parts for h in range(h0, h0 + n)]
+            assert covered == list(range(heads))
+            counts = [n for _, n in parts if n]
+            assert max(counts) - min(counts) <= 1
+    assert head_partition(12, 8, 0) == (0, 2) and head_partition(12, 8, 7) == (11, 1)
+    assert head_partition(2, 4, 3) == (2, 0)
+    with pytest.raises(ValueError):
+        head_partition(12, 2, 2)
+
+
 def test_testing_hook_validates_and_resets():
     assert lib.t3d_testing_set_wait_cycles(-1) == _lib.T3D_ERR_INVALID
     assert lib.t3d_testing_set_wait_cycles(1000) == _lib.T3D_OK

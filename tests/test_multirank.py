@@ -1,10 +1,12 @@
-"""Host-side logic of the N > 1 benchmark path, run as world-size-2 gloo process groups on CPU.
+"""Host-side logic of the N > 1 paths, run as world-size-2 gloo process groups on CPU.
 
-With several GPUs every rank runs its own replica of the hot path (no data-path collective); the
+With several GPUs either every rank runs its own replica of the hot path, or the ranks share one
+layer by head (each its own head range of the same rows); neither has a data-path collective. The
 only cross-rank steps are the host reductions in bench.py: the max of the ranks' step times and the
 sum of their kept-block FLOPs. These tests run those steps on CPU ranks, with per-rank problems whose
-FLOPs come from the oracle's selection on the tiny workload, and check that a rank that leaves before
-a collective makes the other rank's collective fail with an error instead of waiting forever.
+FLOPs come from the oracle's selection on the tiny workload; check that a layer shared by head and
+reassembled equals the one-rank result bit for bit; and check that a rank that leaves before a
+collective makes the other rank's collective fail with an error instead of waiting forever.
 """
 from __future__ import annotations
 
@@ -94,6 +96,69 @@ def test_two_ranks_replicas_reduce_to_whole_job_value():
         assert r["value"] == pytest.approx(sum(flops) / (max(times) * 1e-3) / 1e12, rel=1e-12)
     # top-k keeps k tiles per query tile on every rank: equal FLOPs, different data
     assert flops[0] == flops[1] > 0
+
+
+def _head_shard_worker(rank: int, port: int, out_dir: str, name: str) -> None:
+    import numpy as np
+
+    from block_sparse_video_tile3d_b200 import workloads
+    from block_sparse_video_tile3d_b200.sharding import head_partition
+    from oracle import pipeline
+
+    _init(rank, port, 120.0)
+    try:
+        w = _shard_workload(name)
+        q, k, v = workloads.make_qkv(w)  # every rank holds the same full-width layer
+        mask = workloads.block_mask(w).numpy() if w.mode == "mask" else None
+        h0, n = head_partition(w.heads, WORLD, rank)
+        hs = slice(h0, h0 + n)
+        kw = dict(scale=w.scale, topk=w.k) if w.mode == "topk" else dict(scale=w.scale,
+                                                                          mask=mask[:, hs])
+        mine = pipeline.forward(q[:, :, hs], k[:, :, hs], v[:, :, hs], w.T, w.H, w.W, w.mode,
+                                **kw)["o"]
+        parts = [None] * WORLD
+        dist.all_gather_object(parts, (h0, n, mine))
+        if rank == 0:
+            full = np.zeros((w.B, w.L, w.heads, w.D))
+            for ph0, pn, po in parts:
+                full[:, :, ph0:ph0 + pn] = po
+            kw1 = dict(scale=w.scale, topk=w.k) if w.mode == "topk" else dict(scale=w.scale,
+                                                                               mask=mask)
+            one = pipeline.forward(q, k, v, w.T, w.H, w.W, w.mode, **kw1)["o"]
+            np.save(os.path.join(out_dir, "sharded.npy"), full)
+            np.save(os.path.join(out_dir, "one.npy"), one)
+            with open(os.path.join(out_dir, "ranges.json"), "w") as f:
+                json.dump([[p[0], p[1]] for p in parts], f)
+    finally:
+        dist.destroy_process_group()
+
+
+def _shard_workload(name):
+    from block_sparse_video_tile3d_b200 import workloads
+    if name == "tiny":
+        return workloads.WORKLOADS["tiny"]
+    # the ragged workload's recipe and mask on a smaller ragged grid, with an odd head count
+    return workloads.WORKLOADS["ragged_sliding"].with_(B=2, T=9, H=10, W=13, heads=3)
+
+
+@pytest.mark.parametrize("name", ["tiny", "ragged"])
+def test_two_ranks_share_a_layer_by_head(name):
+    """Each rank runs the whole path (oracle) on its own head range of the same full-width layer;
+    reassembled by head, the result equals the one-rank run bit for bit (no head depends on
+    another, so no data exchange is needed)."""
+    import numpy as np
+
+    port = _free_port()
+    with tempfile.TemporaryDirectory() as d:
+        mp.start_processes(_head_shard_worker, args=(port, d, name), nprocs=WORLD, join=True,
+                           start_method="spawn")
+        full = np.load(os.path.join(d, "sharded.npy"))
+        one = np.load(os.path.join(d, "one.npy"))
+        ranges = json.load(open(os.path.join(d, "ranges.json")))
+    w = _shard_workload(name)
+    assert sorted(h for h0, n in ranges for h in range(h0, h0 + n)) == list(range(w.heads))
+    assert all(n >= 1 for _, n in ranges)
+    np.testing.assert_array_equal(full, one)
 
 
 def _leaver_worker(rank: int, port: int, out_dir: str) -> None:
