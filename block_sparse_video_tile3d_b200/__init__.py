@@ -10,7 +10,8 @@ __version__ = "0.1.0"
 
 _API = (
     "Geom", "Tile3dError", "TileSparseAttention", "block_mask_to_index", "block_sparse_attn_fwd",
-    "block_sparse_attn_workspace_size", "geometry", "tile3d_gather", "tile3d_scatter",
+    "block_sparse_attn_workspace_size", "block_sparse_attn_fwd_lse", "block_sparse_attn_bwd",
+    "block_sparse_attn_bwd_workspace_size", "geometry", "tile3d_gather", "tile3d_scatter",
     "tile3d_scatter_pool", "tile_pool", "tile_prune_queries", "tile_prune_queries_ratio",
     "tile_select_mass", "tile_select_topk", "tile_select_workspace_size",
 )

@@ -50,6 +50,11 @@ SIGNATURES = {
     "block_sparse_attn_fwd": (_I, [_G, _P, _P, _P, _P, _P, _P, _I, _P, _P, _F, _I, _I, _P, _S,
                                    _P, _P]),
     "block_sparse_attn_workspace_size": (_S, [_G, _I]),
+    "block_sparse_attn_fwd_lse": (_I, [_G, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _F, _I, _I, _P,
+                                       _S, _P, _P]),
+    "block_sparse_attn_bwd": (_I, [_G, _P, _P, _P, _P, _P, _P, _P, _P, _I, _P, _P, _F, _I, _I,
+                                   _P, _P, _P, _P, _S, _P, _P]),
+    "block_sparse_attn_bwd_workspace_size": (_S, [_G, _I]),
     "block_sparse_attn_fwd_noalloc": (_I, [_G, _P, _P, _P, _P, _P, _P, _I, _P, _P, _F, _I, _I,
                                            _P, _P]),
     # include/tile3d_testing.h

@@ -21,7 +21,8 @@ __all__ = [
     "tile_select_topk", "tile_select_mass", "tile_select_workspace_size", "tile_prune_queries",
     "tile_prune_queries_ratio",
     "block_mask_to_index",
-    "block_sparse_attn_fwd", "block_sparse_attn_workspace_size", "TileSparseAttention",
+    "block_sparse_attn_fwd", "block_sparse_attn_workspace_size", "block_sparse_attn_fwd_lse",
+    "block_sparse_attn_bwd", "block_sparse_attn_bwd_workspace_size", "TileSparseAttention",
 ]
 
 
@@ -297,6 +298,82 @@ def block_sparse_attn_fwd(q, k, v, kv_idx, kv_cnt, T, H, W, keep=None, src_row=N
                                     scale, int(bool(causal)), nkv, _ptr(workspace), ws_bytes,
                                     _ptr(dev_status), _stream()))
     return out
+
+
+def _attn_common(q, kv_idx, kv_cnt, T, H, W, keep, src_row, head0, heads):
+    B, Lp, nh_row, D = q.shape
+    nT, Lp2, _ = _geometry(int(T), int(H), int(W), B, nh_row, D)
+    nh, ht, h0 = _slice(nh_row, head0, heads)
+    _need(kv_cnt, "kv_cnt", torch.int32, (B, nh, nT))
+    _need(kv_idx, "kv_idx", torch.int32)
+    if kv_idx.dim() != 4 or tuple(kv_idx.shape[:3]) != (B, nh, nT):
+        raise ValueError(f"kv_idx must have shape [B, heads, nT, kmax], got {tuple(kv_idx.shape)}")
+    if keep is not None:
+        _need(keep, "keep", torch.uint8, (B, nh, nT, 64))
+        _need(src_row, "src_row", torch.uint8, (B, nh, nT, 64))
+    return B, Lp2, nh_row, D, nT, nh, ht, h0
+
+
+def block_sparse_attn_fwd_lse(q, k, v, kv_idx, kv_cnt, T, H, W, keep=None, src_row=None,
+                              softmax_scale=None, out=None, lse=None, workspace=None,
+                              dev_status=None, head0=0, heads=None):
+    """:func:`block_sparse_attn_fwd` that also returns each query row's log-sum-exp (fp32
+    ``[B, heads, Lp]``, natural log), for the backward pass. Returns ``(out, lse)``."""
+    B, Lp, nh_row, D, nT, nh, ht, h0 = _attn_common(q, kv_idx, kv_cnt, T, H, W, keep, src_row,
+                                                    head0, heads)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _need(t, name, torch.bfloat16, (B, Lp, nh_row, D))
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, nh, Lp), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(out, "out", torch.bfloat16, (B, Lp, nh_row, D))
+    _need(lse, "lse", torch.float32, (B, nh, Lp))
+    kmax = int(kv_idx.shape[3])
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    g = _geom(B, T, H, W, nh, D, ht, h0)
+    need = int(lib.block_sparse_attn_workspace_size(ctypes.byref(g), kmax))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    check(lib.block_sparse_attn_fwd_lse(ctypes.byref(g), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                        _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt), kmax, _ptr(keep),
+                                        _ptr(src_row), scale, 0, nh, _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _ptr(dev_status), _stream()))
+    return out, lse
+
+
+def block_sparse_attn_bwd_workspace_size(B, T, H, W, heads, D, kmax, heads_total=0, head0=0):
+    g = _geom(B, T, H, W, heads, D, heads_total, head0)
+    return int(lib.block_sparse_attn_bwd_workspace_size(ctypes.byref(g), int(kmax)))
+
+
+def block_sparse_attn_bwd(q, k, v, o, dout, lse, kv_idx, kv_cnt, T, H, W, keep=None,
+                          src_row=None, softmax_scale=None, dq=None, dk=None, dv=None,
+                          workspace=None, dev_status=None, head0=0, heads=None):
+    """Gradients ``(dq, dk, dv)`` (bf16, tile order) of :func:`block_sparse_attn_fwd` for the
+    output gradient ``dout``, with ``o`` and ``lse`` from :func:`block_sparse_attn_fwd_lse`."""
+    B, Lp, nh_row, D, nT, nh, ht, h0 = _attn_common(q, kv_idx, kv_cnt, T, H, W, keep, src_row,
+                                                    head0, heads)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _need(t, name, torch.bfloat16, (B, Lp, nh_row, D))
+    _need(lse, "lse", torch.float32, (B, nh, Lp))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, name, torch.bfloat16, (B, Lp, nh_row, D))
+    kmax = int(kv_idx.shape[3])
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else float(softmax_scale)
+    g = _geom(B, T, H, W, nh, D, ht, h0)
+    need = int(lib.block_sparse_attn_bwd_workspace_size(ctypes.byref(g), kmax))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    check(lib.block_sparse_attn_bwd(ctypes.byref(g), _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                                    _ptr(dout), _ptr(lse), _ptr(kv_idx), _ptr(kv_cnt), kmax,
+                                    _ptr(keep), _ptr(src_row), scale, 0, nh, _ptr(dq), _ptr(dk),
+                                    _ptr(dv), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(),
+                                    _ptr(dev_status), _stream()))
+    return dq, dk, dv
 
 
 class TileSparseAttention:

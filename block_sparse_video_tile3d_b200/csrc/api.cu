@@ -296,6 +296,95 @@ t3d_status block_sparse_attn_fwd(const t3d_geom* g, const void* q, const void* k
   return cuda_status(t3d::launch_attn(geo, a, as_stream(stream)), "block_sparse_attn_fwd");
 }
 
+// The checks every attention entry point makes (BSAAttentionImpl.__init__ contract, pointers,
+// list capacity, pruning geometry).
+static t3d_status check_attn_call(const t3d_geom* g, const t3d::Geo& geo, const void* q,
+                                  const void* k, const void* v, const int32_t* kv_idx,
+                                  const int32_t* kv_cnt, int kmax, const uint8_t* keep,
+                                  const uint8_t* src_row, float softmax_scale, int causal,
+                                  int num_kv_heads) {
+  if (causal != 0)
+    return fail(T3D_ERR_UNSUPPORTED, "the attention is bidirectional; causal=1 is unsupported");
+  if (num_kv_heads != g->heads)
+    return fail(T3D_ERR_UNSUPPORTED,
+                "grouped-query attention is unsupported (num_kv_heads=%d, heads=%d)", num_kv_heads,
+                g->heads);
+  const double expected = 1.0 / sqrt((double)g->D);
+  const double diff = fabs((double)softmax_scale - expected);
+  if (!(diff <= fmax(1e-4 * fmax(fabs((double)softmax_scale), expected), 1e-5)))
+    return fail(T3D_ERR_INVALID, "softmax_scale=%.8g must be 1/sqrt(D)=%.8g", (double)softmax_scale,
+                expected);
+  T3D_CHECK(check_ptr(q, "q"));
+  T3D_CHECK(check_ptr(k, "k"));
+  T3D_CHECK(check_ptr(v, "v"));
+  T3D_CHECK(check_ptr4(kv_idx, "kv_idx"));
+  T3D_CHECK(check_ptr4(kv_cnt, "kv_cnt"));
+  if (kmax < 1 || kmax > geo.nT)
+    return fail(T3D_ERR_INVALID, "kmax=%d must lie in [1, nT=%d]", kmax, geo.nT);
+  if ((keep == nullptr) != (src_row == nullptr))
+    return fail(T3D_ERR_INVALID, "keep and src_row must both be given or both be NULL");
+  if (keep != nullptr && geo.L != geo.Lp)
+    return fail(T3D_ERR_INVALID, "pruned-query attention needs every tile full (L=%d, Lp=%d)",
+                geo.L, geo.Lp);
+  return T3D_OK;
+}
+
+t3d_status block_sparse_attn_fwd_lse(const t3d_geom* g, const void* q, const void* k,
+                                     const void* v, void* o, float* lse, const int32_t* kv_idx,
+                                     const int32_t* kv_cnt, int kmax, const uint8_t* keep,
+                                     const uint8_t* src_row, float softmax_scale, int causal,
+                                     int num_kv_heads, void* workspace, size_t ws_bytes,
+                                     int32_t* dev_status, t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_attn_call(g, geo, q, k, v, kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale,
+                            causal, num_kv_heads));
+  T3D_CHECK(check_ptr(o, "o"));
+  T3D_CHECK(check_ptr(lse, "lse"));
+  const size_t need = t3d::attn_workspace_bytes(geo, kmax);
+  if (ws_bytes < need)
+    return fail(T3D_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
+                ws_bytes, need);
+  T3D_CHECK(check_ptr(workspace, "workspace"));
+  t3d::AttnArgs a{q, k, v, o, kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale,
+                  workspace, ws_bytes, dev_status, g_wait_cycles, lse};
+  return cuda_status(t3d::launch_attn(geo, a, as_stream(stream)), "block_sparse_attn_fwd_lse");
+}
+
+size_t block_sparse_attn_bwd_workspace_size(const t3d_geom* g, int kmax) {
+  t3d::Geo geo;
+  (void)kmax;
+  if (check_geom(g, &geo) != T3D_OK) return 0;
+  return t3d::attn_bwd_workspace_bytes(geo);
+}
+
+t3d_status block_sparse_attn_bwd(const t3d_geom* g, const void* q, const void* k, const void* v,
+                                 const void* o, const void* dout, const float* lse,
+                                 const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                 const uint8_t* keep, const uint8_t* src_row, float softmax_scale,
+                                 int causal, int num_kv_heads, void* dq, void* dk, void* dv,
+                                 void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                 t3d_stream stream) {
+  t3d::Geo geo;
+  T3D_CHECK(check_geom(g, &geo));
+  T3D_CHECK(check_attn_call(g, geo, q, k, v, kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale,
+                            causal, num_kv_heads));
+  T3D_CHECK(check_ptr(o, "o"));
+  T3D_CHECK(check_ptr(dout, "dout"));
+  T3D_CHECK(check_ptr(lse, "lse"));
+  T3D_CHECK(check_ptr(dq, "dq"));
+  T3D_CHECK(check_ptr(dk, "dk"));
+  T3D_CHECK(check_ptr(dv, "dv"));
+  const size_t need = t3d::attn_bwd_workspace_bytes(geo);
+  if (ws_bytes < need)
+    return fail(T3D_ERR_INVALID, "workspace of %zu bytes is smaller than the %zu required",
+                ws_bytes, need);
+  T3D_CHECK(check_ptr(workspace, "workspace"));
+  t3d::AttnBwdArgs a{q, k, v, o, dout, lse, kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale,
+                     dq, dk, dv, workspace, dev_status, g_wait_cycles};
+  return cuda_status(t3d::launch_attn_bwd(geo, a, as_stream(stream)), "block_sparse_attn_bwd");
+}
+
 t3d_status block_sparse_attn_fwd_noalloc(const t3d_geom* g, const void* q, const void* k,
                                          const void* v, void* o, const int32_t* kv_idx,
                                          const int32_t* kv_cnt, int kmax, const uint8_t* keep,

@@ -75,6 +75,7 @@ constexpr int kSoftmaxRegs = 224;
 static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
+constexpr float kLn2 = 0.6931471805599453f;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;       // S buffer b at 128 b
 constexpr uint32_t kColO = 256;
@@ -468,6 +469,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint32_t*>(out + r0 * ld + c) = 0u;
           *reinterpret_cast<uint32_t*>(out + r1 * ld + c) = 0u;
         }
+        if (a.lse != nullptr && wg == 0 && t0 == 0) {
+          float* lr = a.lse + (((long)ui.b * g.heads + ui.h) * g.Lp + (long)ui.i * kTileElems);
+          lr[r0] = -INFINITY;
+          lr[r1] = -INFINITY;
+        }
         continue;
       }
       // mw: the shift this warpgroup used at its latest step of the unit; l is relative to it.
@@ -643,6 +649,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                          (om1 == -INFINITY ? 0.f : ol1 * ex2(om1 - mf1));
         i0 = s0 > 0.f ? 1.f / s0 : 0.f;
         i1 = s1 > 0.f ? 1.f / s1 : 0.f;
+        if (a.lse != nullptr && wg == 0 && t0 == 0) {
+          // log sum_c exp(scale q.k_c) = ln 2 * (final shift + log2 of the sum relative to it)
+          float* lr = a.lse + (((long)ui.b * g.heads + ui.h) * g.Lp + (long)ui.i * kTileElems);
+          lr[r0] = s0 > 0.f ? (mf0 + log2f(s0)) * kLn2 : -INFINITY;
+          lr[r1] = s1 > 0.f ? (mf1 + log2f(s1)) * kLn2 : -INFINITY;
+        }
       }
       // Pruned-query variant: the output rows that take this lane's row (row 16 sp + lane for
       // lane < 16), as a bit mask over the tile's 64 rows: a kept row takes itself, a pruned row

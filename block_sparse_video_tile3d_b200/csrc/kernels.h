@@ -51,7 +51,32 @@ struct AttnArgs {
   size_t ws_bytes;
   int32_t* dev_status;
   long long wait_cycles;  // limit of each pipeline wait, in clock cycles
+  float* lse;             // NULL, or [B, heads, Lp]: each query row's log-sum-exp (natural log)
 };
+
+// Backward pass (attn_bwd.cu): gradients of block_sparse_attn_fwd for an output gradient.
+struct AttnBwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;       // the forward output
+  const void* dout;    // its gradient
+  const float* lse;    // the forward's log-sum-exp per query row, [B, heads, Lp]
+  const int32_t* kv_idx;
+  const int32_t* kv_cnt;
+  int kmax;
+  const uint8_t* keep;
+  const uint8_t* src_row;
+  float scale;
+  void* dq;
+  void* dk;
+  void* dv;
+  void* workspace;     // attn_bwd_workspace_bytes
+  int32_t* dev_status;
+  long long wait_cycles;
+};
+size_t attn_bwd_workspace_bytes(const Geo& g);
+cudaError_t launch_attn_bwd(const Geo& g, const AttnBwdArgs& a, cudaStream_t s);
 
 // Device scratch of the attention kernel: one 32-bit unit counter, padded to 256 bytes.
 constexpr size_t kAttnWorkspaceBytes = 256;

@@ -245,6 +245,54 @@ t3d_status block_sparse_attn_fwd(const t3d_geom* g, const void* q, const void* k
 size_t block_sparse_attn_workspace_size(const t3d_geom* g, int kmax);
 
 /*
+ * block_sparse_attn_fwd_lse — block_sparse_attn_fwd that also returns each query row's
+ * log-sum-exp, the statistic the backward pass needs (training path).
+ * FastVideo API docs, video_sparse_attn_h3 page: tile() gives a gradient-tracking forward its own
+ * buffer; bsa_attn page, BSAAttentionImpl.forward for the forward itself.
+ *   lse: out, fp32 [B, heads, Lp]: lse_r = log sum_c exp(softmax_scale * q_r . k_c) over the valid
+ *        keys of the row's kept tiles (natural log; -inf for a tile with no kept key tile). Pad
+ *        and pruned rows get the value of their own (unused) softmax.
+ *   Every other argument, result and error: as block_sparse_attn_fwd.
+ */
+t3d_status block_sparse_attn_fwd_lse(const t3d_geom* g, const void* q, const void* k,
+                                     const void* v, void* o, float* lse, const int32_t* kv_idx,
+                                     const int32_t* kv_cnt, int kmax, const uint8_t* keep,
+                                     const uint8_t* src_row, float softmax_scale, int causal,
+                                     int num_kv_heads, void* workspace, size_t ws_bytes,
+                                     int32_t* dev_status, t3d_stream stream);
+
+/*
+ * block_sparse_attn_bwd — gradients of block_sparse_attn_fwd with respect to q, k and v.
+ * The pages train through the sparse attention (video_sparse_attn_h3 page, tile(): the
+ * gradient-tracking forward) but print no backward formulas; this is the derivative of the
+ * forward's definition. For an attending query row r with kept keys c:
+ *   p_rc = exp(scale q_r.k_c - lse_r), delta_r = dO_r . o_r, dS_rc = p_rc (dO_r.v_c - delta_r),
+ *   dq_r = scale sum_c dS_rc k_c, dk_c = scale sum_r dS_rc q_r, dv_c = sum_r p_rc dO_r.
+ * No gradient flows through the selection. With keep/src_row (BSA), a pruned row's dO is added to
+ * its source row's and the pruned row's dq is zero. Pad rows and pad keys get zero gradients; a
+ * key tile no query tile kept gets zero dk and dv.
+ *   q, k, v: in, bf16 [B, Lp, heads, D] tile order (the forward's inputs).
+ *   o:       in, the forward's output.  dout: in, bf16 [B, Lp, heads, D]: the output gradient.
+ *   lse:     in, fp32 [B, heads, Lp] from block_sparse_attn_fwd_lse.
+ *   kv_idx, kv_cnt, kmax, keep, src_row, softmax_scale, causal, num_kv_heads: as the forward.
+ *   dq, dk, dv: out, bf16 [B, Lp, heads, D] (the call's heads only).
+ *   workspace: device scratch of at least block_sparse_attn_bwd_workspace_size() bytes (the
+ *            effective output gradient, delta, and the per-key-tile lists of query tiles).
+ * fp32 accumulation in tensor memory; P, dS and the effective dO are rounded to bf16 as MMA
+ * operands; results rounded to bf16 (nearest even). Deterministic: every sum runs in a fixed order.
+ */
+t3d_status block_sparse_attn_bwd(const t3d_geom* g, const void* q, const void* k, const void* v,
+                                 const void* o, const void* dout, const float* lse,
+                                 const int32_t* kv_idx, const int32_t* kv_cnt, int kmax,
+                                 const uint8_t* keep, const uint8_t* src_row, float softmax_scale,
+                                 int causal, int num_kv_heads, void* dq, void* dk, void* dv,
+                                 void* workspace, size_t ws_bytes, int32_t* dev_status,
+                                 t3d_stream stream);
+
+/* Bytes of device workspace block_sparse_attn_bwd needs for this geometry. */
+size_t block_sparse_attn_bwd_workspace_size(const t3d_geom* g, int kmax);
+
+/*
  * block_sparse_attn_fwd_noalloc — block_sparse_attn_fwd for callers that cannot allocate device
  * memory. The paper has no counterpart: this is a library service, not a step of the method.
  * Some callers own no allocator of their own: a plugin inside a host framework whose allocator
