@@ -506,6 +506,68 @@ def run_ours(args, w):
     return 0
 
 
+def run_backward(args, w):
+    """The backward pass on one GPU: selection and forward (with log-sum-exp) once, then K timed
+    calls of block_sparse_attn_bwd for a seeded output gradient. FLOPs count the five products of
+    the backward per kept pair (S = QK^T, dP = dO V^T, dV = P^T dO, dQ = dS K, dK = dS^T Q), each
+    2 * 64 * 64 * D, whatever the kernels recompute."""
+    import torch
+
+    from block_sparse_video_tile3d_b200 import (TileSparseAttention, block_sparse_attn_bwd,
+                                                block_sparse_attn_fwd_lse, tile3d_scatter,
+                                                workloads)
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    q, k, v = workloads.make_qkv(w)
+    do = workloads.make_qkv(w, seed=w.seed + 11)[0]
+    mask = workloads.block_mask(w) if w.mode == "mask" else None
+    model = TileSparseAttention(w.B, w.T, w.H, w.W, w.heads, w.D, mode=w.mode, topk=w.k or None,
+                                mass=w.mass, min_k=w.min_kv, cos_thresh=w.cos_thresh, mask=mask,
+                                device=dev)
+    model(q.to(dev), k.to(dev), v.to(dev))
+    dot = tile3d_scatter(do.to(dev), w.T, w.H, w.W)
+    o, lse = block_sparse_attn_fwd_lse(model.qt, model.kt, model.vt, model.kv_idx, model.kv_cnt,
+                                       w.T, w.H, w.W, keep=model.keep, src_row=model.src_row)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    grads = [torch.empty_like(o) for _ in range(3)]
+
+    def call():
+        block_sparse_attn_bwd(model.qt, model.kt, model.vt, o, dot, lse, model.kv_idx,
+                              model.kv_cnt, w.T, w.H, w.W, keep=model.keep, src_row=model.src_row,
+                              dq=grads[0], dk=grads[1], dv=grads[2], dev_status=status)
+
+    for _ in range(max(args.warmup, 3)):
+        call()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        call()
+    e1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    pairs = int(model.kv_cnt.sum().item())
+    flops = pairs * 10 * 64 * 64 * w.D
+    peaks = _peaks()
+    tflops = flops / (ms * 1e-3) / 1e12
+    line = {"metric": "backward: TFLOPS over kept blocks (5 products of 2*64*64*D per kept pair)",
+            "value": tflops, "unit": "TFLOPS", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "pass": "backward",
+            "config": {"workload": _describe(w), "kept_pairs": pairs, "gflop": flops / 1e9,
+                       "l2": "no flush: Q, K, V, O, dO in tile order exceed the 126 MB L2"},
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
+                         "traffic": None, "kernel": "block_sparse_attn_bwd (all launches)",
+                         "peak_source": f"{peaks['source']} bf16 dense (burst)"},
+            "device_status": int(status.item()), "clocks": clocks}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -514,6 +576,9 @@ def main():
     ap.add_argument("--config", default="small",
                     help="workload: tiny, small, large, bsa, ragged_sliding, ragged_random")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
+                    help="forward: the whole hot path (the benchmark line); backward: the "
+                         "gradients of the fine stage on one GPU")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N > 1: independent replicas (weak scaling) or one layer shared out by "
@@ -527,6 +592,8 @@ def main():
     w = WORKLOADS[args.config]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.which == "backward":
+        return run_backward(args, w)
     return run_ours(args, w)
 
 
