@@ -27,10 +27,10 @@
 // pruned queries) leave no CTA idle before the queue is empty.
 //
 // Roles (12 warps):
-//   warp 0       TMA producer for the K pairs (3-stage ring) and the unit queue
+//   warp 0       TMA producer for the K pairs (2-stage ring) and the unit queue
 //   warp 1       TMEM allocation; one thread issues the S MMAs and their commits
 //   warp 2       one thread issues the PV MMAs and their commits
-//   warp 3       TMA producer for the V pairs (3-stage ring) and for each unit's query tile (one
+//   warp 3       TMA producer for the V pairs (2-stage ring) and for each unit's query tile (one
 //                buffer, refilled once the previous unit's last S has completed, so the next unit's
 //                scores start during the epilogue)
 //   warps 4..11  softmax and epilogue, two warpgroups: warpgroup X takes the steps n with n % 2 == X
@@ -62,8 +62,12 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kKStages = 3;         // K-pair ring depth
-constexpr int kVStages = 3;         // V-pair ring depth
+// K and V pair rings of two stages, one per S / P buffer: stage gp & 1 is free once S(gp - 2)
+// (for K) or PV(gp - 2) (for V) has completed, which the S and PV issuers already signal on
+// s_full / pv_done, so the producers wait on those barriers and no separate "stage empty" commit
+// is issued (an MMA-side commit costs the issuing thread about as much as an MMA).
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
 constexpr int kUnitRing = 8;        // units published ahead by the queue reader
 constexpr int kThreads = 384;       // 12 warps: producers / MMA, two softmax halves
 constexpr int kSoftmaxThreads = 256;  // both softmax warpgroups
@@ -99,11 +103,11 @@ struct alignas(1024) SmemLayout {
   uint8_t k[kKStages][Cfg<kD>::kPairBytes];
   uint8_t v[kVStages][Cfg<kD>::kPairBytes];
   uint8_t q[Cfg<kD>::kQBytes];
-  uint64_t k_full[kKStages], k_empty[kKStages];
-  uint64_t v_full[kVStages], v_empty[kVStages];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t k_full[kKStages];  // a K pair landed (TMA -> S issuer)
+  uint64_t v_full[kVStages];  // a V pair landed (TMA -> PV issuer)
+  uint64_t s_full[2], s_empty[2];  // s_full[b]: S of a step in buffer b (also frees K stage b)
   uint64_t p_full[2];   // P of a step written to TMEM buffer (step & 1) (softmax -> MMA)
-  uint64_t pv_done[2];  // that step's PV MMAs complete: its P buffer free, O current (MMA -> softmax)
+  uint64_t pv_done[2];  // that step's PV MMAs complete: its P buffer and V stage free, O current
   uint64_t q_full;    // the unit's Q loaded (TMA -> MMA)
   uint64_t q_empty;   // the unit's last S MMA complete: Q may be overwritten (MMA -> producer)
   uint64_t o_full;    // the unit's last PV complete (MMA -> softmax)
@@ -178,14 +182,17 @@ struct Maps {
 };
 
 // Loads the K or V pair of step gp of unit ui into stage gp % kStages of a ring once the MMAs that
-// read the stage's previous pair have completed (lane 0 of a producer warp). False on a timeout.
+// read the stage's previous pair have completed, as signalled on `done` (s_full for K, pv_done
+// for V: with two stages, stage gp % 2 is step gp's buffer) (lane 0 of a producer warp). False on
+// a timeout.
 template <int kD, int kStages>
 __device__ __forceinline__ bool load_pair(const Geo& g, const UnitInfo& ui, int n, long gp,
                                           const CUtensorMap* map,
                                           uint8_t (*ring)[Cfg<kD>::kPairBytes], uint64_t* full,
-                                          uint64_t* empty, volatile int* abort_flag, long long lim) {
+                                          uint64_t* done, volatile int* abort_flag, long long lim) {
+  static_assert(kStages == 2, "a stage is step gp's S / P buffer");
   const int st = (int)(gp % kStages);
-  if (!mbar_wait(&empty[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag, lim)) return false;
+  if (!mbar_wait(&done[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag, lim)) return false;
   int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
   if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
   if (jb < 0) jb = ja;
@@ -219,8 +226,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &s.abort;
 
   if (threadIdx.x == 0) {
-    for (int t = 0; t < kKStages; ++t) { mbar_init(&s.k_full[t], 1); mbar_init(&s.k_empty[t], 1); }
-    for (int t = 0; t < kVStages; ++t) { mbar_init(&s.v_full[t], 1); mbar_init(&s.v_empty[t], 1); }
+    for (int t = 0; t < kKStages; ++t) mbar_init(&s.k_full[t], 1);
+    for (int t = 0; t < kVStages; ++t) mbar_init(&s.v_full[t], 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s.s_full[t], 1);
       mbar_init(&s.s_empty[t], kWgThreads);
@@ -283,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nxt = (int)atomicAdd(next_unit, 1u);
           const UnitInfo ui = unit_info(g, a, u);
           for (int n = 0; n < ui.npairs; ++n, ++gp) {  // gp counts the loads issued
-            if (!load_pair<kD, kKStages>(g, ui, n, gp, &maps.k, s.k, s.k_full, s.k_empty,
+            if (!load_pair<kD, kKStages>(g, ui, n, gp, &maps.k, s.k, s.k_full, s.s_full,
                                          abort_flag, lim)) {
               ok = false;
               break;
@@ -315,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, g.head0 + ui.h, row0);
           ++nq;
           for (int n = 0; n < ui.npairs; ++n, ++gp) {  // gp counts the loads issued
-            if (!load_pair<kD, kVStages>(g, ui, n, gp, &maps.v, s.v, s.v_full, s.v_empty,
+            if (!load_pair<kD, kVStages>(g, ui, n, gp, &maps.v, s.v, s.v_full, s.pv_done,
                                          abort_flag, lim)) {
               ok = false;
               break;
@@ -365,7 +372,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                        db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), C::idesc_s, kk ? 1u : 0u);
             }
             mma_commit(&s.s_full[b]);
-            mma_commit(&s.k_empty[ks]);
             if (n == np - 1) mma_commit(&s.q_empty);
           }
           ++active;
@@ -404,7 +410,6 @@ __global__ void __launch_bounds__(kThreads, 1)
               mma_bf16_ts(tmem + kColO, tmem + kColP + 64 * (uint32_t)(gp & 1) + 8 * kk,
                           db0 + kk * (2048 >> 4), C::idesc_o, (n == 0 && kk == 0) ? 0u : 1u);
             mma_commit(&s.pv_done[gp & 1]);
-            mma_commit(&s.v_empty[vs]);
             if (n == np - 1) mma_commit(&s.o_full);
           }
           ++active;
