@@ -74,8 +74,8 @@ constexpr int kSoftmaxThreads = 256;  // both softmax warpgroups
 constexpr int kWgThreads = 128;       // one softmax warpgroup
 constexpr int kTeardownBar = 5;       // named barrier of all threads before TMEM is released
 constexpr int kLaunchRegs = 168;      // 65536 / 384, rounded down to a multiple of 8
-constexpr int kProducerRegs = 56;
-constexpr int kSoftmaxRegs = 224;
+constexpr int kProducerRegs = 72;
+constexpr int kSoftmaxRegs = 216;
 static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kThreads * kLaunchRegs,
               "register split exceeds the launch allocation");
 constexpr float kShiftSlack = 8.f;  // log2 units: P <= 256 between shift updates
@@ -102,20 +102,21 @@ template <int kD>
 struct alignas(1024) SmemLayout {
   uint8_t k[kKStages][Cfg<kD>::kPairBytes];
   uint8_t v[kVStages][Cfg<kD>::kPairBytes];
-  uint8_t q[Cfg<kD>::kQBytes];
+  uint8_t q[2][Cfg<kD>::kQBytes];  // query tiles of consecutive units alternate buffers
   uint64_t k_full[kKStages];  // a K pair landed (TMA -> S issuer)
   uint64_t v_full[kVStages];  // a V pair landed (TMA -> PV issuer)
   uint64_t s_full[2], s_empty[2];  // s_full[b]: S of a step in buffer b (also frees K stage b)
   uint64_t p_full[2];   // P of a step written to TMEM buffer (step & 1) (softmax -> MMA)
   uint64_t pv_done[2];  // that step's PV MMAs complete: its P buffer and V stage free, O current
-  uint64_t q_full;    // the unit's Q loaded (TMA -> MMA)
-  uint64_t q_empty;   // the unit's last S MMA complete: Q may be overwritten (MMA -> producer)
+  uint64_t q_full[2];   // a unit's Q loaded into buffer (unit & 1) (TMA -> MMA)
+  uint64_t q_empty[2];  // that unit's last S MMA complete: the buffer may be refilled
   uint64_t o_full;    // the unit's last PV complete (MMA -> softmax)
   uint64_t o_empty;   // O read by the epilogue (softmax -> MMA)
   uint64_t drain[2];  // all MMAs of the S issuer / the PV issuer complete
   uint64_t m_ready[2];      // shift of a step (parity b) published by warpgroup b
   uint64_t unit_full[kUnitRing], unit_empty[kUnitRing];  // the unit queue's ring
   int unit[kUnitRing];      // unit index, or -1 once the queue is exhausted
+  int ucnt[kUnitRing];      // its kv_cnt entry as read from global memory
   float mrow[2][64];        // [step & 1][row]: that shift
   float xsum[2][2][4][16];  // [unit & 1][warpgroup][warp % 4][row]: running sums, end of a unit
   float xm[2][2][4][16];    // [unit & 1][warpgroup][warp % 4][row]: the shift they are relative to
@@ -133,13 +134,17 @@ struct UnitInfo {
   const int32_t* list;
 };
 
-__device__ __forceinline__ UnitInfo unit_info(const Geo& g, const AttnArgs& a, int u) {
+// kv_cnt entry of unit u (one global load; the queue reader publishes it with the unit).
+__device__ __forceinline__ int unit_count(const AttnArgs& a, int u) {
+  return a.kv_cnt[u];  // units are numbered (b, h, i) row-major, like kv_cnt
+}
+
+__device__ __forceinline__ UnitInfo unit_info(const Geo& g, const AttnArgs& a, int u, int c) {
   UnitInfo r;
   r.i = u % g.nT;
   const int bh = u / g.nT;
   r.h = bh % g.heads;
   r.b = bh / g.heads;
-  const int c = a.kv_cnt[(long)bh * g.nT + r.i];
   r.over = c > a.kmax;
   r.under = c < 0;
   r.cnt = r.under ? 0 : (r.over ? a.kmax : c);
@@ -161,17 +166,19 @@ __device__ __forceinline__ void fail(SmemLayout<kD>& s, int32_t* status) {
   report(status, T3D_DEV_TIMEOUT);
 }
 
-// Next unit from the ring (every reader calls it once per unit, in the same order): the unit index,
-// or -1 when the queue is exhausted or the wait gave up (then `ok` is cleared).
+// Next unit from the ring (every reader calls it once per unit, in the same order): the unit index
+// and its kv_cnt entry, or -1 when the queue is exhausted or the wait gave up (then `ok` is
+// cleared).
 template <int kD>
 __device__ __forceinline__ int take_unit(SmemLayout<kD>& s, long& nu, volatile int* abort_flag,
-                                         long long lim, bool& ok) {
+                                         long long lim, bool& ok, int& cnt) {
   const int slot = (int)(nu % kUnitRing);
   if (!mbar_wait(&s.unit_full[slot], (uint32_t)((nu / kUnitRing) & 1), abort_flag, lim)) {
     ok = false;
     return -1;
   }
   const int u = s.unit[slot];
+  cnt = s.ucnt[slot];
   mbar_arrive(&s.unit_empty[slot]);
   ++nu;
   return u;
@@ -192,8 +199,8 @@ __device__ __forceinline__ bool load_pair(const Geo& g, const UnitInfo& ui, int 
                                           uint64_t* done, volatile int* abort_flag, long long lim) {
   static_assert(kStages == 2, "a stage is step gp's S / P buffer");
   const int st = (int)(gp % kStages);
+  int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);  // read while waiting
   if (!mbar_wait(&done[st], (uint32_t)(((gp / kStages) & 1) ^ 1), abort_flag, lim)) return false;
-  int ja = list_tile(g, ui, 2 * n), jb = list_tile(g, ui, 2 * n + 1);
   if (ja < 0) ja = 0;  // masked in the softmax; any finite tile will do
   if (jb < 0) jb = ja;
   mbar_expect_tx(&full[st], Cfg<kD>::kPairBytes);
@@ -239,8 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.unit_full[t], 1);
       mbar_init(&s.unit_empty[t], kUnitReaders);
     }
-    mbar_init(&s.q_full, 1);
-    mbar_init(&s.q_empty, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s.q_full[t], 1);
+      mbar_init(&s.q_empty[t], 1);
+    }
     mbar_init(&s.o_full, 1);
     mbar_init(&s.o_empty, kSoftmaxThreads);
     mbar_init(&s.drain[0], 1);
@@ -263,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   // Registers move from the producer / issuer warpgroup to the softmax warpgroups: 384 threads
-  // launch with 168 each; 128 x 56 + 256 x 224 is the same total. The two sides never share code
+  // launch with 168 each; 128 x 72 + 256 x 216 is the same total. The two sides never share code
   // after the split (each ends with its own arrival at the teardown barrier).
   if (warp < 4) {
     regs_dec<kProducerRegs>();
@@ -274,6 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         long nu = 0, gp = 0;
         bool ok = true;
         int cur = (int)atomicAdd(next_unit, 1u);
+        int cur_cnt = cur < total_units ? unit_count(a, cur) : 0;
         while (ok) {
           const int slot = (int)(nu % kUnitRing);
           if (!mbar_wait(&s.unit_empty[slot], (uint32_t)(((nu / kUnitRing) & 1) ^ 1), abort_flag,
@@ -283,20 +293,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const int u = cur < total_units ? cur : -1;
           s.unit[slot] = u;
+          s.ucnt[slot] = cur_cnt;
           mbar_arrive(&s.unit_full[slot]);
           ++nu;
           if (u < 0) break;
-          // The next index is fetched now and used after this unit's loads, hiding its latency.
+          // The next index (and then its count) is fetched now and used after this unit's loads,
+          // hiding both latencies.
           const int nxt = (int)atomicAdd(next_unit, 1u);
-          const UnitInfo ui = unit_info(g, a, u);
+          const UnitInfo ui = unit_info(g, a, u, cur_cnt);
+          int nxt_cnt = 0;
           for (int n = 0; n < ui.npairs; ++n, ++gp) {  // gp counts the loads issued
             if (!load_pair<kD, kKStages>(g, ui, n, gp, &maps.k, s.k, s.k_full, s.s_full,
                                          abort_flag, lim)) {
               ok = false;
               break;
             }
+            if (n == 0 && nxt < total_units) nxt_cnt = unit_count(a, nxt);
           }
+          if (ui.npairs == 0 && nxt < total_units) nxt_cnt = unit_count(a, nxt);
           cur = nxt;
+          cur_cnt = nxt_cnt;
         }
         if (!ok) fail(s, a.dev_status);
         drain_ring<kKStages>(s.k_full, gp);
@@ -308,18 +324,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         int nq = 0;  // query tiles loaded
         bool ok = true;
         while (ok) {
-          const int u = take_unit(s, nu, abort_flag, lim, ok);
+          int cnt = 0;
+          const int u = take_unit(s, nu, abort_flag, lim, ok, cnt);
           if (u < 0) break;
-          const UnitInfo ui = unit_info(g, a, u);
+          const UnitInfo ui = unit_info(g, a, u, cnt);
           if (ui.npairs == 0) continue;
-          if (!mbar_wait(&s.q_empty, (uint32_t)((nq & 1) ^ 1), abort_flag, lim)) {
+          // Q buffer nq & 1 is free once the last S of the unit two back has completed, so a
+          // unit's query tile loads while the previous unit is still running.
+          const int qb = nq & 1;
+          if (!mbar_wait(&s.q_empty[qb], (uint32_t)(((nq >> 1) & 1) ^ 1), abort_flag, lim)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&s.q_full, C::kQBytes);
+          mbar_expect_tx(&s.q_full[qb], C::kQBytes);
           const int row0 = ui.b * g.Lp + ui.i * kTileElems;
           for (int hh = 0; hh < C::kHalves; ++hh)
-            tma_load_3d(s.q + hh * kTileBytes, &maps.q, &s.q_full, 64 * hh, g.head0 + ui.h, row0);
+            tma_load_3d(s.q[qb] + hh * kTileBytes, &maps.q, &s.q_full[qb], 64 * hh,
+                        g.head0 + ui.h, row0);
           ++nq;
           for (int n = 0; n < ui.npairs; ++n, ++gp) {  // gp counts the loads issued
             if (!load_pair<kD, kVStages>(g, ui, n, gp, &maps.v, s.v, s.v_full, s.pv_done,
@@ -331,7 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) fail(s, a.dev_status);
         drain_ring<kVStages>(s.v_full, gp);
-        if (nq > 0) mbar_wait(&s.q_full, (uint32_t)((nq - 1) & 1), nullptr);
+        for (int t = nq - 2; t < nq; ++t)
+          if (t >= 0) mbar_wait(&s.q_full[t & 1], (uint32_t)((t >> 1) & 1), nullptr);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------- S issuer
@@ -346,13 +368,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         // Shared-memory descriptors are linear in the start address (bits 0-13 hold address >> 4 and
         // every buffer lies below 256 KB), so each MMA's operand is a base descriptor plus a constant.
         const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
-        const uint64_t dq = sdesc_sw128(smem_u32(s.q), 16, 1024);
+        const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0]), 16, 1024);
         while (ok) {
-          const int u = take_unit(s, nu, abort_flag, lim, ok);
+          int cnt = 0;
+          const int u = take_unit(s, nu, abort_flag, lim, ok, cnt);
           if (u < 0) break;
-          const int np = unit_info(g, a, u).npairs;
+          const int np = unit_info(g, a, u, cnt).npairs;
           if (np == 0) continue;
-          if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag, lim)) { ok = false; break; }
+          const int qb = active & 1;
+          if (!mbar_wait(&s.q_full[qb], (uint32_t)((active >> 1) & 1), abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          const uint64_t dq = dq0 + (uint64_t)(qb * (C::kQBytes >> 4));
           for (int n = 0; n < np; ++n, ++gp) {
             // S(gp) = Q . K_pair^T into S buffer gp & 1, once the softmax has read S(gp - 2).
             const int ks = (int)(gp % kKStages);
@@ -372,7 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                        db0 + ((hh * 2 * kTileBytes + st * 32) >> 4), C::idesc_s, kk ? 1u : 0u);
             }
             mma_commit(&s.s_full[b]);
-            if (n == np - 1) mma_commit(&s.q_empty);
+            if (n == np - 1) mma_commit(&s.q_empty[qb]);
           }
           ++active;
         }
@@ -389,9 +417,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 2 * kTileBytes, 1024);
         while (ok) {
-          const int u = take_unit(s, nu, abort_flag, lim, ok);
+          int cnt = 0;
+          const int u = take_unit(s, nu, abort_flag, lim, ok, cnt);
           if (u < 0) break;
-          const int np = unit_info(g, a, u).npairs;
+          const int np = unit_info(g, a, u, cnt).npairs;
           if (np == 0) continue;
           for (int n = 0; n < np; ++n, ++gp) {
             // O (+)= P . V_pair of step gp; the unit's first PV overwrites O once the epilogue of the
@@ -453,7 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     while (true) {
       bool got = true;
-      const int u = take_unit(s, nu, abort_flag, lim, got);
+      int cnt = 0;
+      const int u = take_unit(s, nu, abort_flag, lim, got, cnt);
       if (!got) give_up();
       // Both warps of a pair leave together (a failed wait in either ends both).
       if (named_bar_or(bar_id, 64, failed)) {
@@ -461,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       if (u < 0) break;
-      const UnitInfo ui = unit_info(g, a, u);
+      const UnitInfo ui = unit_info(g, a, u, cnt);
       if (reporter && (ui.over || ui.under))
         report(a.dev_status, ui.over ? T3D_DEV_OVERFLOW : T3D_DEV_INDEX_RANGE);
       const long row0 = (long)ui.b * g.Lp + (long)ui.i * kTileElems;
@@ -565,8 +595,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (mw1 != n1) l1 = (mw1 == -INFINITY) ? 0.f : l1 * ex2(mw1 - n1);
         mw0 = n0;
         mw1 = n1;
-        // O follows it too: rescale the warp's rows (factor 1 where the shift held) once the
-        // previous step's PV has landed; our own PV of this step is issued only after our P.
+        // P = exp2(x * scale - shift) as bf16 pairs, computed before any wait on the PV MMAs: keys
+        // 8j + 2 t0, + 1 go to P column 4j + t0 (the layout tcgen05.st 16x128b writes).
+        const float ns0 = n0 == -INFINITY ? 0.f : -n0, ns1 = n1 == -INFINITY ? 0.f : -n1;
+        uint32_t pw[2][16];  // keys 0..63, 64..127
+        {
+          float ls0[2] = {0.f, 0.f}, ls1[2] = {0.f, 0.f};
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float p00 = ex2(fmaf(__uint_as_float(v[4 * j]), sl2, ns0));
+            const float p01 = ex2(fmaf(__uint_as_float(v[4 * j + 1]), sl2, ns0));
+            const float p10 = ex2(fmaf(__uint_as_float(v[4 * j + 2]), sl2, ns1));
+            const float p11 = ex2(fmaf(__uint_as_float(v[4 * j + 3]), sl2, ns1));
+            ls0[j & 1] += p00 + p01;
+            ls1[j & 1] += p10 + p11;
+            __nv_bfloat162 q0 = __floats2bfloat162_rn(p00, p01);
+            __nv_bfloat162 q1 = __floats2bfloat162_rn(p10, p11);
+            pw[j >> 3][2 * (j & 7)] = *reinterpret_cast<uint32_t*>(&q0);
+            pw[j >> 3][2 * (j & 7) + 1] = *reinterpret_cast<uint32_t*>(&q1);
+          }
+          l0 += ls0[0] + ls0[1];
+          l1 += ls1[0] + ls1[1];
+        }
+        // Our P buffer is free once the PV of our previous step (two steps back) has landed.
+        if (gs >= 2) {
+          if (!mbar_wait(&s.pv_done[wg], (uint32_t)(((gs - 2) >> 1) & 1), abort_flag, lim))
+            give_up();
+          tc_fence_after();
+        }
+        tmem_st_16x128b_x8(t_p, pw[0]);
+        tmem_st_16x128b_x8(t_p + 32, pw[1]);
+        // O follows the shift too: rescale the warp's rows (factor 1 where the shift held) once the
+        // previous step's PV has landed; our own PV of this step is issued only after this.
         if (n > 0 && __any_sync(0xffffffffu, up0 || up1)) {
           if (!mbar_wait(&s.pv_done[wg ^ 1], (uint32_t)(((gs - 1) >> 1) & 1), abort_flag, lim))
             give_up();
@@ -588,37 +648,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_16x256b_x8(lane_base + kColO + 64 * hc, o);
           }
           tmem_wait_st();
-        }
-        // Our P buffer is free once the PV of our previous step (two steps back) has landed.
-        if (gs >= 2) {
-          if (!mbar_wait(&s.pv_done[wg], (uint32_t)(((gs - 2) >> 1) & 1), abort_flag, lim))
-            give_up();
-          tc_fence_after();
-        }
-        // P = exp2(x * scale - shift) as bf16 pairs: keys 8j + 2 t0, + 1 go to P column 4j + t0
-        // (the layout tcgen05.st 16x128b writes), in two stores of 32 columns.
-        const float ns0 = n0 == -INFINITY ? 0.f : -n0, ns1 = n1 == -INFINITY ? 0.f : -n1;
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t pw[16];
-          float ls0[2] = {0.f, 0.f}, ls1[2] = {0.f, 0.f};
-#pragma unroll
-          for (int jj = 0; jj < 8; ++jj) {
-            const int j = 8 * hh + jj;
-            const float p00 = ex2(fmaf(__uint_as_float(v[4 * j]), sl2, ns0));
-            const float p01 = ex2(fmaf(__uint_as_float(v[4 * j + 1]), sl2, ns0));
-            const float p10 = ex2(fmaf(__uint_as_float(v[4 * j + 2]), sl2, ns1));
-            const float p11 = ex2(fmaf(__uint_as_float(v[4 * j + 3]), sl2, ns1));
-            ls0[jj & 1] += p00 + p01;
-            ls1[jj & 1] += p10 + p11;
-            __nv_bfloat162 q0 = __floats2bfloat162_rn(p00, p01);
-            __nv_bfloat162 q1 = __floats2bfloat162_rn(p10, p11);
-            pw[2 * jj] = *reinterpret_cast<uint32_t*>(&q0);
-            pw[2 * jj + 1] = *reinterpret_cast<uint32_t*>(&q1);
-          }
-          l0 += ls0[0] + ls0[1];
-          l1 += ls1[0] + ls1[1];
-          tmem_st_16x128b_x8(t_p + 32 * hh, pw);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -697,19 +726,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float ia = __shfl_sync(0xffffffffu, i0, 4 * (lane & 7));
         const float ib = __shfl_sync(0xffffffffu, i1, 4 * (lane & 7));
         const float inv = (lane & 15) < 8 ? ia : ib;
+        // All of this warpgroup's O columns come into registers first, so O is released to the
+        // next unit's first PV before the normalisation and the global stores.
+        uint32_t o[kCols / 32][32];
+#pragma unroll
+        for (int c = 0; c < kCols / 32; ++c) tmem_ld32(lane_base + kColO + col0 + 32 * c, o[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&s.o_empty);
 #pragma unroll
         for (int c = 0; c < kCols / 32; ++c) {
           const int cc = col0 + 32 * c;
-          uint32_t o[32];
-          tmem_ld32(lane_base + kColO + cc, o);
-          tmem_wait_ld();
           if (lane < 16) {
             uint4 w4[4];
             uint32_t* w = reinterpret_cast<uint32_t*>(w4);
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              __nv_bfloat162 y = __floats2bfloat162_rn(__uint_as_float(o[2 * e]) * inv,
-                                                       __uint_as_float(o[2 * e + 1]) * inv);
+              __nv_bfloat162 y = __floats2bfloat162_rn(__uint_as_float(o[c][2 * e]) * inv,
+                                                       __uint_as_float(o[c][2 * e + 1]) * inv);
               w[e] = *reinterpret_cast<uint32_t*>(&y);
             }
             // Every output row that takes this row's result; rows past the tile's valid count
@@ -723,8 +757,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        tc_fence_before();
-        mbar_arrive(&s.o_empty);
       }
       ++active;
     }

@@ -53,8 +53,8 @@ def _mass_no_crossing(row, scale, tau, min_k):
     return np.sort(order[:m])
 
 
-def _keys_all_slots(sets_i, vc):
-    parts = [64 * int(j) + np.arange(64) for j in sets_i]
+def _keys_all_slots(sets_i, vc, E=64):
+    parts = [E * int(j) + np.arange(E) for j in sets_i]
     return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
 
 
