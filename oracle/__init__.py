@@ -14,8 +14,9 @@ Modules:
   attention  softmax attention restricted to the kept (query tile, key tile) pairs
   attention_bwd  its gradients with respect to Q, K and V (the backward pass)
   pipeline   the four stages chained, as the hot path runs them
+  packed     packed multi-region sequences (dense segments plus video regions), tiles of 64 or 128
 
 Every function is pinned by a CPU test against something other than itself (closed forms,
 brute force on tiny inputs, invariants, library routines for the dense special case).
 """
-from . import tiling, pool, select, bsa, attention, attention_bwd, pipeline  # noqa: F401
+from . import tiling, pool, select, bsa, attention, attention_bwd, pipeline, packed  # noqa: F401

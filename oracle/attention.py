@@ -21,8 +21,8 @@ import numpy as np
 TILE_ELEMS = 64
 
 
-def _key_rows(sets_i, vc) -> np.ndarray:
-    parts = [TILE_ELEMS * int(j) + np.arange(int(vc[int(j)])) for j in sets_i]
+def _key_rows(sets_i, vc, E: int = TILE_ELEMS) -> np.ndarray:
+    parts = [E * int(j) + np.arange(int(vc[int(j)])) for j in sets_i]
     if not parts:
         return np.zeros(0, dtype=np.int64)
     return np.concatenate(parts)
@@ -45,23 +45,25 @@ def attend_rows(q_rows: np.ndarray, k_rows: np.ndarray, v_rows: np.ndarray, scal
 
 
 def block_sparse_attention(qt, kt, vt, vc, sets, scale: float, keep=None, src=None,
-                           q_tiles=None, return_wsum: bool = False):
-    """Block-sparse attention on padded tile-ordered ``[B, 64*nT, heads, D]`` tensors.
+                           q_tiles=None, return_wsum: bool = False, tile_elems: int = TILE_ELEMS):
+    """Block-sparse attention on padded tile-ordered ``[B, E*nT, heads, D]`` tensors (``E`` =
+    ``tile_elems``: 64, or 128 for the packed sequences' large tile).
 
     ``sets[b][h][i]``: kept key tiles of query tile ``i``. ``keep``/``src`` (``[B, heads, nT, 64]``)
     switch on the pruned-query variant: only kept rows attend, pruned rows copy ``src``'s output.
     ``q_tiles``: optional list of ``(b, h, i)`` to compute (other rows stay 0), for sampled checks.
     Returns fp64 ``[B, 64*nT, heads, D]`` (and the per-row weight sums if asked)."""
     B, Lp, nh, D = qt.shape
-    nT = Lp // TILE_ELEMS
+    E = int(tile_elems)
+    nT = Lp // E
     out = np.zeros((B, Lp, nh, D), dtype=np.float64)
     wsum = np.zeros((B, Lp, nh), dtype=np.float64)
     todo = q_tiles if q_tiles is not None else [(b, h, i) for b in range(B) for h in range(nh)
                                                  for i in range(nT)]
     for (b, h, i) in todo:
-        rows_k = _key_rows(sets[b][h][i], vc)
+        rows_k = _key_rows(sets[b][h][i], vc, E)
         n_q = int(vc[i])
-        base = TILE_ELEMS * i
+        base = E * i
         if rows_k.size == 0:
             continue
         if keep is None:

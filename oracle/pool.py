@@ -13,14 +13,16 @@ import numpy as np
 TILE_ELEMS = 64
 
 
-def tile_mean_pool(y: np.ndarray, vc: np.ndarray) -> np.ndarray:
-    """Padded tile order ``[B, 64*nT, heads, D]`` -> pooled ``[B, heads, nT, D]`` (fp64)."""
+def tile_mean_pool(y: np.ndarray, vc: np.ndarray, tile_elems: int = TILE_ELEMS) -> np.ndarray:
+    """Padded tile order ``[B, E*nT, heads, D]`` -> pooled ``[B, heads, nT, D]`` (fp64); ``E`` =
+    ``tile_elems`` rows per tile (64, or 128 for the packed sequences' large tile)."""
     B, Lp, nh, D = y.shape
-    nT = Lp // TILE_ELEMS
-    assert nT * TILE_ELEMS == Lp and len(vc) == nT
+    E = int(tile_elems)
+    nT = Lp // E
+    assert nT * E == Lp and len(vc) == nT
     out = np.zeros((B, nh, nT, D), dtype=np.float64)
     for i in range(nT):
         n = int(vc[i])
-        rows = y[:, TILE_ELEMS * i:TILE_ELEMS * i + n].astype(np.float64)  # [B, n, heads, D]
+        rows = y[:, E * i:E * i + n].astype(np.float64)  # [B, n, heads, D]
         out[:, :, i, :] = rows.sum(axis=1) / n
     return out
