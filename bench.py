@@ -568,13 +568,153 @@ def run_backward(args, w):
     return 0
 
 
+def packed_oracle_sample(w, geo_ref, q, k, v, heads, q_tiles=None):
+    """The CPU oracle's packed path for the given heads (scatter, pooling, scores, per-region
+    selection, attention for the first ``q_tiles`` query tiles or all). Returns (seconds, flops,
+    pairs)."""
+    import torch
+
+    from oracle import attention, packed, pool, select
+
+    E = geo_ref["E"]
+    t0 = time.perf_counter()
+    pairs = 0
+    rates = packed.span_keep_rates(len(geo_ref["spans"]), w.sparsity, w.ref_keep_rate, True)
+    nT = len(geo_ref["vc"])
+    for b in range(w.B):
+        for h in heads:
+            sl = lambda x: x[b:b + 1, :, h:h + 1].to(torch.float64).numpy()  # noqa: E731
+            qt, kt, vt = (packed.scatter(sl(x), geo_ref) for x in (q, k, v))
+            pq, pk = (pool.tile_mean_pool(x, geo_ref["vc"], E) for x in (qt, kt))
+            sets = packed.select(select.tile_scores(pq, pk), geo_ref, rates)
+            n = nT if q_tiles is None else min(q_tiles, nT)
+            attention.block_sparse_attention(qt, kt, vt, geo_ref["vc"], sets, w.D ** -0.5,
+                                             q_tiles=[(0, 0, i) for i in range(n)], tile_elems=E)
+            pairs += sum(len(sets[0][0][i]) for i in range(n))
+    sec = time.perf_counter() - t0
+    return sec, pairs * 4 * E * E * w.D, pairs
+
+
+def run_packed(args, w):
+    """A packed multi-region sequence (dense prefix, reference and generated video regions) on one
+    GPU: scatter, pooling, per-region selection, attention and gather, timed per stage."""
+    import torch
+
+    from block_sparse_video_tile3d_b200 import packed as P
+    from block_sparse_video_tile3d_b200 import workloads
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("the packed workload runs on one GPU")
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    q, k, v = workloads.make_packed_qkv(w)
+    mod = P.PackedTileSparseAttention(list(w.segments), w.heads, w.D, tile_size=w.tile_size,
+                                      sparsity=w.sparsity, ref_keep_rate=w.ref_keep_rate, device=dev)
+    g = mod.geo
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    od = torch.empty_like(qd)
+    stages = mod.stages(qd, kd, vd, od)
+    names = [n for n, _ in stages]
+    sampler = ClockSampler(0)
+    for _ in range(max(args.warmup, 3)):
+        for _, launch in stages:
+            launch()
+    torch.cuda.synchronize()
+    pairs = int(mod.kv_cnt.sum().item())
+    E = g.E
+    flops = pairs * 4 * E * E * w.D
+    nst = len(stages)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(nst + 1)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for st in range(args.steps):
+        ev[st][0].record()
+        for j, (_, launch) in enumerate(stages):
+            launch()
+            ev[st][j + 1].record()
+    torch.cuda.synchronize()
+    total_ms = ev[0][0].elapsed_time(ev[-1][-1])
+    stage_ms = {n: sum(ev[st][j].elapsed_time(ev[st][j + 1]) for st in range(args.steps)) / args.steps
+                for j, n in enumerate(names)}
+    clocks = sampler.stop()
+    ms_step = total_ms / args.steps
+    status = int(mod.status.item())
+    # end to end: pinned host inputs in, output back, every step inside the timed region
+    hosts = tuple(x.pin_memory() for x in (q, k, v))
+    oh = torch.empty(od.shape, dtype=od.dtype).pin_memory()
+    ref = od.cpu()
+    e2e_steps = max(4, min(args.steps, 20))
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(e2e_steps):
+        for dst, src in zip((qd, kd, vd), hosts):
+            dst.copy_(src, non_blocking=True)
+        mod(qd, kd, vd, od)
+        oh.copy_(od, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    peaks = _peaks()
+    attn_ms = stage_ms["attention"]
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    row_bytes = w.heads * w.D * 2
+    rows, buf = g.rows * w.B, g.buffer_rows * w.B
+    byt = {"scatter_q": (rows + buf) * row_bytes, "scatter_k": (rows + buf) * row_bytes,
+           "scatter_v": (rows + buf) * row_bytes, "pool_q": buf * row_bytes,
+           "pool_k": buf * row_bytes, "gather": (rows + buf) * row_bytes}
+    stage_report = {n: {"ms": round(stage_ms[n], 4),
+                        "gbs": round(byt[n] / (stage_ms[n] * 1e-3) / 1e9, 1) if n in byt else None,
+                        "bytes": byt.get(n)} for n in names}
+    line = {
+        "metric": METRIC.replace("28,672 tok×12 heads", f"packed {g.rows:,} tok×{w.heads} heads"),
+        "value": flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOPS",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "ms_per_call": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": (f"{w.name}: B={w.B}, heads={w.heads}, D={w.D}, segments "
+                                f"{list(w.segments)} (dense rows / region token grids), tile "
+                                f"{E} ({'x'.join(map(str, g.tile_shape))}), {g.n_tiles} tiles "
+                                f"({g.n_prefix} dense), generated keep {1 - w.sparsity:g}, "
+                                f"reference keep {w.ref_keep_rate:g}"),
+                   "kept_pairs": pairs, "metric_flops": f"4 * {E} * {E} * D per kept tile pair",
+                   "kept_block_gflop": flops / 1e9,
+                   "l2": f"no flush: packed Q/K/V of {3 * rows * row_bytes / 1e6:.0f} MB exceed "
+                         "the 126 MB L2"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                     "kernel": "block_sparse_attn_fwd_packed",
+                     "peak_source": f"{peaks['source']} bf16 dense (burst)", "ms_per_launch": attn_ms},
+        "stages": stage_report,
+        "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+                "steps": e2e_steps, "output_matches_device_run": bool(torch.equal(oh, ref)),
+                "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
+                "d2h_bytes_per_step": od.numel() * od.element_size()},
+        "gpu_launches": args.steps * (nst + 1),  # the attention call launches a list-rewrite kernel too
+        "device_status": status,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        from oracle import packed as opk
+        ref_geo = opk.packed_geometry(list(w.segments), P.TILE_SHAPES[E])
+        sec, fl, np_ = packed_oracle_sample(w, ref_geo, q, k, v, [0], max(1, g.n_tiles // 8))
+        line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": _cores(),
+                                "kind": "oracle",
+                                "sample": (f"fp64 numpy oracle, packed path for head 0 of {w.heads}, "
+                                           f"attention of the first {max(1, g.n_tiles // 8)} of "
+                                           f"{g.n_tiles} query tiles: {np_:,} kept pairs in "
+                                           f"{sec:.1f} s")}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="small",
-                    help="workload: tiny, small, large, bsa, ragged_sliding, ragged_random")
+                    help="workload: tiny, small, large, bsa, ragged_sliding, ragged_random, "
+                         "packed, packed_tiny")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--pass", dest="which", default="forward", choices=["forward", "backward"],
                     help="forward: the whole hot path (the benchmark line); backward: the "
@@ -588,7 +728,13 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    from block_sparse_video_tile3d_b200.workloads import WORKLOADS
+    from block_sparse_video_tile3d_b200.workloads import PACKED_WORKLOADS, WORKLOADS
+    if args.config in PACKED_WORKLOADS:
+        if args.impl == "reference" or args.which == "backward":
+            print(json.dumps({"impl": args.impl, "unavailable": "the packed workload has the forward "
+                              "benchmark of this library only"}))
+            return 0
+        return run_packed(args, PACKED_WORKLOADS[args.config])
     w = WORKLOADS[args.config]
     if args.impl == "reference":
         return run_reference(args, w)

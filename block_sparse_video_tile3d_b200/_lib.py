@@ -1,4 +1,5 @@
-"""ctypes binding of libtile3d.so (the C ABI declared in include/tile3d.h).
+"""ctypes binding of libtile3d.so (the C ABI declared in include/tile3d.h and
+include/tile3d_packed.h).
 
 Argument marshalling only. The library must have been built in-tree
 (``python -m block_sparse_video_tile3d_b200.build``); importing this module without it raises
@@ -26,11 +27,33 @@ class Geom(ctypes.Structure):
                 ("head0", ctypes.c_int)]
 
 
+class Segment(ctypes.Structure):
+    """``t3d_segment``: a dense run (rows > 0) or a video region of t x h x w tokens (rows = 0)."""
+    _fields_ = [("rows", ctypes.c_int), ("t", ctypes.c_int), ("h", ctypes.c_int), ("w", ctypes.c_int)]
+
+
+class PackedLayout(ctypes.Structure):
+    """``t3d_packed_layout``."""
+    _fields_ = [("n_tiles", ctypes.c_int), ("rows", ctypes.c_int), ("n_prefix", ctypes.c_int),
+                ("n_regions", ctypes.c_int)]
+
+
+class Packed(ctypes.Structure):
+    """``t3d_packed``: a packed tile buffer as the device calls see it."""
+    _fields_ = [("B", ctypes.c_int), ("heads", ctypes.c_int), ("D", ctypes.c_int),
+                ("heads_total", ctypes.c_int), ("head0", ctypes.c_int), ("tile_elems", ctypes.c_int),
+                ("n_tiles", ctypes.c_int), ("rows", ctypes.c_int), ("slot_row", ctypes.c_void_p),
+                ("vc", ctypes.c_void_p)]
+
+
+T3D_PACKED_EXEMPT, T3D_PACKED_COMPETE, T3D_PACKED_DENSE = 0, 1, 2
+
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _F = ctypes.c_float
 _S = ctypes.c_size_t
 _G = ctypes.POINTER(Geom)
+_PK = ctypes.POINTER(Packed)
 
 # name -> (restype, argtypes), in the order of include/tile3d.h, then include/tile3d_testing.h
 SIGNATURES = {
@@ -57,6 +80,17 @@ SIGNATURES = {
     "block_sparse_attn_bwd_workspace_size": (_S, [_G, _I]),
     "block_sparse_attn_fwd_noalloc": (_I, [_G, _P, _P, _P, _P, _P, _P, _I, _P, _P, _F, _I, _I,
                                            _P, _P]),
+    # include/tile3d_packed.h
+    "t3d_packed_geometry": (_I, [ctypes.POINTER(Segment), _I, _I, _I, _I,
+                                 ctypes.POINTER(PackedLayout), _P, _P, _P]),
+    "tile3d_scatter_packed": (_I, [_PK, _P, _P, _P]),
+    "tile3d_gather_packed": (_I, [_PK, _P, _P, _P]),
+    "tile_pool_packed": (_I, [_PK, _P, _P, _P]),
+    "tile_select_packed_capacity": (_I, [_I, _I, _I, _I, _P, _P, ctypes.POINTER(_I)]),
+    "tile_select_packed": (_I, [_PK, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _S, _P, _P]),
+    "tile_select_packed_workspace_size": (_S, [_PK]),
+    "block_sparse_attn_fwd_packed": (_I, [_PK, _P, _P, _P, _P, _P, _P, _I, _F, _P, _S, _P, _P]),
+    "block_sparse_attn_packed_workspace_size": (_S, [_PK, _I]),
     # include/tile3d_testing.h
     "t3d_testing_set_wait_cycles": (_I, [ctypes.c_longlong]),
 }

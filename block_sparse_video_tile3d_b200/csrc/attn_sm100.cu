@@ -257,7 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     s.abort = 0;
     fence_mbar_init();
   }
-  for (int t = threadIdx.x; t < g.nT; t += kThreads) s.vc[t] = (uint8_t)tile_valid_count(g, t);
+  for (int t = threadIdx.x; t < g.nT; t += kThreads)
+    s.vc[t] = a.vc_tab != nullptr ? a.vc_tab[t] : (uint8_t)tile_valid_count(g, t);
   if (warp == 0 && lane == 0) {
     tma_prefetch(&maps.q);
     tma_prefetch(&maps.k);

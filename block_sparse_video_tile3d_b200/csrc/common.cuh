@@ -12,6 +12,7 @@
 #include <stdint.h>
 
 #include "tile3d.h"
+#include "tile3d_packed.h"
 
 namespace t3d {
 

@@ -52,6 +52,7 @@ struct AttnArgs {
   int32_t* dev_status;
   long long wait_cycles;  // limit of each pipeline wait, in clock cycles
   float* lse;             // NULL, or [B, heads, Lp]: each query row's log-sum-exp (natural log)
+  const uint8_t* vc_tab;  // NULL, or the valid rows of every 64-row unit (packed sequences)
 };
 
 // Backward pass (attn_bwd.cu): gradients of block_sparse_attn_fwd for an output gradient.
@@ -88,5 +89,34 @@ cudaError_t launch_attn(const Geo& g, const AttnArgs& a, cudaStream_t s);
 // current device (looked up on the first call per device).
 constexpr size_t kNoAllocScratchBytes = 256;
 cudaError_t noalloc_scratch(void** ptr);
+
+// Packed multi-region sequences (packed.cu): a padded buffer of n_tiles tiles of E = 64 or 128
+// rows whose slot map (packed row of every slot, -1 for a pad) and valid counts are device arrays.
+struct PackedGeo {
+  int B, heads, D, heads_total, head0;
+  int E, n_tiles, rows;  // rows per tile, tiles, packed rows per batch entry
+  int row_chunks, row_stride, row_off;  // as in Geo
+  const int32_t* slot_row;  // [n_tiles * E]
+  const int32_t* vc;        // [n_tiles]
+};
+cudaError_t launch_scatter_packed(const PackedGeo& p, const void* x, void* y, cudaStream_t s);
+cudaError_t launch_gather_packed(const PackedGeo& p, const void* y, void* x, cudaStream_t s);
+cudaError_t launch_pool_packed(const PackedGeo& p, const void* y, float* pooled, cudaStream_t s);
+size_t attn_packed_workspace_bytes(const PackedGeo& p, int kmax);
+cudaError_t launch_attn_packed(const PackedGeo& p, const AttnArgs& a, cudaStream_t s);
+// The 64-row-unit geometry the attention kernel runs a packed buffer with.
+Geo packed_attn_geo(const PackedGeo& p);
+
+// Per-region selection of a packed sequence (select.cu), scores as launch_select_topk. mode:
+// T3D_PACKED_EXEMPT / _COMPETE / _DENSE; k[r] tiles of region r (tiles lo[r] .. hi[r] - 1) are kept
+// per query tile past the n_prefix dense tiles (exempt), k_total of all tiles (compete).
+constexpr int kMaxRegions = 16;
+struct SpanSpec {
+  int mode, n_prefix, n_regions, k_total;
+  int lo[kMaxRegions], hi[kMaxRegions], k[kMaxRegions];
+};
+cudaError_t launch_select_spans(const Geo& g, const float* pq, const float* pk, const SpanSpec& sp,
+                                int kmax, int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
+                                cudaStream_t s);
 
 }  // namespace t3d

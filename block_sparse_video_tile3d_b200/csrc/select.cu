@@ -593,6 +593,44 @@ __global__ void __launch_bounds__(kSelThreads) mass_rows_kernel(Geo g, const flo
   }
 }
 
+// One warp per query tile of a packed buffer: its kept tiles by region (tile3d_packed.h).
+// Exempt mode: prefix tiles for every row, everything for a prefix row, else the top k[r] of each
+// region's stretch of the score row, shifted to buffer indices; regions follow the prefix in tile
+// order, so the concatenation is ascending. Compete mode: one top-k over the row.
+__global__ void __launch_bounds__(kSelThreads) spans_rows_kernel(Geo g, const float* __restrict__ S,
+                                                                 int ldS, SpanSpec sp, int kmax,
+                                                                 int32_t* __restrict__ kv_idx,
+                                                                 int32_t* __restrict__ kv_cnt) {
+  __shared__ int hist[kSelThreads / 32][256];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long rows = (long)g.B * g.heads * g.nT;
+  for (long r = (long)blockIdx.x * (kSelThreads / 32) + w; r < rows;
+       r += (long)gridDim.x * (kSelThreads / 32)) {
+    const int i = (int)(r % g.nT);
+    const float* row = S + r * ldS;
+    int32_t* out = kv_idx + r * kmax;
+    int cnt;
+    if (sp.mode == T3D_PACKED_DENSE || (sp.mode == T3D_PACKED_EXEMPT && i < sp.n_prefix)) {
+      for (int j = lane; j < g.nT; j += 32) out[j] = j;
+      cnt = g.nT;
+    } else if (sp.mode == T3D_PACKED_COMPETE) {
+      cnt = select_topk_any(row, g.nT, sp.k_total, out, hist[w]);
+    } else {
+      for (int j = lane; j < sp.n_prefix; j += 32) out[j] = j;
+      cnt = sp.n_prefix;
+      for (int q = 0; q < sp.n_regions; ++q) {
+        const int lo = sp.lo[q];
+        const int c = select_topk_any(row + lo, sp.hi[q] - lo, sp.k[q], out + cnt, hist[w]);
+        __syncwarp();
+        for (int j = lane; j < c; j += 32) out[cnt + j] += lo;
+        cnt += c;
+      }
+    }
+    if (lane == 0) kv_cnt[r] = cnt;
+    __syncwarp();
+  }
+}
+
 // One warp per row of the block map.
 __global__ void mask_to_index_kernel(Geo g, const uint8_t* __restrict__ mask, int kmax,
                                      int32_t* __restrict__ kv_idx, int32_t* __restrict__ kv_cnt,
@@ -878,6 +916,17 @@ cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, f
   if (e != cudaSuccess) return e;
   mass_rows_kernel<<<sel_grid(g), kSelThreads, smem, s>>>(g, S, ldS, scale, mass, min_k, kmax,
                                                           kv_idx, kv_cnt, dev_status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_spans(const Geo& g, const float* pq, const float* pk, const SpanSpec& sp,
+                                int kmax, int32_t* kv_idx, int32_t* kv_cnt, void* workspace,
+                                cudaStream_t s) {
+  float* S = nullptr;
+  int ldS = 0;
+  cudaError_t e = launch_scores(g, pq, pk, workspace, &S, &ldS, s);
+  if (e != cudaSuccess) return e;
+  spans_rows_kernel<<<sel_grid(g), kSelThreads, 0, s>>>(g, S, ldS, sp, kmax, kv_idx, kv_cnt);
   return cudaGetLastError();
 }
 

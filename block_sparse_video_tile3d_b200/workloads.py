@@ -158,3 +158,42 @@ def block_mask(w: Workload) -> torch.Tensor:
     if w.mask == "random":
         return random_block_mask(w.B, w.heads, w.nT, w.density, w.seed)
     raise ValueError(f"workload {w.name} has no fixed block mask")
+
+
+# ------------------------------------------------------------------ packed multi-region sequences
+
+@dataclasses.dataclass(frozen=True)
+class PackedWorkload:
+    """A packed sequence (video_sparse_attn_h3 page, build()): dense segments (row counts) and
+    video regions (token grids, patch 1), the last region the generated video."""
+    name: str
+    B: int
+    heads: int
+    D: int
+    segments: tuple
+    tile_size: int
+    sparsity: float
+    ref_keep_rate: float
+    seed: int
+
+
+PACKED_WORKLOADS = {
+    # a text prefix, one reference clip at half the frames and the generated clip of the small
+    # layer's grid, with 128-token tiles
+    "packed": PackedWorkload("packed", 1, 12, 128, (512, (8, 32, 56), (16, 32, 56)), 128, 0.875,
+                             0.25, 1005),
+    "packed_tiny": PackedWorkload("packed_tiny", 1, 2, 64, (37, (4, 8, 8), (5, 8, 12)), 128, 0.75,
+                                  0.5, 1006),
+}
+
+
+def packed_rows(w: PackedWorkload) -> int:
+    return sum(s if isinstance(s, int) else s[0] * s[1] * s[2] for s in w.segments)
+
+
+def make_packed_qkv(w: PackedWorkload, seed: int | None = None):
+    """Q, K, V as bf16 CPU tensors ``[B, rows, heads, D]`` in packed order: i.i.d. N(0, 1) (the
+    region structure only sets where the tiles lie)."""
+    g = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    shape = (w.B, packed_rows(w), w.heads, w.D)
+    return tuple(torch.randn(shape, generator=g).to(torch.bfloat16) for _ in range(3))

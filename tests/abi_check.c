@@ -5,6 +5,7 @@
 #include <stdlib.h>
 
 #include "tile3d.h"
+#include "tile3d_packed.h"
 
 int main(int argc, char** argv) {
   if (argc != 7) {
