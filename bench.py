@@ -662,9 +662,14 @@ def run_packed(args, w):
     byt = {"scatter_q": (rows + buf) * row_bytes, "scatter_k": (rows + buf) * row_bytes,
            "scatter_v": (rows + buf) * row_bytes, "pool_q": buf * row_bytes,
            "pool_k": buf * row_bytes, "gather": (rows + buf) * row_bytes}
+    kmax = mod.kv_idx.shape[-1]
+    byt["select"] = (2 * w.B * w.heads * g.n_tiles * w.D * 4
+                     + w.B * w.heads * g.n_tiles * (kmax + 1) * 4)
     stage_report = {n: {"ms": round(stage_ms[n], 4),
                         "gbs": round(byt[n] / (stage_ms[n] * 1e-3) / 1e9, 1) if n in byt else None,
                         "bytes": byt.get(n)} for n in names}
+    coarse_ms = sum(stage_ms[n] for n in names if n != "attention")
+    coarse_bytes = sum(byt[n] for n in names if n != "attention")
     line = {
         "metric": METRIC.replace("28,672 tok×12 heads", f"packed {g.rows:,} tok×{w.heads} heads"),
         "value": flops / (ms_step * 1e-3) / 1e12, "unit": "TFLOPS",
@@ -684,6 +689,10 @@ def run_packed(args, w):
                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
                      "kernel": "block_sparse_attn_fwd_packed",
                      "peak_source": f"{peaks['source']} bf16 dense (burst)", "ms_per_launch": attn_ms},
+        "coarse_and_tiling": {"ms": coarse_ms, "bytes": coarse_bytes,
+                              "gbs": coarse_bytes / (coarse_ms * 1e-3) / 1e9,
+                              "frac_hbm": coarse_bytes / (coarse_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                              "hbm_peak_gbs": peaks["hbm_gbs"]},
         "stages": stage_report,
         "e2e": {"value": flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
                 "steps": e2e_steps, "output_matches_device_run": bool(torch.equal(oh, ref)),
@@ -696,13 +705,18 @@ def run_packed(args, w):
     if not args.no_cpu_baseline:
         from oracle import packed as opk
         ref_geo = opk.packed_geometry(list(w.segments), P.TILE_SHAPES[E])
+        # calibrate on a small slice, then size the sample (whole heads, all query tiles) to the
+        # CPU budget
         sec, fl, np_ = packed_oracle_sample(w, ref_geo, q, k, v, [0], max(1, g.n_tiles // 8))
+        per_head = sec * 8
+        nh = int(max(1, min(w.heads, args.cpu_budget // max(per_head, 1e-3))))
+        sec, fl, np_ = packed_oracle_sample(w, ref_geo, q, k, v, list(range(nh)))
         line["cpu_baseline"] = {"value": fl / sec / 1e12, "unit": "TFLOPS", "cores": _cores(),
                                 "kind": "oracle",
-                                "sample": (f"fp64 numpy oracle, packed path for head 0 of {w.heads}, "
-                                           f"attention of the first {max(1, g.n_tiles // 8)} of "
-                                           f"{g.n_tiles} query tiles: {np_:,} kept pairs in "
-                                           f"{sec:.1f} s")}
+                                "sample": (f"fp64 numpy oracle, whole packed path (scatter, pool, "
+                                           f"score, per-region select, attend all {g.n_tiles} "
+                                           f"query tiles) for heads 0..{nh - 1} of {w.heads}: "
+                                           f"{np_:,} kept pairs in {sec:.1f} s")}
     print(json.dumps(line), flush=True)
     return 0
 
