@@ -659,12 +659,12 @@ def run_packed(args, w):
     achieved = flops / (attn_ms * 1e-3) / 1e12
     row_bytes = w.heads * w.D * 2
     rows, buf = g.rows * w.B, g.buffer_rows * w.B
-    byt = {"scatter_q": (rows + buf) * row_bytes, "scatter_k": (rows + buf) * row_bytes,
-           "scatter_v": (rows + buf) * row_bytes, "pool_q": buf * row_bytes,
-           "pool_k": buf * row_bytes, "gather": (rows + buf) * row_bytes}
+    pooled_bytes = w.B * w.heads * g.n_tiles * w.D * 4
+    byt = {"scatter_pool_q": (rows + buf) * row_bytes + pooled_bytes,
+           "scatter_pool_k": (rows + buf) * row_bytes + pooled_bytes,
+           "scatter_v": (rows + buf) * row_bytes, "gather": (rows + buf) * row_bytes}
     kmax = mod.kv_idx.shape[-1]
-    byt["select"] = (2 * w.B * w.heads * g.n_tiles * w.D * 4
-                     + w.B * w.heads * g.n_tiles * (kmax + 1) * 4)
+    byt["select"] = 2 * pooled_bytes + w.B * w.heads * g.n_tiles * (kmax + 1) * 4
     stage_report = {n: {"ms": round(stage_ms[n], 4),
                         "gbs": round(byt[n] / (stage_ms[n] * 1e-3) / 1e9, 1) if n in byt else None,
                         "bytes": byt.get(n)} for n in names}

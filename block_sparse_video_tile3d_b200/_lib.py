@@ -86,6 +86,7 @@ SIGNATURES = {
     "tile3d_scatter_packed": (_I, [_PK, _P, _P, _P]),
     "tile3d_gather_packed": (_I, [_PK, _P, _P, _P]),
     "tile_pool_packed": (_I, [_PK, _P, _P, _P]),
+    "tile3d_scatter_pool_packed": (_I, [_PK, _P, _P, _P, _P]),
     "tile_select_packed_capacity": (_I, [_I, _I, _I, _I, _P, _P, ctypes.POINTER(_I)]),
     "tile_select_packed": (_I, [_PK, _P, _P, _I, _I, _I, _P, _P, _I, _P, _P, _P, _S, _P, _P]),
     "tile_select_packed_workspace_size": (_S, [_PK]),

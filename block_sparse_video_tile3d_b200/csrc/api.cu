@@ -638,6 +638,17 @@ t3d_status tile_pool_packed(const t3d_packed* p, const void* y, float* pooled, t
   return cuda_status(t3d::launch_pool_packed(g, y, pooled, as_stream(stream)), "tile_pool_packed");
 }
 
+t3d_status tile3d_scatter_pool_packed(const t3d_packed* p, const void* x, void* y, float* pooled,
+                                      t3d_stream stream) {
+  t3d::PackedGeo g;
+  T3D_CHECK(check_packed(p, &g));
+  T3D_CHECK(check_ptr(x, "x"));
+  T3D_CHECK(check_ptr(y, "y"));
+  T3D_CHECK(check_ptr(pooled, "pooled"));
+  return cuda_status(t3d::launch_scatter_pool_packed(g, x, y, pooled, as_stream(stream)),
+                     "tile3d_scatter_pool_packed");
+}
+
 t3d_status tile_select_packed_capacity(int n_tiles, int mode, int n_prefix, int n_regions,
                                        const int32_t* spans, const double* keep_rates, int* kmax) {
   if (n_tiles < 1 || kmax == nullptr) return fail(T3D_ERR_INVALID, "n_tiles >= 1 and kmax needed");

@@ -102,6 +102,8 @@ struct PackedGeo {
 cudaError_t launch_scatter_packed(const PackedGeo& p, const void* x, void* y, cudaStream_t s);
 cudaError_t launch_gather_packed(const PackedGeo& p, const void* y, void* x, cudaStream_t s);
 cudaError_t launch_pool_packed(const PackedGeo& p, const void* y, float* pooled, cudaStream_t s);
+cudaError_t launch_scatter_pool_packed(const PackedGeo& p, const void* x, void* y, float* pooled,
+                                       cudaStream_t s);
 size_t attn_packed_workspace_bytes(const PackedGeo& p, int kmax);
 cudaError_t launch_attn_packed(const PackedGeo& p, const AttnArgs& a, cudaStream_t s);
 // The 64-row-unit geometry the attention kernel runs a packed buffer with.

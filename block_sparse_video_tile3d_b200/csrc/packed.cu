@@ -122,6 +122,67 @@ __global__ void __launch_bounds__(32 * kPoolRows) pool_packed_kernel(PackedGeo p
   }
 }
 
+// Scatter fused with pooling, grid (ceil(row_chunks / 32), n_tiles, B), block (32, kPoolRows): the
+// CTA moves one 512-byte column slab of one tile, thread (lane, ry) copying chunk column `lane` of
+// the tile's slots ry, ry + kPoolRows, ... from their packed rows (zeros for pads) and summing the
+// valid ones; the partial sums are combined in shared memory and divided by the valid count.
+__global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_packed_kernel(
+    PackedGeo p, const uint4* __restrict__ x, uint4* __restrict__ y, float* __restrict__ pooled) {
+  __shared__ float part[kPoolRows][32 * 8 + 4];
+  const int lane = threadIdx.x;
+  const int ry = threadIdx.y;
+  const int i = blockIdx.y;
+  const int b = blockIdx.z;
+  const int c = blockIdx.x * 32 + lane;
+  const int vc = p.vc[i];
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  if (c < p.row_chunks) {
+    const long dst0 = ((long)b * p.n_tiles * p.E + (long)i * p.E) * p.row_stride + p.row_off + c;
+    const long src_b = (long)b * p.rows;
+    const int32_t* sr = p.slot_row + (long)i * p.E;
+    // The tile's rows this thread moves, up to 8 (E / kPoolRows), loaded before any is used.
+    constexpr int kMaxPer = 128 / kPoolRows;
+    const int per = p.E / kPoolRows;
+    uint4 u[kMaxPer];
+#pragma unroll
+    for (int t = 0; t < kMaxPer; ++t) {
+      const int srow = t < per ? sr[ry + kPoolRows * t] : -1;
+      u[t] = srow >= 0 ? __ldg(x + (src_b + srow) * p.row_stride + p.row_off + c)
+                       : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int t = 0; t < kMaxPer; ++t) {
+      if (t >= per) break;
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[t]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] += f.x;
+        acc[2 * e + 1] += f.y;
+      }
+      y[dst0 + (long)(ry + kPoolRows * t) * p.row_stride] = u[t];
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[ry][lane * 8 + e] = acc[e];
+  __syncthreads();
+  const int t = ry * 32 + lane;
+  const int cc = t >> 3;
+  const int e = t & 7;
+  const int col_chunk = blockIdx.x * 32 + cc;
+  if (t < 32 * 8 && col_chunk < p.row_chunks) {  // the first 256 threads: 32 chunks x 8 elements
+    float sum = 0.f;
+#pragma unroll
+    for (int q = 0; q < kPoolRows; ++q) sum += part[q][cc * 8 + e];
+    const int col = col_chunk * 8 + e;
+    const int h = col / p.D;
+    const int d = col - h * p.D;
+    pooled[(((long)b * p.heads + h) * p.n_tiles + i) * p.D + d] = vc > 0 ? sum / (float)vc : 0.f;
+  }
+}
+
 // Valid counts of the kernel's 64-row units, and (128-row tiles) the half-tile lists.
 __global__ void attn_packed_prep_kernel(PackedGeo p, const int32_t* __restrict__ kv_idx,
                                         const int32_t* __restrict__ kv_cnt, int kmax,
@@ -208,6 +269,15 @@ cudaError_t launch_pool_packed(const PackedGeo& p, const void* y, float* pooled,
   dim3 grid((p.row_chunks + 31) / 32, p.n_tiles, p.B);
   dim3 block(32, kPoolRows);
   pool_packed_kernel<<<grid, block, 0, s>>>(p, static_cast<const uint4*>(y), pooled);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_scatter_pool_packed(const PackedGeo& p, const void* x, void* y, float* pooled,
+                                       cudaStream_t s) {
+  dim3 grid((p.row_chunks + 31) / 32, p.n_tiles, p.B);
+  dim3 block(32, kPoolRows);
+  scatter_pool_packed_kernel<<<grid, block, 0, s>>>(p, static_cast<const uint4*>(x),
+                                                    static_cast<uint4*>(y), pooled);
   return cudaGetLastError();
 }
 

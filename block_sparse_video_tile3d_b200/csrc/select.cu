@@ -215,13 +215,68 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
   tot = warp_sum(tot);
   const float target = mass * tot;
   // Largest key thr with sum_{key >= thr} e >= target: the key of the tile at which the running
-  // sum (descending order) first reaches the target.
+  // sum (descending order) first reaches the target. First a search on the values: a bracket
+  // [lo, hi) with F(lo) >= target > F(hi), F(t) = sum of the e >= t, narrowed by interpolating F
+  // linearly (Illinois rule against a stalling end) until exactly one value lies in it — that
+  // value is the crossing tile's, and F(lo) is then the sum of the same tiles in the same order as
+  // the emission below recomputes. Rows where that does not happen within the step budget (ties
+  // at the crossing value) take the bit-by-bit key search.
   uint32_t prefix = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = prefix | (1u << bit);
-    float s = 0.f;
-    for (int j = lane; j < nT; j += 32) s += (float_key(row[j]) >= cand) ? row[j] : 0.f;
-    if (warp_sum(s) >= target) prefix = cand;
+  bool found = false;
+  {
+    float lo = 0.f, hi = 2.f;  // every e lies in [0, 1]
+    float Flo = tot, Fhi = 0.f;
+    int clo = nT, chi = 0;
+    float wlo = 1.f, whi = 1.f;
+    int side = 0;
+    for (int step = 0; step < 24; ++step) {
+      if (clo - chi == 1) {
+        float v = -1.f;
+        for (int j = lane; j < nT; j += 32)
+          if (row[j] >= lo && row[j] < hi) v = row[j];
+        v = warp_max(v);
+        prefix = float_key(v);
+        found = true;
+        break;
+      }
+      const float a = wlo * (Flo - target), bb = whi * (target - Fhi);
+      float t = fmaf(hi - lo, __fdividef(a, a + bb), lo);
+      if (!(t > lo && t < hi)) t = 0.5f * (lo + hi);
+      if (!(t > lo && t < hi)) break;
+      float ft = 0.f;
+      int ct = 0;
+      for (int j = lane; j < nT; j += 32) {
+        if (row[j] >= t) {
+          ft += row[j];
+          ++ct;
+        }
+      }
+      ft = warp_sum(ft);
+      ct = warp_sum_int(ct);
+      if (ft >= target) {
+        lo = t;
+        Flo = ft;
+        clo = ct;
+        whi = side == 1 ? 0.5f * whi : 1.f;
+        wlo = 1.f;
+        side = 1;
+      } else {
+        hi = t;
+        Fhi = ft;
+        chi = ct;
+        wlo = side == -1 ? 0.5f * wlo : 1.f;
+        whi = 1.f;
+        side = -1;
+      }
+    }
+  }
+  if (!found) {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      float s = 0.f;
+      for (int j = lane; j < nT; j += 32) s += (float_key(row[j]) >= cand) ? row[j] : 0.f;
+      if (warp_sum(s) >= target) prefix = cand;
+    }
   }
   float above = 0.f;
   int n_above = 0;
@@ -665,61 +720,103 @@ constexpr int kPruneThreads = 256;
 // keep_size == 0: threshold mode (rows with cosine to the block mean above cos_thresh are pruned);
 // keep_size > 0: ratio mode (the keep_size rows with the lowest cosine are kept, lowest index on
 // ties). Either way a pruned row copies its most cosine-similar kept row.
-__global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_bfloat16* __restrict__ q,
+// One CTA per (batch, head, 64-row block), 8 warps of 8 rows each. Lane l of a warp holds 16-byte
+// chunk l % kChunks of rows 8 w + kRowsPerLoad t + l / kChunks (t < kLoads) in registers as fp32;
+// column sums, row norms and dot products with the block mean come from warp shuffles and a small
+// shared-memory combine across warps. The rows go to shared memory only when some row is pruned
+// (for the source search), and the kept-row mean is the block mean when nothing is pruned.
+template <int kD>
+__global__ void __launch_bounds__(kPruneThreads, kD == 128 ? 2 : 1) prune_kernel(Geo g, const __nv_bfloat16* __restrict__ q,
                                                               float cos_thresh, int keep_size,
                                                               uint8_t* __restrict__ keep,
                                                               uint8_t* __restrict__ src_row,
                                                               float* __restrict__ pq_kept) {
+  constexpr int kChunks = kD / 8;              // 16-byte chunks of a row
+  constexpr int kRowsPerLoad = 32 / kChunks;   // rows one warp-wide load covers
+  constexpr int kWarps = kPruneThreads / 32;
+  constexpr int kRowsPerWarp = kTileElems / kWarps;
+  constexpr int kLoads = kRowsPerWarp / kRowsPerLoad;
+  constexpr int ld = kD + 1;
   extern __shared__ float sm[];
-  const int D = g.D, ld = D + 1;
-  float* qs = sm;                       // [64][D+1]
-  float* mu = qs + kTileElems * ld;     // [D]
-  float* n2 = mu + D;                   // [64] squared row norms
-  float* cosm = n2 + kTileElems;        // [64] cosine to the block mean
-  int* keep_s = reinterpret_cast<int*>(cosm + kTileElems);  // [64]
-  int* src_s = keep_s + kTileElems;                         // [64]
+  float* qs = sm;                          // [64][D+1], filled only when a row is pruned
+  __shared__ float part[kWarps][kD];       // per-warp column sums
+  __shared__ float mu[kD];
+  __shared__ float n2[kTileElems], cosm[kTileElems];
+  __shared__ int keep_s[kTileElems], src_s[kTileElems];
   __shared__ float mu_n2;
   __shared__ int n_keep;
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
-  const long row_stride = (long)g.heads_total * D;
+  const int chunk = lane % kChunks, sub = lane / kChunks;
+  const long row_stride = (long)g.heads_total * kD;
   const __nv_bfloat16* base =
-      q + ((long)b * g.Lp + (long)i * kTileElems) * row_stride + (long)(g.head0 + h) * D;
-  for (int e = tid; e < kTileElems * D / 8; e += kPruneThreads) {
-    const int r = e / (D / 8), c = e - r * (D / 8);
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(base + r * row_stride) + c);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+      q + ((long)b * g.Lp + (long)i * kTileElems) * row_stride + (long)(g.head0 + h) * kD;
+  float x[kLoads][8];
+  uint4 u[kLoads];
 #pragma unroll
-    for (int t = 0; t < 4; ++t) {
-      const float2 f = __bfloat1622float2(h2[t]);
-      qs[r * ld + c * 8 + 2 * t] = f.x;
-      qs[r * ld + c * 8 + 2 * t + 1] = f.y;
+  for (int t = 0; t < kLoads; ++t) {
+    const int r = kRowsPerWarp * w + kRowsPerLoad * t + sub;
+    u[t] = __ldg(reinterpret_cast<const uint4*>(base + r * row_stride) + chunk);
+  }
+#pragma unroll
+  for (int t = 0; t < kLoads; ++t) {
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[t]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h2[e]);
+      x[t][2 * e] = f.x;
+      x[t][2 * e + 1] = f.y;
+    }
+  }
+  // Column sums over this warp's rows: over t in registers, then over the lanes holding the same
+  // chunk of other rows.
+  {
+    float cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float v = 0.f;
+#pragma unroll
+      for (int t = 0; t < kLoads; ++t) v += x[t][e];
+#pragma unroll
+      for (int o = kChunks; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      cs[e] = v;
+    }
+    if (sub == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[w][chunk * 8 + e] = cs[e];
     }
   }
   __syncthreads();
-  for (int d = tid; d < D; d += kPruneThreads) {
-    float s = 0.f;
-    for (int r = 0; r < kTileElems; ++r) s += qs[r * ld + d];
-    mu[d] = s / (float)kTileElems;
+  if (tid < kD) {
+    float v = 0.f;
+#pragma unroll
+    for (int q2 = 0; q2 < kWarps; ++q2) v += part[q2][tid];
+    mu[tid] = v / (float)kTileElems;
   }
   __syncthreads();
   if (w == 0) {
-    float s = 0.f;
-    for (int d = lane; d < D; d += 32) s += mu[d] * mu[d];
-    s = warp_sum(s);
-    if (lane == 0) mu_n2 = s;
+    float v = 0.f;
+    for (int d = lane; d < kD; d += 32) v += mu[d] * mu[d];
+    v = warp_sum(v);
+    if (lane == 0) mu_n2 = v;
   }
   __syncthreads();
-  for (int r = w; r < kTileElems; r += kPruneThreads / 32) {
+  // Row norms and dot products with the mean: per lane over its chunk, then over the chunk lanes.
+#pragma unroll
+  for (int t = 0; t < kLoads; ++t) {
     float a = 0.f, dm = 0.f;
-    for (int d = lane; d < D; d += 32) {
-      const float x = qs[r * ld + d];
-      a += x * x;
-      dm += x * mu[d];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      a = fmaf(x[t][e], x[t][e], a);
+      dm = fmaf(x[t][e], mu[chunk * 8 + e], dm);
     }
-    a = warp_sum(a);
-    dm = warp_sum(dm);
-    if (lane == 0) {
+#pragma unroll
+    for (int o = 1; o < kChunks; o <<= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+      dm += __shfl_xor_sync(0xffffffffu, dm, o);
+    }
+    if (chunk == 0) {
+      const int r = kRowsPerWarp * w + kRowsPerLoad * t + sub;
       n2[r] = a;
       cosm[r] = (a == 0.f || mu_n2 == 0.f) ? 0.f : dm / (sqrtf(a) * sqrtf(mu_n2));
     }
@@ -766,8 +863,52 @@ __global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_
     if (lane == 0) n_keep = nk;
   }
   __syncthreads();
+  const long blk = (((long)b * g.heads + h) * g.nT + i);
+  const int nk = n_keep;
+  if (nk == kTileElems) {
+    // Nothing pruned: every row is its own source and the kept-row mean is the block mean.
+    if (tid < kD) pq_kept[blk * kD + tid] = mu[tid];
+    if (tid < kTileElems) {
+      keep[blk * kTileElems + tid] = 1;
+      src_row[blk * kTileElems + tid] = (uint8_t)tid;
+    }
+    return;
+  }
+  // Some rows are pruned: the rows go to shared memory for the source search, and the kept-row
+  // mean is summed from the registers with the keep mask.
+#pragma unroll
+  for (int t = 0; t < kLoads; ++t) {
+    const int r = kRowsPerWarp * w + kRowsPerLoad * t + sub;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) qs[r * ld + chunk * 8 + e] = x[t][e];
+  }
+  {
+    float cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float v = 0.f;
+#pragma unroll
+      for (int t = 0; t < kLoads; ++t)
+        v += keep_s[kRowsPerWarp * w + kRowsPerLoad * t + sub] ? x[t][e] : 0.f;
+#pragma unroll
+      for (int o = kChunks; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      cs[e] = v;
+    }
+    __syncthreads();  // every warp is past reading `part` above
+    if (sub == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part[w][chunk * 8 + e] = cs[e];
+    }
+  }
+  __syncthreads();
+  if (tid < kD) {
+    float v = 0.f;
+#pragma unroll
+    for (int q2 = 0; q2 < kWarps; ++q2) v += part[q2][tid];
+    pq_kept[blk * kD + tid] = v / (float)nk;
+  }
   // Each pruned row takes the most cosine-similar kept row (lowest index on ties).
-  for (int r = w; r < kTileElems; r += kPruneThreads / 32) {
+  for (int r = w; r < kTileElems; r += kWarps) {
     if (keep_s[r]) {
       if (lane == 0) src_s[r] = r;
       continue;
@@ -777,7 +918,7 @@ __global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_
     for (int j = lane; j < kTileElems; j += 32) {
       if (!keep_s[j]) continue;
       float dot = 0.f;
-      for (int d = 0; d < D; ++d) dot = fmaf(qs[r * ld + d], qs[j * ld + d], dot);
+      for (int d = 0; d < kD; ++d) dot = fmaf(qs[r * ld + d], qs[j * ld + d], dot);
       const float c = (n2[r] == 0.f || n2[j] == 0.f) ? 0.f : dot / (sqrtf(n2[r]) * sqrtf(n2[j]));
       if (c > best || (c == best && j < bj)) { best = c; bj = j; }
     }
@@ -790,12 +931,6 @@ __global__ void __launch_bounds__(kPruneThreads) prune_kernel(Geo g, const __nv_
     if (lane == 0) src_s[r] = bj;
   }
   __syncthreads();
-  const long blk = (((long)b * g.heads + h) * g.nT + i);
-  for (int d = tid; d < D; d += kPruneThreads) {
-    float s = 0.f;
-    for (int r = 0; r < kTileElems; ++r) s += keep_s[r] ? qs[r * ld + d] : 0.f;
-    pq_kept[blk * D + d] = s / (float)n_keep;
-  }
   if (tid < kTileElems) {
     keep[blk * kTileElems + tid] = (uint8_t)keep_s[tid];
     src_row[blk * kTileElems + tid] = (uint8_t)src_s[tid];
@@ -941,14 +1076,24 @@ cudaError_t launch_mask_to_index(const Geo& g, const uint8_t* mask, int kmax, in
 
 cudaError_t launch_prune(const Geo& g, const void* q, float cos_thresh, int keep_size, uint8_t* keep,
                          uint8_t* src_row, float* pq_kept, cudaStream_t s) {
-  const size_t smem = ((size_t)kTileElems * (g.D + 1) + g.D + 2 * kTileElems) * sizeof(float) +
-                      2 * kTileElems * sizeof(int);
-  cudaError_t e = cudaFuncSetAttribute(prune_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
+  // Dynamic shared memory: the block's rows as fp32 (read only when some row is pruned).
+  const size_t smem = (size_t)kTileElems * (g.D + 1) * sizeof(float);
   dim3 grid(g.nT, g.heads, g.B);
-  prune_kernel<<<grid, kPruneThreads, smem, s>>>(g, static_cast<const __nv_bfloat16*>(q),
-                                                 cos_thresh, keep_size, keep, src_row, pq_kept);
+  const __nv_bfloat16* qq = static_cast<const __nv_bfloat16*>(q);
+  cudaError_t e;
+  if (g.D == 128) {
+    e = cudaFuncSetAttribute(prune_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    prune_kernel<128><<<grid, kPruneThreads, smem, s>>>(g, qq, cos_thresh, keep_size, keep,
+                                                        src_row, pq_kept);
+  } else {
+    e = cudaFuncSetAttribute(prune_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    prune_kernel<64><<<grid, kPruneThreads, smem, s>>>(g, qq, cos_thresh, keep_size, keep,
+                                                       src_row, pq_kept);
+  }
   return cudaGetLastError();
 }
 

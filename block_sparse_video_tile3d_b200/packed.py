@@ -19,7 +19,8 @@ from .api import _need, _ptr, _slice, _stream
 
 __all__ = [
     "TILE_SHAPES", "PackedGeometry", "span_keep_rates", "tile3d_scatter_packed",
-    "tile3d_gather_packed", "tile_pool_packed", "tile_select_packed", "block_sparse_attn_fwd_packed",
+    "tile3d_gather_packed", "tile_pool_packed", "tile3d_scatter_pool_packed", "tile_select_packed",
+    "block_sparse_attn_fwd_packed",
     "PackedTileSparseAttention",
 ]
 
@@ -142,6 +143,23 @@ def tile_pool_packed(y: torch.Tensor, geo: PackedGeometry, out: torch.Tensor | N
     return out
 
 
+def tile3d_scatter_pool_packed(x: torch.Tensor, geo: PackedGeometry, out: torch.Tensor | None = None,
+                               pooled: torch.Tensor | None = None, head0: int = 0,
+                               heads: int | None = None):
+    """``tile3d_scatter_packed`` and ``tile_pool_packed`` in one pass: ``(y, pooled)``."""
+    B, L, nh, D = x.shape
+    _need(x, "x", torch.bfloat16, (B, geo.rows, nh, D))
+    p, B, nh, D, hh = _call_struct(geo, x, head0, heads)
+    if out is None:
+        out = torch.empty((B, geo.buffer_rows, nh, D), dtype=torch.bfloat16, device=x.device)
+    if pooled is None:
+        pooled = torch.empty((B, hh, geo.n_tiles, D), dtype=torch.float32, device=x.device)
+    _need(out, "out", torch.bfloat16, (B, geo.buffer_rows, nh, D))
+    _need(pooled, "pooled", torch.float32, (B, hh, geo.n_tiles, D))
+    check(lib.tile3d_scatter_pool_packed(ctypes.byref(p), _ptr(x), _ptr(out), _ptr(pooled), _stream()))
+    return out, pooled
+
+
 def _spans_args(geo: PackedGeometry, keep_rates, mode: int):
     spans = (ctypes.c_int32 * len(geo.spans_flat))(*geo.spans_flat)
     rates = (ctypes.c_double * geo.n_regions)(*[float(r) for r in keep_rates])
@@ -250,11 +268,9 @@ class PackedTileSparseAttention:
         """The path as named launches over persistent buffers (for timing each stage)."""
         g, d = self.geo, self._buffers(q)
         return [
-            ("scatter_q", lambda: tile3d_scatter_packed(q, g, out=d["qt"])),
-            ("scatter_k", lambda: tile3d_scatter_packed(k, g, out=d["kt"])),
+            ("scatter_pool_q", lambda: tile3d_scatter_pool_packed(q, g, out=d["qt"], pooled=d["pq"])),
+            ("scatter_pool_k", lambda: tile3d_scatter_pool_packed(k, g, out=d["kt"], pooled=d["pk"])),
             ("scatter_v", lambda: tile3d_scatter_packed(v, g, out=d["vt"])),
-            ("pool_q", lambda: tile_pool_packed(d["qt"], g, out=d["pq"])),
-            ("pool_k", lambda: tile_pool_packed(d["kt"], g, out=d["pk"])),
             ("select", lambda: tile_select_packed(d["pq"], d["pk"], g, self.keep_rates, self.mode,
                                                   workspace=d["ws_sel"], dev_status=self.status,
                                                   kv_idx=d["kv_idx"], kv_cnt=d["kv_cnt"])),

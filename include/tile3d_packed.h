@@ -110,6 +110,15 @@ t3d_status tile3d_gather_packed(const t3d_packed* p, const void* y, void* x, t3d
  */
 t3d_status tile_pool_packed(const t3d_packed* p, const void* y, float* pooled, t3d_stream stream);
 
+/*
+ * tile3d_scatter_pool_packed — tile3d_scatter_packed and tile_pool_packed in one pass over the
+ * packed rows: y and pooled are what the two calls would write, up to the order of the fp32
+ * additions. Saves re-reading y.
+ *   x: in, packed order.  y: out, buffer order.  pooled: out, fp32 [B, heads, n_tiles, D].
+ */
+t3d_status tile3d_scatter_pool_packed(const t3d_packed* p, const void* x, void* y, float* pooled,
+                                      t3d_stream stream);
+
 #define T3D_PACKED_EXEMPT 0  /* dense tiles exempt from selection; per-region top-k */
 #define T3D_PACKED_COMPETE 1 /* one top-k over all tiles (one region only) */
 #define T3D_PACKED_DENSE 2   /* every tile kept (a dense layer or a dense step) */

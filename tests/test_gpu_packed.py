@@ -46,6 +46,17 @@ def test_scatter_gather_and_pool(name, E):
     np.testing.assert_allclose(pooled.cpu().numpy(), want_p, rtol=1e-5, atol=1e-6)
 
 
+@pytest.mark.parametrize("E", [64, 128])
+def test_fused_scatter_pool_equals_the_two_calls(E):
+    geo, ref = _geos(SEQS["prefix_two_regions"], E)
+    x = _x(2, geo.rows, 3, 128, seed=31 + E)
+    y, pooled = P.tile3d_scatter_pool_packed(x.cuda(), geo)
+    y2 = P.tile3d_scatter_packed(x.cuda(), geo)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    want_p = pool.tile_mean_pool(packed.scatter(f64(x), ref), ref["vc"], E)
+    np.testing.assert_allclose(pooled.cpu().numpy(), want_p, rtol=1e-5, atol=1e-6)
+
+
 def test_head_range_scatter_leaves_other_heads():
     geo, ref = _geos(SEQS["prefix_two_regions"], 128)
     x = _x(1, geo.rows, 4, 64, seed=9).cuda()

@@ -175,8 +175,9 @@ def test_workload_selection_small_full():
     assert stats["exact"] >= 0.5 * w.heads * w.nT
 
 
-def test_prune_matches_oracle_structured():
-    w = workloads.WORKLOADS["bsa"].with_(T=8, H=8, W=12, heads=3)
+@pytest.mark.parametrize("D", [128, 64])
+def test_prune_matches_oracle_structured(D):
+    w = workloads.WORKLOADS["bsa"].with_(T=8, H=8, W=12, heads=3, D=D)
     q, _, _ = workloads.make_qkv(w)
     q = workloads.make_structured_queries(w, q)
     qt = tile3d_scatter(q.cuda(), w.T, w.H, w.W)
