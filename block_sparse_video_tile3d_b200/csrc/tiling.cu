@@ -126,66 +126,85 @@ __global__ void __launch_bounds__(32 * kPoolRows) pool_kernel(Geo g, const uint4
   }
 }
 
-// Fused scatter + pool: grid (ceil(row_chunks / 32), nT, B), block (32, kPoolRows). The CTA moves
-// one 512-byte column slab of one tile: thread (lane, ry) copies chunk column `lane` of the tile's
-// padded rows ry, ry + kPoolRows, ... from their raster rows (zeros for pad slots) and sums the
-// valid ones; the partial sums are combined in shared memory and divided by the valid count.
+// Fused scatter + pool: grid (ceil(row_chunks / 32), ceil(nT / kSpTiles), B), block (32,
+// kPoolRows). The CTA moves one 512-byte column slab of kSpTiles consecutive tiles: thread (lane,
+// ry) copies chunk column `lane` of each tile's padded rows ry, ry + kPoolRows, ... from their
+// raster rows (zeros for pad slots) and sums the valid ones; the partial sums are combined in
+// shared memory and divided by the valid count. All of a thread's loads (kSpTiles * 4 rows) are
+// issued before any is used.
+constexpr int kSpTiles = 2;
+
 __global__ void __launch_bounds__(32 * kPoolRows) scatter_pool_kernel(Geo g,
                                                                       const uint4* __restrict__ x,
                                                                       uint4* __restrict__ y,
                                                                       float* __restrict__ pooled) {
-  __shared__ float part[kPoolRows][32 * 8 + 4];
-  __shared__ int src_row[kTileElems];
+  __shared__ float part[kSpTiles][kPoolRows][32 * 8 + 4];
+  __shared__ int src_row[kSpTiles][kTileElems];
   const int lane = threadIdx.x;
   const int ry = threadIdx.y;
-  const int i = blockIdx.y;
+  const int i0 = blockIdx.y * kSpTiles;
   const int b = blockIdx.z;
   const int c = blockIdx.x * 32 + lane;
   const int t = ry * 32 + lane;
-  if (t < kTileElems) src_row[t] = padded_to_raster(g, i * kTileElems + t);
+  for (int e = t; e < kSpTiles * kTileElems; e += 32 * kPoolRows) {
+    const int tt = e / kTileElems, slot = e - tt * kTileElems;
+    src_row[tt][slot] = i0 + tt < g.nT ? padded_to_raster(g, (i0 + tt) * kTileElems + slot) : -1;
+  }
   __syncthreads();
-  float acc[8];
+  constexpr int kPer = kTileElems / kPoolRows;
+  float acc[kSpTiles][8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  for (int tt = 0; tt < kSpTiles; ++tt)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[tt][e] = 0.f;
   if (c < g.row_chunks) {
-    // All four of this thread's rows are loaded before any is used, so the four loads are in
-    // flight together; pad slots read as zero and add nothing to the sums.
-    constexpr int kPer = kTileElems / kPoolRows;
-    const long dst0 = ((long)b * g.Lp + (long)i * kTileElems) * g.row_stride + g.row_off + c;
     const long src_b = (long)b * g.L;
-    uint4 u[kPer];
+    uint4 u[kSpTiles][kPer];
 #pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-      const int sr = src_row[ry + kPoolRows * t];
-      u[t] = sr >= 0 ? ld_nc(x + (src_b + sr) * g.row_stride + g.row_off + c)
-                     : make_uint4(0u, 0u, 0u, 0u);
+    for (int tt = 0; tt < kSpTiles; ++tt) {
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int sr = src_row[tt][ry + kPoolRows * k];
+        u[tt][k] = sr >= 0 ? ld_nc(x + (src_b + sr) * g.row_stride + g.row_off + c)
+                           : make_uint4(0u, 0u, 0u, 0u);
+      }
     }
 #pragma unroll
-    for (int t = 0; t < kPer; ++t) {
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[t]);
+    for (int tt = 0; tt < kSpTiles; ++tt) {
+      if (i0 + tt >= g.nT) break;
+      const long dst0 = ((long)b * g.Lp + (long)(i0 + tt) * kTileElems) * g.row_stride + g.row_off + c;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h2[e]);
-        acc[2 * e] += f.x;
-        acc[2 * e + 1] += f.y;
+      for (int k = 0; k < kPer; ++k) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u[tt][k]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(h2[e]);
+          acc[tt][2 * e] += f.x;
+          acc[tt][2 * e + 1] += f.y;
+        }
+        y[dst0 + (long)(ry + kPoolRows * k) * g.row_stride] = u[tt][k];
       }
-      y[dst0 + (long)(ry + kPoolRows * t) * g.row_stride] = u[t];
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) part[ry][lane * 8 + e] = acc[e];
+  for (int tt = 0; tt < kSpTiles; ++tt)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[tt][ry][lane * 8 + e] = acc[tt][e];
   __syncthreads();
-  const int cc = t >> 3;
+  // The first 256 threads finalise tile 0's 32 chunks x 8 elements, the next 256 tile 1's.
+  const int tt = t >> 8;
+  const int cc = (t & 255) >> 3;
   const int e = t & 7;
   const int col_chunk = blockIdx.x * 32 + cc;
-  if (t < 32 * 8 && col_chunk < g.row_chunks) {  // the first 256 threads: 32 chunks x 8 elements
+  if (tt < kSpTiles && i0 + tt < g.nT && col_chunk < g.row_chunks) {
     float sum = 0.f;
 #pragma unroll
-    for (int q = 0; q < kPoolRows; ++q) sum += part[q][cc * 8 + e];
+    for (int q = 0; q < kPoolRows; ++q) sum += part[tt][q][cc * 8 + e];
     const int col = col_chunk * 8 + e;
     const int h = col / g.D;
     const int d = col - h * g.D;
-    pooled[(((long)b * g.heads + h) * g.nT + i) * g.D + d] = sum / (float)tile_valid_count(g, i);
+    pooled[(((long)b * g.heads + h) * g.nT + i0 + tt) * g.D + d] =
+        sum / (float)tile_valid_count(g, i0 + tt);
   }
 }
 
@@ -213,7 +232,7 @@ cudaError_t launch_gather(const Geo& g, const void* y, void* x, cudaStream_t s) 
 
 cudaError_t launch_scatter_pool(const Geo& g, const void* x, void* y, float* pooled,
                                 cudaStream_t s) {
-  dim3 grid((g.row_chunks + 31) / 32, g.nT, g.B);
+  dim3 grid((g.row_chunks + 31) / 32, (g.nT + kSpTiles - 1) / kSpTiles, g.B);
   dim3 block(32, kPoolRows);
   scatter_pool_kernel<<<grid, block, 0, s>>>(g, static_cast<const uint4*>(x), static_cast<uint4*>(y),
                                              pooled);
