@@ -21,16 +21,22 @@ namespace {
 constexpr int kCopyThreads = 256;
 constexpr int kPoolRows = 16;
 
+// A warp copies one row of n 16-byte chunks; each lane issues up to eight loads before it stores.
 __device__ __forceinline__ void copy_row16(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                            int n, int lane) {
-  int c = lane;
-  for (; c + 32 < n; c += 64) {
-    const uint4 a = __ldg(src + c);
-    const uint4 b = __ldg(src + c + 32);
-    dst[c] = a;
-    dst[c + 32] = b;
+  for (int c0 = 0; c0 < n; c0 += 256) {
+    uint4 u[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = c0 + lane + 32 * k;
+      if (c < n) u[k] = __ldg(src + c);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = c0 + lane + 32 * k;
+      if (c < n) dst[c] = u[k];
+    }
   }
-  for (; c < n; c += 32) dst[c] = __ldg(src + c);
 }
 
 // One warp per buffer row (pads written as zeros).

@@ -17,20 +17,22 @@ constexpr int kCopyThreads = 256;
 
 __device__ __forceinline__ uint4 ld_nc(const uint4* p) { return __ldg(p); }
 
+// A warp copies one row of n 16-byte chunks; each lane issues up to eight loads before it stores.
 __device__ __forceinline__ void copy_row(const uint4* __restrict__ src, uint4* __restrict__ dst,
                                          int n, int lane) {
-  int c = lane;
-  for (; c + 96 < n; c += 128) {
-    const uint4 a = ld_nc(src + c);
-    const uint4 b = ld_nc(src + c + 32);
-    const uint4 d = ld_nc(src + c + 64);
-    const uint4 e = ld_nc(src + c + 96);
-    dst[c] = a;
-    dst[c + 32] = b;
-    dst[c + 64] = d;
-    dst[c + 96] = e;
+  for (int c0 = 0; c0 < n; c0 += 256) {
+    uint4 u[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = c0 + lane + 32 * k;
+      if (c < n) u[k] = ld_nc(src + c);
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int c = c0 + lane + 32 * k;
+      if (c < n) dst[c] = u[k];
+    }
   }
-  for (; c < n; c += 32) dst[c] = ld_nc(src + c);
 }
 
 __device__ __forceinline__ void zero_row(uint4* __restrict__ dst, int n, int lane) {
