@@ -358,10 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------- S issuer
-      // A thread's tcgen05.mma issue proceeds at about the rate the tensor pipe retires MMAs, so a
-      // thread that also waits on barriers leaves the pipe idle meanwhile: S and PV have one issuing
-      // thread each, and the pipe takes work from whichever is ready. tcgen05.commit tracks the MMAs
-      // of the committing thread only, which is what each barrier below needs.
+      // An mbarrier wait (or any acquire followed by tcgen05.fence) in the thread that issues MMAs
+      // lets that thread's queued MMAs drain before its next MMA issues, about 150 cycles of idle
+      // pipe per wait point, while the same wait in another thread costs the pipe nothing. So S and
+      // PV have one issuing thread each: the pipe takes work from whichever is ready, and each
+      // thread's waits are covered by the other's queued MMAs. tcgen05.commit tracks the MMAs of
+      // the committing thread only, which is what each barrier below needs.
       if (lane == 0) {
         int active = 0;  // units with at least one pair, in order
         long nu = 0, gp = 0;  // units taken, global step index
