@@ -186,10 +186,13 @@ __device__ int select_topk_any(const float* row, int n, int k, int32_t* out, int
 
 // Cumulative-mass selection of one row (one warp). The scores in row[0..nT) are replaced by
 // e_j = exp(scale * (S_j - max S)); tiles are ranked by e (ties: lower index) and the smallest
-// prefix whose sum reaches mass * sum(e) is kept (at least min_k, at most kmax tiles, the most
-// probable ones; T3D_DEV_OVERFLOW when truncated). Writes ascending indices to out, returns the count.
+// prefix whose sum reaches mass * sum(e) is kept. Writes ascending indices to out and returns the
+// count; when the count falls outside [min_k, kmax] (T3D_DEV_OVERFLOW above kmax) it writes
+// nothing and returns -1 - k, k the number of highest-scoring tiles to keep instead, which
+// mass_fix_kernel then selects from the score row (that rare path stays out of this kernel, whose
+// register count, and so its occupancy, it would otherwise set).
 __device__ int select_mass_row(float* row, int nT, float scale, float mass, int min_k, int kmax,
-                               int32_t* out, int32_t* dev_status, int* hist) {
+                               int32_t* out, int32_t* dev_status) {
   const int lane = threadIdx.x & 31;
   if (mass >= 1.f) {
     // Every probability of a softmax is positive, so the running sum reaches 1 only with the last
@@ -200,7 +203,7 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
       return nT;
     }
     if (lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
-    return select_topk_any(row, nT, kmax, out, hist);
+    return -1 - kmax;
   }
   float mx = -INFINITY;
   for (int j = lane; j < nT; j += 32) mx = fmaxf(mx, row[j]);
@@ -314,9 +317,163 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
   if (count < floor_k || count > kmax) {
     const int kk = count < floor_k ? floor_k : kmax;
     if (count > kmax && lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
-    count = select_topk_any(row, nT, imin(kk, kmax), out, hist);
-  } else {
-    emit_threshold(row, nT, prefix, need_eq, out, kmax);
+    return -1 - imin(kk, kmax);
+  }
+  emit_threshold(row, nT, prefix, need_eq, out, kmax);
+  return count;
+}
+
+// select_mass_row with the row in registers (lane l holds entries l + 32 i, i < KPL): the same
+// operations in the same order, so the same sums and the same selection, without the shared-memory
+// traffic and address arithmetic of every pass. Pads hold -1, below every e.
+template <int KPL>
+__device__ int select_mass_row_reg(const float* __restrict__ srow, int nT, float scale, float mass,
+                                   int min_k, int kmax, int32_t* out, int32_t* dev_status) {
+  const int lane = threadIdx.x & 31;
+  const unsigned lt = lanemask_lt();
+  float e[KPL];
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const int j = lane + 32 * i;
+    e[i] = j < nT ? srow[j] : -INFINITY;
+  }
+  if (mass >= 1.f) {
+    if (nT <= kmax) {
+      for (int j = lane; j < nT; j += 32) out[j] = j;
+      return nT;
+    }
+    if (lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
+    return -1 - kmax;
+  }
+  float mx = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) mx = fmaxf(mx, e[i]);
+  mx = warp_max(mx);
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    if (lane + 32 * i < nT) {
+      e[i] = expf(scale * (e[i] - mx));
+      tot += e[i];
+    } else {
+      e[i] = -1.f;
+    }
+  }
+  tot = warp_sum(tot);
+  const float target = mass * tot;
+  uint32_t prefix = 0;
+  bool found = false;
+  {
+    float lo = 0.f, hi = 2.f;
+    float Flo = tot, Fhi = 0.f;
+    int clo = nT, chi = 0;
+    float wlo = 1.f, whi = 1.f;
+    int side = 0;
+    for (int step = 0; step < 24; ++step) {
+      if (clo - chi == 1) {
+        float v = -1.f;
+#pragma unroll
+        for (int i = 0; i < KPL; ++i)
+          if (e[i] >= lo && e[i] < hi) v = e[i];
+        v = warp_max(v);
+        prefix = float_key(v);
+        found = true;
+        break;
+      }
+      const float a = wlo * (Flo - target), bb = whi * (target - Fhi);
+      float t = fmaf(hi - lo, __fdividef(a, a + bb), lo);
+      if (!(t > lo && t < hi)) t = 0.5f * (lo + hi);
+      if (!(t > lo && t < hi)) break;
+      float ft = 0.f;
+      int ct = 0;
+#pragma unroll
+      for (int i = 0; i < KPL; ++i) {
+        if (e[i] >= t) {
+          ft += e[i];
+          ++ct;
+        }
+      }
+      ft = warp_sum(ft);
+      ct = warp_sum_int(ct);
+      if (ft >= target) {
+        lo = t;
+        Flo = ft;
+        clo = ct;
+        whi = side == 1 ? 0.5f * whi : 1.f;
+        wlo = 1.f;
+        side = 1;
+      } else {
+        hi = t;
+        Fhi = ft;
+        chi = ct;
+        wlo = side == -1 ? 0.5f * wlo : 1.f;
+        whi = 1.f;
+        side = -1;
+      }
+    }
+  }
+  if (!found) {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = prefix | (1u << bit);
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < KPL; ++i) sum += (e[i] >= 0.f && float_key(e[i]) >= cand) ? e[i] : 0.f;
+      if (warp_sum(sum) >= target) prefix = cand;
+    }
+  }
+  float above = 0.f;
+  int n_above = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    if (e[i] >= 0.f && float_key(e[i]) > prefix) {
+      above += e[i];
+      ++n_above;
+    }
+  }
+  above = warp_sum(above);
+  n_above = warp_sum_int(n_above);
+  // Tiles tied at the threshold are taken in ascending index until the target is reached.
+  int need_eq = 0;
+  {
+    float acc = above;
+    bool done = false;
+#pragma unroll
+    for (int i = 0; i < KPL; ++i) {
+      if (done) break;
+      const bool eq = e[i] >= 0.f && float_key(e[i]) == prefix;
+      unsigned eqb = __ballot_sync(0xffffffffu, eq);
+      while (eqb != 0u && !done) {
+        const int src = __ffs(eqb) - 1;
+        const float ev = __shfl_sync(0xffffffffu, e[i], src);
+        if (acc < target) {
+          acc += ev;
+          ++need_eq;
+        }
+        if (acc >= target) done = true;
+        eqb &= eqb - 1u;
+      }
+    }
+  }
+  const int count = n_above + need_eq;
+  const int floor_k = imin(min_k, nT);
+  if (count < floor_k || count > kmax) {
+    const int kk = count < floor_k ? floor_k : kmax;
+    if (count > kmax && lane == 0) report(dev_status, T3D_DEV_OVERFLOW);
+    return -1 - imin(kk, kmax);
+  }
+  int written = 0, eq_seen = 0;
+#pragma unroll
+  for (int i = 0; i < KPL; ++i) {
+    const bool valid = e[i] >= 0.f;
+    const uint32_t key = valid ? float_key(e[i]) : 0u;
+    const bool eq = valid && key == prefix;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool sel = (valid && key > prefix) || (eq && eq_seen + __popc(eqb & lt) < need_eq);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    const int pos = written + __popc(sb & lt);
+    if (sel && pos < kmax) out[pos] = lane + 32 * i;
+    written += __popc(sb);
+    eq_seen += __popc(eqb);
   }
   return count;
 }
@@ -624,27 +781,52 @@ __global__ void __launch_bounds__(kSelThreads) topk_rows_kernel(Geo g, const flo
 
 // One warp per query tile: cumulative-mass selection from its score row, staged in the warp's
 // shared-memory row buffer (the search reads it many times).
+template <int KPL>
 __global__ void __launch_bounds__(kSelThreads) mass_rows_kernel(Geo g, const float* __restrict__ S,
                                                                 int ldS, float scale, float mass,
                                                                 int min_k, int kmax,
                                                                 int32_t* __restrict__ kv_idx,
                                                                 int32_t* __restrict__ kv_cnt,
                                                                 int32_t* dev_status) {
-  extern __shared__ float rowbuf[];  // [8 warps][nT], then [8 warps][256] histogram ints
+  extern __shared__ float rowbuf[];  // KPL == 0: [8 warps][nT]
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nT = g.nT;
-  float* row = rowbuf + (long)w * nT;
-  int* hist = reinterpret_cast<int*>(rowbuf + (long)(kSelThreads / 32) * nT) + w * 256;
   const long rows = (long)g.B * g.heads * nT;
   for (long r = (long)blockIdx.x * (kSelThreads / 32) + w; r < rows;
        r += (long)gridDim.x * (kSelThreads / 32)) {
     const float* src = S + r * ldS;
-    for (int j = lane; j < nT; j += 32) row[j] = src[j];
+    int count;
+    if constexpr (KPL == 0) {
+      float* row = rowbuf + (long)w * nT;
+      for (int j = lane; j < nT; j += 32) row[j] = src[j];
+      __syncwarp();
+      count = select_mass_row(row, nT, scale, mass, min_k, kmax, kv_idx + r * kmax, dev_status);
+    } else {
+      count = select_mass_row_reg<KPL>(src, nT, scale, mass, min_k, kmax, kv_idx + r * kmax,
+                                       dev_status);
+    }
+    if (lane == 0) kv_cnt[r] = count;  // -1 - k: mass_fix_kernel keeps the top k instead
     __syncwarp();
-    const int count = select_mass_row(row, nT, scale, mass, min_k, kmax, kv_idx + r * kmax,
-                                      dev_status, hist);
-    if (lane == 0) kv_cnt[r] = count;
+  }
+}
+
+// One warp per row that mass_rows_kernel marked (kv_cnt = -1 - k): its k highest-scoring tiles
+// from the score row (ascending indices, ties to the lower index).
+__global__ void __launch_bounds__(kSelThreads) mass_fix_kernel(Geo g, const float* __restrict__ S,
+                                                               int ldS, int kmax,
+                                                               int32_t* __restrict__ kv_idx,
+                                                               int32_t* __restrict__ kv_cnt) {
+  __shared__ int hist[kSelThreads / 32][256];
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long rows = (long)g.B * g.heads * g.nT;
+  for (long r = (long)blockIdx.x * (kSelThreads / 32) + w; r < rows;
+       r += (long)gridDim.x * (kSelThreads / 32)) {
+    const int c = kv_cnt[r];
+    if (c >= 0) continue;
     __syncwarp();
+    const int n = select_topk_any(S + r * ldS, g.nT, -1 - c, kv_idx + r * kmax, hist[w]);
+    __syncwarp();
+    if (lane == 0) kv_cnt[r] = n;
   }
 }
 
@@ -1045,12 +1227,30 @@ cudaError_t launch_select_mass(const Geo& g, const float* pq, const float* pk, f
   int ldS = 0;
   cudaError_t e = launch_scores(g, pq, pk, workspace, &S, &ldS, s);
   if (e != cudaSuccess) return e;
-  const size_t smem = (size_t)(kSelThreads / 32) * ((size_t)g.nT * sizeof(float) + 256 * sizeof(int));
-  e = cudaFuncSetAttribute(mass_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
+  const int grid = sel_grid(g);
+  if (g.nT <= 128)
+    mass_rows_kernel<4><<<grid, kSelThreads, 0, s>>>(g, S, ldS, scale, mass, min_k, kmax, kv_idx,
+                                                     kv_cnt, dev_status);
+  else if (g.nT <= 256)
+    mass_rows_kernel<8><<<grid, kSelThreads, 0, s>>>(g, S, ldS, scale, mass, min_k, kmax, kv_idx,
+                                                     kv_cnt, dev_status);
+  else if (g.nT <= 512)
+    mass_rows_kernel<16><<<grid, kSelThreads, 0, s>>>(g, S, ldS, scale, mass, min_k, kmax, kv_idx,
+                                                      kv_cnt, dev_status);
+  else if (g.nT <= 1024)
+    mass_rows_kernel<32><<<grid, kSelThreads, 0, s>>>(g, S, ldS, scale, mass, min_k, kmax, kv_idx,
+                                                      kv_cnt, dev_status);
+  else {
+    const size_t smem = (size_t)(kSelThreads / 32) * (size_t)g.nT * sizeof(float);
+    e = cudaFuncSetAttribute(mass_rows_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+    if (e != cudaSuccess) return e;
+    mass_rows_kernel<0><<<grid, kSelThreads, smem, s>>>(g, S, ldS, scale, mass, min_k, kmax,
+                                                        kv_idx, kv_cnt, dev_status);
+  }
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  mass_rows_kernel<<<sel_grid(g), kSelThreads, smem, s>>>(g, S, ldS, scale, mass, min_k, kmax,
-                                                          kv_idx, kv_cnt, dev_status);
+  mass_fix_kernel<<<sel_grid(g), kSelThreads, 0, s>>>(g, S, ldS, kmax, kv_idx, kv_cnt);
   return cudaGetLastError();
 }
 
