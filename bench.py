@@ -279,6 +279,49 @@ def _source_sha() -> str:
     return h.hexdigest()[:16]
 
 
+# Kernels of this library one call of each stage launches, read off the launch code (csrc/*.cu);
+# used only when the profiler count below is unavailable. The attention calls also issue a 4-byte
+# memset of the work-queue counter, which is not a kernel of this library.
+STATIC_KERNELS = {
+    "scatter_q": 1, "scatter_k": 1, "scatter_v": 1, "scatter_pool_q": 1, "scatter_pool_k": 1,
+    "mask_to_index": 1, "prune_q": 1,
+    "select_topk": 3,   # split, tensor-core scores, top-k rows
+    "select_mass": 4,   # split, scores, mass rows, floor / cap fix-up
+    "select": 3,        # packed: split, scores, per-span rows
+    "attention": 1,
+    "attention_packed": 2,  # packed: list rewrite into 64-row halves, attention
+    "gather": 1,
+}
+
+
+def count_launches(stages, packed: bool = False) -> tuple[dict, str]:
+    """Kernels each stage launches, counted on the device: every stage runs once more (untimed)
+    under torch.profiler's CUDA activity trace and its kernel records are counted (memsets and
+    copies excluded). Falls back to STATIC_KERNELS if the profiler cannot trace."""
+    import torch
+    key = {"attention": "attention_packed"} if packed else {}
+    static = {n: STATIC_KERNELS[key.get(n, n)] for n, _ in stages}
+    if os.environ.get("CUDA_INJECTION64_PATH"):  # under ncu: leave CUPTI to it
+        return static, "static (launch code); another profiler is attached"
+    try:
+        from torch.autograd import DeviceType
+        from torch.profiler import ProfilerActivity, profile
+        counts = {}
+        for name, launch in stages:
+            torch.cuda.synchronize()
+            with profile(activities=[ProfilerActivity.CUDA]) as prof:
+                launch()
+                torch.cuda.synchronize()
+            counts[name] = sum(1 for e in prof.events()
+                               if e.device_type == DeviceType.CUDA
+                               and not e.name.startswith(("Memset", "Memcpy", "[")))
+        if min(counts.values()) < 1:  # every stage launches at least one kernel
+            return static, "static (launch code); the profiler recorded no kernels"
+        return counts, "torch.profiler CUDA kernel records, one untimed call per stage"
+    except Exception as exc:  # noqa: BLE001 - the count is a report, not a result
+        return static, f"static (launch code); profiler unavailable: {type(exc).__name__}"
+
+
 def _ncu_traffic(workload: str):
     """Per-launch DRAM bytes of the attention kernel from ``profiles/attn_traffic.json`` (written
     from an ncu capture), if that capture was taken on the current kernel source; else None. The
@@ -367,6 +410,7 @@ def run_ours(args, w):
     stage_ms = {n: sum(ev[s][j].elapsed_time(ev[s][j + 1]) for s in range(args.steps)) / args.steps
                 for j, n in enumerate(names)}
     clocks = sampler.stop()
+    launches, launch_src = count_launches(stages)
     total_ms = max_over_ranks(total_ms)
     ms_step = total_ms / args.steps
     status = model.device_status()
@@ -493,7 +537,8 @@ def run_ours(args, w):
                               "i's compute and download",
                 "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                 "d2h_bytes_per_step": od.numel() * od.element_size()},
-        "gpu_launches": args.steps * nst,
+        "gpu_launches": args.steps * sum(launches.values()),
+        "gpu_launches_per_step": {"by_stage": launches, "source": launch_src},
         "device_status": status,
         "clocks": clocks,
     }
@@ -636,6 +681,7 @@ def run_packed(args, w):
     stage_ms = {n: sum(ev[st][j].elapsed_time(ev[st][j + 1]) for st in range(args.steps)) / args.steps
                 for j, n in enumerate(names)}
     clocks = sampler.stop()
+    launches, launch_src = count_launches(stages, packed=True)
     ms_step = total_ms / args.steps
     status = int(mod.status.item())
     # end to end: pinned host inputs in, output back, every step inside the timed region
@@ -698,7 +744,8 @@ def run_packed(args, w):
                 "steps": e2e_steps, "output_matches_device_run": bool(torch.equal(oh, ref)),
                 "h2d_bytes_per_step": 3 * q.numel() * q.element_size(),
                 "d2h_bytes_per_step": od.numel() * od.element_size()},
-        "gpu_launches": args.steps * (nst + 1),  # the attention call launches a list-rewrite kernel too
+        "gpu_launches": args.steps * sum(launches.values()),
+        "gpu_launches_per_step": {"by_stage": launches, "source": launch_src},
         "device_status": status,
         "clocks": clocks,
     }

@@ -206,3 +206,64 @@ def test_module_end_to_end(E):
         rows = same[tile_of]
         assert rows.mean() >= 0.8
         assert_attn_close(got[:, rows, h], want[:, rows, h], f"module E={E} head {h}")
+
+
+@pytest.mark.parametrize("E", [64, 128])
+def test_head_range_pool_and_attention(E):
+    """A call on heads 1..2 of 4-head rows equals the full call on those heads and leaves the
+    other heads of the output untouched."""
+    geo, ref = _geos(SEQS["prefix_two_regions"], E)
+    q, k, v = (_x(1, geo.rows, 4, 64, seed=s).cuda() for s in (41, 42, 43))
+    qt, kt, vt = (P.tile3d_scatter_packed(t, geo) for t in (q, k, v))
+    full_p = P.tile_pool_packed(qt, geo)
+    part_p = P.tile_pool_packed(qt, geo, head0=1, heads=2)
+    assert torch.equal(part_p, full_p[:, 1:3])
+    y, pooled = P.tile3d_scatter_pool_packed(q, geo, head0=1, heads=2)
+    np.testing.assert_allclose(pooled.cpu().numpy(), full_p[:, 1:3].cpu().numpy(),
+                               rtol=1e-6, atol=1e-7)
+    pk = P.tile_pool_packed(kt, geo)
+    rates = packed.span_keep_rates(2, 0.6, 0.5, True)
+    kv_idx, kv_cnt = P.tile_select_packed(full_p, pk, geo, rates)
+    o_full = P.block_sparse_attn_fwd_packed(qt, kt, vt, kv_idx, kv_cnt, geo)
+    o = torch.full_like(qt, 5.0)
+    P.block_sparse_attn_fwd_packed(qt, kt, vt, kv_idx[:, 1:3].contiguous(),
+                                   kv_cnt[:, 1:3].contiguous(), geo, out=o, head0=1, heads=2)
+    assert torch.equal(o[:, :, 1:3], o_full[:, :, 1:3])
+    assert bool((o[:, :, 0] == 5.0).all()) and bool((o[:, :, 3] == 5.0).all())
+
+
+@pytest.mark.parametrize("kind", ["dense_layer", "compete"])
+def test_module_dense_and_compete(kind):
+    """The module in its other two selection modes against the oracle: a dense layer keeps every
+    tile (output exact to the dense oracle); compete mode, one top-k over all tiles of a
+    one-region sequence."""
+    E = 64
+    seq = [90, (8, 12, 16)]
+    kw = {"dense_layer": True} if kind == "dense_layer" else {"exempt": False}
+    mod = P.PackedTileSparseAttention(seq, heads=2, D=64, tile_size=E, sparsity=0.75, **kw)
+    geo = mod.geo
+    ref = packed.packed_geometry(packed.token_segments(seq, (1, 1, 1)), packed.TILE_SHAPES[E])
+    q, k, v = (_x(1, geo.rows, 2, 64, seed=s) for s in (51, 52, 53))
+    out = mod(q.cuda(), k.cuda(), v.cuda())
+    assert int(mod.status.item()) == 0
+    qt, kt, vt = (packed.scatter(f64(t), ref) for t in (q, k, v))
+    pq, pk = (pool.tile_mean_pool(t, ref["vc"], E) for t in (qt, kt))
+    S = select.tile_scores(pq, pk)
+    want_sets = packed.select(S, ref, mod.keep_rates, exempt=(kind == "dense_layer"),
+                              dense=(kind == "dense_layer"))
+    got_sets = gpu_sets(mod.kv_idx, mod.kv_cnt)
+    n_exact = _check_sets(got_sets, want_sets, S, ref, mod.keep_rates, mod.mode)
+    assert n_exact >= 0.8 * 2 * geo.n_tiles
+    if kind == "dense_layer":
+        assert n_exact == 2 * geo.n_tiles
+    want = packed.gather(attention.block_sparse_attention(qt, kt, vt, ref["vc"], want_sets,
+                                                          64 ** -0.5, tile_elems=E), ref)
+    got = f64(out)
+    tile_of = np.empty(geo.rows, dtype=np.int64)
+    sr = ref["slot_row"]
+    tile_of[sr[sr >= 0]] = np.nonzero(sr >= 0)[0] // E
+    for h in range(2):
+        same = np.array([np.array_equal(got_sets[0][h][i], want_sets[0][h][i])
+                         for i in range(geo.n_tiles)])
+        rows = same[tile_of]
+        assert_attn_close(got[:, rows, h], want[:, rows, h], f"module {kind} head {h}")

@@ -234,3 +234,34 @@ def test_bsa_full_size(structured):
     # oracle's own fp64 scores: the pooled softmax is near uniform, so neighbouring tiles at the cut
     # often differ by less than the 1e-3 relative gap
     assert n_exact >= 0.15 * n_rows
+
+
+@pytest.mark.parametrize("mode", ["topk", "bsa", "mask", "packed"])
+def test_launch_count_matches_the_launch_code(mode):
+    """The bench's per-stage kernel count, taken with the profiler, equals the table read off the
+    launch code (which the bench reports when the profiler cannot trace)."""
+    import bench
+    from block_sparse_video_tile3d_b200 import packed as P
+    if mode == "packed":
+        mod = P.PackedTileSparseAttention([40, (8, 8, 8), (4, 8, 12)], heads=2, D=64,
+                                          tile_size=128, sparsity=0.5, ref_keep_rate=0.5)
+        rows = mod.geo.rows
+        q, k, v = (torch.randn((1, rows, 2, 64), device="cuda").to(torch.bfloat16)
+                   for _ in range(3))
+        stages = mod.stages(q, k, v, torch.empty_like(q))
+        table = {n: bench.STATIC_KERNELS["attention_packed" if n == "attention" else n]
+                 for n, _ in stages}
+    else:
+        w = workloads.WORKLOADS["tiny"]
+        kw = {"topk": {"topk": w.k}, "bsa": {"mass": 0.9, "min_k": 2, "cos_thresh": 0.5},
+              "mask": {"mask": workloads.block_mask(w.with_(mask="sliding", mode="mask"))}}[mode]
+        m = TileSparseAttention(w.B, w.T, w.H, w.W, w.heads, w.D, mode=mode, **kw)
+        q, k, v = (x.cuda() for x in workloads.make_qkv(w))
+        stages = m.stages(q, k, v)
+        table = {n: bench.STATIC_KERNELS[n] for n, _ in stages}
+    for _, launch in stages:
+        launch()
+    torch.cuda.synchronize()
+    counts, source = bench.count_launches(stages, packed=(mode == "packed"))
+    assert source.startswith("torch.profiler"), source
+    assert counts == table
