@@ -53,7 +53,11 @@ __device__ __forceinline__ void bwd_fail(int* abort, int32_t* status) {
 }
 
 // ------------------------------------------------------------------------------------ prep
-// Grid (nT, heads, B), 256 threads. Rows are accumulated in fp32 in shared memory.
+// Grid (nT, heads, B), 256 threads. A tile without pruned rows (the common case) goes through
+// registers in 16-byte chunks: dOe = dO on valid rows, zero on pad rows, and delta from the
+// chunk's eight products summed over the row's chunks by shuffles. A tile with pruned rows
+// accumulates rows in fp32 in shared memory, one column per thread with rows in order, so the
+// sums are deterministic.
 template <int kD>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(Geo g, const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dout,
@@ -61,6 +65,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(Geo g, const __nv_bfloat1
                                                        const uint8_t* __restrict__ src_row,
                                                        __nv_bfloat16* __restrict__ dout_eff,
                                                        float* __restrict__ delta) {
+  constexpr int kChunks = kD / 8;             // 16-byte chunks of a row
+  constexpr int kRowsPerPass = 256 / kChunks;  // rows one pass of the block covers
   __shared__ float acc[kTileElems][kD + 1];
   __shared__ int target[kTileElems];  // row whose gradient a row's dO adds to (-1: none)
   const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -69,6 +75,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(Geo g, const __nv_bfloat1
   const long ld = (long)g.heads_total * kD;
   const long base = ((long)b * g.Lp + (long)i * kTileElems) * ld + (long)(g.head0 + h) * kD;
   const long blk = ((long)b * g.heads + h) * g.nT + i;
+  bool moved = false;  // this row's dO goes to another row
   if (tid < kTileElems) {
     int t = tid < vc ? tid : -1;
     if (t >= 0 && keep != nullptr && keep[blk * kTileElems + tid] == 0) {
@@ -76,6 +83,36 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(Geo g, const __nv_bfloat1
       t = sr < kTileElems ? sr : tid;
     }
     target[tid] = t;
+    moved = t >= 0 && t != tid;
+  }
+  if (!__syncthreads_or(moved)) {
+    const int c = tid % kChunks, r0 = tid / kChunks;
+    uint4 dv[kTileElems / kRowsPerPass], ov[kTileElems / kRowsPerPass];
+#pragma unroll
+    for (int p = 0; p < kTileElems / kRowsPerPass; ++p) {  // every load in flight first
+      const long at = base + (long)(r0 + p * kRowsPerPass) * ld + 8 * c;
+      dv[p] = *reinterpret_cast<const uint4*>(dout + at);
+      ov[p] = *reinterpret_cast<const uint4*>(o + at);
+    }
+#pragma unroll
+    for (int p = 0; p < kTileElems / kRowsPerPass; ++p) {
+      const int r = r0 + p * kRowsPerPass;
+      if (r >= vc) dv[p] = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(dout_eff + base + (long)r * ld + 8 * c) = dv[p];
+      const __nv_bfloat162* x = reinterpret_cast<const __nv_bfloat162*>(&dv[p]);
+      const __nv_bfloat162* y = reinterpret_cast<const __nv_bfloat162*>(&ov[p]);
+      float sum = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 xf = __bfloat1622float2(x[e]), yf = __bfloat1622float2(y[e]);
+        sum = fmaf(xf.x, yf.x, sum);
+        sum = fmaf(xf.y, yf.y, sum);
+      }
+#pragma unroll
+      for (int off = kChunks / 2; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+      if (c == 0) delta[blk * kTileElems + r] = sum;
+    }
+    return;
   }
   for (int e = tid; e < kTileElems * kD; e += 256) acc[e / kD][e % kD] = 0.f;
   __syncthreads();
@@ -380,8 +417,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const float lse0 = a.lse[rowbase + r0] * kLog2e, lse1 = a.lse[rowbase + r1] * kLog2e;
       const float dl0 = a.delta[rowbase + r0], dl1 = a.delta[rowbase + r1];
+      // key tiles of the next step, loaded one step ahead
+      int na = 0 < cnt ? list[0] : -1, nb = 1 < cnt ? list[1] : -1;
       for (int n = 0; n < np; ++n, ++gp) {
-        const int ja = 2 * n < cnt ? list[2 * n] : -1, jb = 2 * n + 1 < cnt ? list[2 * n + 1] : -1;
+        const int ja = na, jb = nb;
+        na = 2 * n + 2 < cnt ? list[2 * n + 2] : -1;
+        nb = 2 * n + 3 < cnt ? list[2 * n + 3] : -1;
         if (!mbar_wait(&s.s_full, (uint32_t)(gp & 1), abort_flag, lim)) give_up();
         tc_fence_after();
         uint32_t sv[64], pv[64];
@@ -683,22 +724,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         continue;
       }
       const bool key0 = r0 < vcj, key1 = r1 < vcj;
-      for (int n = 0; n < cnt; ++n, ++gs) {
-        int i = list[n];
-        if (i < 0 || i >= g.nT) i = 0;  // unreachable: lists come from in-range entries
+      // A step's query tile and the lse, delta and keep flags of this thread's 16 query columns
+      // are loaded one step ahead (and the list entry two steps ahead), so that no step waits on
+      // a chain of global loads.
+      auto tile_at = [&](int n) {
+        const int i = n < cnt ? list[n] : 0;
+        return (i < 0 || i >= g.nT) ? 0 : i;  // out-of-range: unreachable, lists are in range
+      };
+      struct Meta {
+        int i;
+        float l[16], d[16];
+        uint8_t k[16];
+      };
+      auto fetch = [&](int i, Meta& m) {
+        m.i = i;
         const long qrow = ((long)bh * g.nT + i) * kTileElems;  // [B, heads, Lp] index of row 0
-        const int vci = s.vc[i];
-        // lse (log2 units) and delta of this thread's 16 query columns; -inf lse masks a column
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const long qc = qrow + 8 * (c >> 1) + 2 * t0 + (c & 1);
+          m.l[c] = a.lse[qc];
+          m.d[c] = a.delta[qc];
+          m.k[c] = a.keep != nullptr ? a.keep[qc] : (uint8_t)1;
+        }
+      };
+      Meta nxt;
+      fetch(tile_at(0), nxt);
+      int i_ahead = tile_at(1);
+      for (int n = 0; n < cnt; ++n, ++gs) {
+        const Meta cur = nxt;
+        if (n + 1 < cnt) fetch(i_ahead, nxt);
+        i_ahead = tile_at(n + 2);
+        const int vci = s.vc[cur.i];
+        // lse (log2 units) and delta of this thread's 16 query columns; +inf lse masks a column
         float lq[16], dq[16];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int qc = 8 * jj + 2 * t0 + e;
-            const bool live = qc < vci && (a.keep == nullptr || a.keep[qrow + qc] != 0);
-            lq[2 * jj + e] = live ? a.lse[qrow + qc] * kLog2e : INFINITY;
-            dq[2 * jj + e] = live ? a.delta[qrow + qc] : 0.f;
-          }
+        for (int c = 0; c < 16; ++c) {
+          const int qc = 8 * (c >> 1) + 2 * t0 + (c & 1);
+          const bool live = qc < vci && cur.k[c] != 0;
+          lq[c] = live ? cur.l[c] * kLog2e : INFINITY;
+          dq[c] = live ? cur.d[c] : 0.f;
         }
         if (!mbar_wait(&s.s_full, (uint32_t)(gs & 1), abort_flag, lim)) give_up();
         tc_fence_after();
