@@ -28,7 +28,8 @@
 //                     S^T = K.Q^T and dP^T = V.dOe^T into TMEM, the softmax warps form P^T and
 //                     dS^T as bf16 in TMEM, then dV += P^T.dOe and dK += dS^T.Q.
 // Both contraction kernels are persistent (one CTA per SM, units in static round robin) with one
-// TMA producer thread, one MMA issuer thread and one softmax warpgroup; every wait is bounded as
+// TMA producer thread, two MMA issuer threads (the step's two products; the two accumulations)
+// and one softmax warpgroup; every wait is bounded as
 // in the forward kernel (on a timeout: T3D_DEV_TIMEOUT, drain, free TMEM, return).
 #include "kernels.h"
 #include "sm100.cuh"
@@ -39,7 +40,7 @@ namespace {
 using namespace sm100;
 
 constexpr uint32_t kTileBytes = 64 * 128;  // 64 rows x 128 B: one 64-element column block
-constexpr int kBwdThreads = 256;           // warp 0 producer, warp 1 MMA, warps 4..7 softmax
+constexpr int kBwdThreads = 256;  // warp 0 producer, warps 1 and 2 MMA issuers, warps 4..7 softmax
 constexpr int kTeardown = 1;               // named barrier of all threads before TMEM is freed
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -200,7 +201,7 @@ struct alignas(1024) DqSmem {
   uint64_t s_full, s_empty;    // S and dP of a step in TMEM / read by the softmax
   uint64_t ds_full, ds_empty;  // dS of a step in TMEM / read by its dQ MMAs
   uint64_t dq_full, dq_empty;  // a unit's dQ complete / read by the epilogue
-  uint64_t drain;
+  uint64_t drain[2];           // every MMA of the S / dP issuer, of the dQ issuer, complete
   uint8_t vc[kMaxTiles];
   uint32_t tmem_base;
   int abort;
@@ -250,7 +251,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&s.ds_empty, 1);
     mbar_init(&s.dq_full, 1);
     mbar_init(&s.dq_empty, 128);
-    mbar_init(&s.drain, 1);
+    mbar_init(&s.drain[0], 1);
+    mbar_init(&s.drain[1], 1);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -320,42 +322,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (nq > 0) mbar_wait(&s.q_full, (uint32_t)((nq - 1) & 1), nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------- S and dP issuer
+    // S / dP and dQ have one issuing thread each (as in the forward kernel): an mbarrier wait in
+    // the thread that issues MMAs lets its queued MMAs drain first, and the other thread's queued
+    // MMAs keep the pipe busy meanwhile.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(64, 128, false, false);
-      constexpr uint32_t idesc_q = idesc_bf16(64, kD, false, true);
       const uint64_t dq_ = sdesc_sw128(smem_u32(s.q), 16, 1024);
       const uint64_t ddo = sdesc_sw128(smem_u32(s.dout), 16, 1024);
       const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
       const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 16, 1024);
-      const uint64_t dkm = sdesc_sw128(smem_u32(s.k[0]), 2 * kTileBytes, 1024);  // K pair, MN-major
       long gp = 0;
       int active = 0;
       bool ok = true;
-      // dQ += dS(step) . K_pair(step); the unit's first one overwrites dQ once it has been read.
-      auto issue_dq = [&](long step, int n_in_unit) -> bool {
-        const int st = (int)(step % C::kStages);
-        if ((n_in_unit == 0 &&
-             !mbar_wait(&s.dq_empty, (uint32_t)((active & 1) ^ 1), abort_flag, lim)) ||
-            !mbar_wait(&s.ds_full, (uint32_t)(step & 1), abort_flag, lim))
-          return false;
-        tc_fence_after();
-        const uint64_t b0 = dkm + (uint64_t)(st * (C::kPair >> 4));
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)  // 16 keys per MMA
-          mma_bf16_ts(tmem + kDqColDQ, tmem + kDqColDS + 8 * kk, b0 + kk * (2048 >> 4), idesc_q,
-                      (n_in_unit == 0 && kk == 0) ? 0u : 1u);
-        mma_commit(&s.ds_empty);
-        mma_commit(&s.kv_empty[st]);
-        return true;
-      };
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         int cnt;
         const int32_t* list;
         const int np = unit_pairs(u, cnt, list);
         if (np == 0) continue;
         if (!mbar_wait(&s.q_full, (uint32_t)(active & 1), abort_flag, lim)) { ok = false; break; }
-        for (int n = 0; n < np && ok; ++n, ++gp) {
+        for (int n = 0; n < np; ++n, ++gp) {
           const int st = (int)(gp % C::kStages);
           if (!mbar_wait(&s.kv_full[st], (uint32_t)((gp / C::kStages) & 1), abort_flag, lim) ||
               !mbar_wait(&s.s_empty, (uint32_t)((gp & 1) ^ 1), abort_flag, lim)) {
@@ -375,15 +361,51 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           mma_commit(&s.s_full);
           if (n == np - 1) mma_commit(&s.q_empty);
-          if (n > 0 && !issue_dq(gp - 1, n - 1)) { ok = false; break; }
         }
-        if (ok && !issue_dq(gp - 1, np - 1)) ok = false;
+        ++active;
+      }
+      if (!ok) bwd_fail(&s.abort, a.dev_status);
+      mma_commit(&s.drain[0]);
+      mbar_wait(&s.drain[0], 0, nullptr);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------- dQ issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_q = idesc_bf16(64, kD, false, true);
+      const uint64_t dkm = sdesc_sw128(smem_u32(s.k[0]), 2 * kTileBytes, 1024);  // K pair, MN-major
+      long gp = 0;
+      int active = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        int cnt;
+        const int32_t* list;
+        const int np = unit_pairs(u, cnt, list);
+        if (np == 0) continue;
+        for (int n = 0; n < np; ++n, ++gp) {
+          // dQ += dS(step) . K_pair(step); the unit's first one overwrites dQ once the epilogue
+          // has read it. The stage's K and V are free once this completes (its S and dP, which
+          // the softmax read before writing dS, completed earlier).
+          const int st = (int)(gp % C::kStages);
+          if ((n == 0 && !mbar_wait(&s.dq_empty, (uint32_t)((active & 1) ^ 1), abort_flag, lim)) ||
+              !mbar_wait(&s.ds_full, (uint32_t)(gp & 1), abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t b0 = dkm + (uint64_t)(st * (C::kPair >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)  // 16 keys per MMA
+            mma_bf16_ts(tmem + kDqColDQ, tmem + kDqColDS + 8 * kk, b0 + kk * (2048 >> 4), idesc_q,
+                        (n == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(&s.ds_empty);
+          mma_commit(&s.kv_empty[st]);
+        }
         if (ok) mma_commit(&s.dq_full);
         ++active;
       }
       if (!ok) bwd_fail(&s.abort, a.dev_status);
-      mma_commit(&s.drain);
-      mbar_wait(&s.drain, 0, nullptr);
+      mma_commit(&s.drain[1]);
+      mbar_wait(&s.drain[1], 0, nullptr);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax and epilogue
@@ -521,7 +543,7 @@ struct alignas(1024) KvSmem {
   uint64_t s_full, s_empty;    // S^T and dP^T of a step in TMEM / read by the softmax
   uint64_t p_full, p_empty;    // P^T and dS^T of a step in TMEM / read by their MMAs
   uint64_t acc_full, acc_empty;  // a unit's dK and dV complete / read by the epilogue
-  uint64_t drain;
+  uint64_t drain[2];             // every MMA of the S / dP issuer, of the dK / dV issuer, complete
   uint8_t vc[kMaxTiles];
   uint32_t tmem_base;
   int abort;
@@ -555,7 +577,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(&s.p_empty, 1);
     mbar_init(&s.acc_full, 1);
     mbar_init(&s.acc_empty, 128);
-    mbar_init(&s.drain, 1);
+    mbar_init(&s.drain[0], 1);
+    mbar_init(&s.drain[1], 1);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -618,48 +641,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (nk > 0) mbar_wait(&s.kv_full, (uint32_t)((nk - 1) & 1), nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+    // ------------------------------------------------------------- S^T and dP^T issuer
+    // As in the dQ kernel, the two products of a step and the two accumulations have one issuing
+    // thread each.
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(64, 64, false, false);
-      constexpr uint32_t idesc_acc = idesc_bf16(64, kD, false, true);
       const uint64_t dkd = sdesc_sw128(smem_u32(s.k), 16, 1024);
       const uint64_t dvd = sdesc_sw128(smem_u32(s.v), 16, 1024);
       const uint64_t dq0 = sdesc_sw128(smem_u32(s.q[0]), 16, 1024);
       const uint64_t ddo0 = sdesc_sw128(smem_u32(s.dout[0]), 16, 1024);
-      const uint64_t dqm0 = sdesc_sw128(smem_u32(s.q[0]), kTileBytes, 1024);     // MN-major
-      const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0]), kTileBytes, 1024);  // MN-major
       long gs = 0;
       int active = 0;
       bool ok = true;
-      // dV += P^T(step) . dOe(step) and dK += dS^T(step) . Q(step); the unit's first ones
-      // overwrite the accumulators once the epilogue has read them.
-      auto issue_acc = [&](long step, int n_in_unit) -> bool {
-        const int st = (int)(step % C::kStages);
-        if ((n_in_unit == 0 &&
-             !mbar_wait(&s.acc_empty, (uint32_t)((active & 1) ^ 1), abort_flag, lim)) ||
-            !mbar_wait(&s.p_full, (uint32_t)(step & 1), abort_flag, lim))
-          return false;
-        tc_fence_after();
-        const uint64_t bq = dqm0 + (uint64_t)(st * (C::kOne >> 4));
-        const uint64_t bdo = ddom0 + (uint64_t)(st * (C::kOne >> 4));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // 16 query rows per MMA
-          const uint32_t accum = (n_in_unit == 0 && kk == 0) ? 0u : 1u;
-          mma_bf16_ts(tmem + kKvColDV, tmem + kKvColP + 8 * kk, bdo + kk * (2048 >> 4), idesc_acc,
-                      accum);
-          mma_bf16_ts(tmem + kKvColDK, tmem + kKvColDS + 8 * kk, bq + kk * (2048 >> 4), idesc_acc,
-                      accum);
-        }
-        mma_commit(&s.p_empty);
-        mma_commit(&s.qd_empty[st]);
-        return true;
-      };
       for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
         const int32_t* list;
         const int cnt = unit_list(u, list);
         if (cnt == 0) continue;
         if (!mbar_wait(&s.kv_full, (uint32_t)(active & 1), abort_flag, lim)) { ok = false; break; }
-        for (int n = 0; n < cnt && ok; ++n, ++gs) {
+        for (int n = 0; n < cnt; ++n, ++gs) {
           const int st = (int)(gs % C::kStages);
           if (!mbar_wait(&s.qd_full[st], (uint32_t)((gs / C::kStages) & 1), abort_flag, lim) ||
               !mbar_wait(&s.s_empty, (uint32_t)((gs & 1) ^ 1), abort_flag, lim)) {
@@ -677,18 +676,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mma_bf16(tmem + kKvColDP, dvd + o, dob + o, idesc_s, kk ? 1u : 0u);
           }
           mma_commit(&s.s_full);
-          if (n > 0 && !issue_acc(gs - 1, n - 1)) { ok = false; break; }
         }
-        if (ok && !issue_acc(gs - 1, cnt - 1)) ok = false;
-        if (ok) {
-          mma_commit(&s.kv_empty);
-          mma_commit(&s.acc_full);
-        }
+        if (ok) mma_commit(&s.kv_empty);  // only these MMAs read the unit's K and V
         ++active;
       }
       if (!ok) bwd_fail(&s.abort, a.dev_status);
-      mma_commit(&s.drain);
-      mbar_wait(&s.drain, 0, nullptr);
+      mma_commit(&s.drain[0]);
+      mbar_wait(&s.drain[0], 0, nullptr);
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------- dV and dK issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_acc = idesc_bf16(64, kD, false, true);
+      const uint64_t dqm0 = sdesc_sw128(smem_u32(s.q[0]), kTileBytes, 1024);     // MN-major
+      const uint64_t ddom0 = sdesc_sw128(smem_u32(s.dout[0]), kTileBytes, 1024);  // MN-major
+      long gs = 0;
+      int active = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < total_units && ok; u += gridDim.x) {
+        const int32_t* list;
+        const int cnt = unit_list(u, list);
+        if (cnt == 0) continue;
+        for (int n = 0; n < cnt; ++n, ++gs) {
+          // dV += P^T(step) . dOe(step) and dK += dS^T(step) . Q(step); the unit's first ones
+          // overwrite the accumulators once the epilogue has read them. The stage's Q and dOe are
+          // free once these complete (the step's S^T and dP^T completed earlier).
+          const int st = (int)(gs % C::kStages);
+          if ((n == 0 && !mbar_wait(&s.acc_empty, (uint32_t)((active & 1) ^ 1), abort_flag, lim)) ||
+              !mbar_wait(&s.p_full, (uint32_t)(gs & 1), abort_flag, lim)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bq = dqm0 + (uint64_t)(st * (C::kOne >> 4));
+          const uint64_t bdo = ddom0 + (uint64_t)(st * (C::kOne >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // 16 query rows per MMA
+            const uint32_t accum = (n == 0 && kk == 0) ? 0u : 1u;
+            mma_bf16_ts(tmem + kKvColDV, tmem + kKvColP + 8 * kk, bdo + kk * (2048 >> 4),
+                        idesc_acc, accum);
+            mma_bf16_ts(tmem + kKvColDK, tmem + kKvColDS + 8 * kk, bq + kk * (2048 >> 4),
+                        idesc_acc, accum);
+          }
+          mma_commit(&s.p_empty);
+          mma_commit(&s.qd_empty[st]);
+        }
+        if (ok) mma_commit(&s.acc_full);
+        ++active;
+      }
+      if (!ok) bwd_fail(&s.abort, a.dev_status);
+      mma_commit(&s.drain[1]);
+      mbar_wait(&s.drain[1], 0, nullptr);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax and epilogue
