@@ -25,8 +25,9 @@
 //                     S = Q.K^T and dP = dOe.V^T into TMEM, the softmax warps form dS as bf16 in
 //                     TMEM, then dQ += dS.K (A = dS from TMEM, B = the K pair, MN-major);
 //   bwd_dkdv_kernel   per key tile (M = 64 keys) over the query tiles of its list (N = 64):
-//                     S^T = K.Q^T and dP^T = V.dOe^T into TMEM, the softmax warps form P^T and
-//                     dS^T as bf16 in TMEM, then dV += P^T.dOe and dK += dS^T.Q.
+//                     S^T = K.Q^T and dP^T = V.dOe^T into one of two TMEM buffers, the softmax
+//                     warps write P^T and dS^T as bf16 over them, then dV += P^T.dOe and
+//                     dK += dS^T.Q; the next step's products go to the other buffer meanwhile.
 // Both contraction kernels are persistent (one CTA per SM, units in static round robin) with one
 // TMA producer thread, two MMA issuer threads (the step's two products; the two accumulations)
 // and one softmax warpgroup; every wait is bounded as
@@ -540,8 +541,9 @@ struct alignas(1024) KvSmem {
   uint8_t v[C::kOne];
   uint64_t qd_full[C::kStages], qd_empty[C::kStages];
   uint64_t kv_full, kv_empty;  // the unit's K and V tiles landed / no longer read
-  uint64_t s_full, s_empty;    // S^T and dP^T of a step in TMEM / read by the softmax
-  uint64_t p_full, p_empty;    // P^T and dS^T of a step in TMEM / read by their MMAs
+  uint64_t s_full[2];    // S^T and dP^T of a step in TMEM buffer b (steps alternate buffers)
+  uint64_t p_full[2];    // P^T and dS^T of that step written over them by the softmax
+  uint64_t buf_free[2];  // the dV / dK MMAs that read buffer b have completed
   uint64_t acc_full, acc_empty;  // a unit's dK and dV complete / read by the epilogue
   uint64_t drain[2];             // every MMA of the S / dP issuer, of the dK / dV issuer, complete
   uint8_t vc[kMaxTiles];
@@ -549,8 +551,10 @@ struct alignas(1024) KvSmem {
   int abort;
 };
 
-constexpr uint32_t kKvColS = 0, kKvColDP = 64, kKvColP = 128, kKvColDS = 160, kKvColDV = 256,
-                   kKvColDK = 384;
+// TMEM columns: S^T of buffers 0 / 1 at 0 / 64, dP^T at 128 / 192 (fp32, 64 query columns each);
+// P^T and dS^T (bf16 pairs, 32 columns) are written over the first half of their step's S^T and
+// dP^T once the softmax has read them; dV and dK accumulate at 256 and 384.
+constexpr uint32_t kKvColS = 0, kKvColDP = 128, kKvBuf = 64, kKvColDV = 256, kKvColDK = 384;
 
 template <int kD>
 __global__ void __launch_bounds__(kBwdThreads, 1)
@@ -571,10 +575,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(&s.kv_full, 1);
     mbar_init(&s.kv_empty, 1);
-    mbar_init(&s.s_full, 1);
-    mbar_init(&s.s_empty, 128);
-    mbar_init(&s.p_full, 128);
-    mbar_init(&s.p_empty, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.p_full[t], 128);
+      mbar_init(&s.buf_free[t], 1);
+    }
     mbar_init(&s.acc_full, 1);
     mbar_init(&s.acc_empty, 128);
     mbar_init(&s.drain[0], 1);
@@ -659,23 +664,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (cnt == 0) continue;
         if (!mbar_wait(&s.kv_full, (uint32_t)(active & 1), abort_flag, lim)) { ok = false; break; }
         for (int n = 0; n < cnt; ++n, ++gs) {
+          // Step gs uses TMEM buffer gs & 1, free once the dV / dK MMAs of step gs - 2 are done.
           const int st = (int)(gs % C::kStages);
+          const int bf = (int)(gs & 1);
           if (!mbar_wait(&s.qd_full[st], (uint32_t)((gs / C::kStages) & 1), abort_flag, lim) ||
-              !mbar_wait(&s.s_empty, (uint32_t)((gs & 1) ^ 1), abort_flag, lim)) {
+              !mbar_wait(&s.buf_free[bf], (uint32_t)(((gs >> 1) & 1) ^ 1), abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t qb = dq0 + (uint64_t)(st * (C::kOne >> 4));
           const uint64_t dob = ddo0 + (uint64_t)(st * (C::kOne >> 4));
+          const uint32_t d_s = tmem + kKvColS + kKvBuf * bf, d_dp = tmem + kKvColDP + kKvBuf * bf;
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const int hh = kk >> 2, sub = kk & 3;
             const uint64_t o = (uint64_t)((hh * kTileBytes + sub * 32) >> 4);
-            mma_bf16(tmem + kKvColS, dkd + o, qb + o, idesc_s, kk ? 1u : 0u);
-            mma_bf16(tmem + kKvColDP, dvd + o, dob + o, idesc_s, kk ? 1u : 0u);
+            mma_bf16(d_s, dkd + o, qb + o, idesc_s, kk ? 1u : 0u);
+            mma_bf16(d_dp, dvd + o, dob + o, idesc_s, kk ? 1u : 0u);
           }
-          mma_commit(&s.s_full);
+          mma_commit(&s.s_full[bf]);
         }
         if (ok) mma_commit(&s.kv_empty);  // only these MMAs read the unit's K and V
         ++active;
@@ -702,23 +710,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           // overwrite the accumulators once the epilogue has read them. The stage's Q and dOe are
           // free once these complete (the step's S^T and dP^T completed earlier).
           const int st = (int)(gs % C::kStages);
+          const int bf = (int)(gs & 1);
           if ((n == 0 && !mbar_wait(&s.acc_empty, (uint32_t)((active & 1) ^ 1), abort_flag, lim)) ||
-              !mbar_wait(&s.p_full, (uint32_t)(gs & 1), abort_flag, lim)) {
+              !mbar_wait(&s.p_full[bf], (uint32_t)((gs >> 1) & 1), abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint64_t bq = dqm0 + (uint64_t)(st * (C::kOne >> 4));
           const uint64_t bdo = ddom0 + (uint64_t)(st * (C::kOne >> 4));
+          const uint32_t a_p = tmem + kKvColS + kKvBuf * bf, a_ds = tmem + kKvColDP + kKvBuf * bf;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // 16 query rows per MMA
             const uint32_t accum = (n == 0 && kk == 0) ? 0u : 1u;
-            mma_bf16_ts(tmem + kKvColDV, tmem + kKvColP + 8 * kk, bdo + kk * (2048 >> 4),
-                        idesc_acc, accum);
-            mma_bf16_ts(tmem + kKvColDK, tmem + kKvColDS + 8 * kk, bq + kk * (2048 >> 4),
-                        idesc_acc, accum);
+            mma_bf16_ts(tmem + kKvColDV, a_p + 8 * kk, bdo + kk * (2048 >> 4), idesc_acc, accum);
+            mma_bf16_ts(tmem + kKvColDK, a_ds + 8 * kk, bq + kk * (2048 >> 4), idesc_acc, accum);
           }
-          mma_commit(&s.p_empty);
+          mma_commit(&s.buf_free[bf]);
           mma_commit(&s.qd_empty[st]);
         }
         if (ok) mma_commit(&s.acc_full);
@@ -802,14 +810,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           lq[c] = live ? cur.l[c] * kLog2e : INFINITY;
           dq[c] = live ? cur.d[c] : 0.f;
         }
-        if (!mbar_wait(&s.s_full, (uint32_t)(gs & 1), abort_flag, lim)) give_up();
+        const int bf = (int)(gs & 1);
+        const uint32_t t_s = lane_base + kKvColS + kKvBuf * bf;
+        const uint32_t t_dp = lane_base + kKvColDP + kKvBuf * bf;
+        if (!mbar_wait(&s.s_full[bf], (uint32_t)((gs >> 1) & 1), abort_flag, lim)) give_up();
         tc_fence_after();
         uint32_t sv[32], pv[32];
-        tmem_ld_16x256b_x8(lane_base + kKvColS, sv);
-        tmem_ld_16x256b_x8(lane_base + kKvColDP, pv);
+        tmem_ld_16x256b_x8(t_s, sv);
+        tmem_ld_16x256b_x8(t_dp, pv);
         tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&s.s_empty);
         uint32_t pw[16], dw[16];
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
@@ -831,13 +840,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           dw[2 * jj] = *reinterpret_cast<const uint32_t*>(&d0);
           dw[2 * jj + 1] = *reinterpret_cast<const uint32_t*>(&d1);
         }
-        if (!mbar_wait(&s.p_empty, (uint32_t)((gs & 1) ^ 1), abort_flag, lim)) give_up();
-        tc_fence_after();
-        tmem_st_16x128b_x8(lane_base + kKvColP, pw);
-        tmem_st_16x128b_x8(lane_base + kKvColDS, dw);
+        // Written over the S^T and dP^T just read (no other reader: the buffer's next MMAs wait
+        // for the dV / dK MMAs of this step).
+        tmem_st_16x128b_x8(t_s, pw);
+        tmem_st_16x128b_x8(t_dp, dw);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&s.p_full);
+        mbar_arrive(&s.p_full[bf]);
       }
       // ---- epilogue: dV and scale * dK for the valid key rows, zero for pad rows
       if (!mbar_wait(&s.acc_full, (uint32_t)(active & 1), abort_flag, lim)) give_up();
