@@ -29,8 +29,8 @@
 //                     warps write P^T and dS^T as bf16 over them, then dV += P^T.dOe and
 //                     dK += dS^T.Q; the next step's products go to the other buffer meanwhile.
 // Both contraction kernels are persistent (one CTA per SM, units in static round robin) with one
-// TMA producer thread, two MMA issuer threads (the step's two products; the two accumulations)
-// and one softmax warpgroup; every wait is bounded as
+// TMA producer thread, MMA issuer threads (dQ: S, dP and dQ one each; dK/dV: the step's two
+// products, the two accumulations) and one softmax warpgroup; every wait is bounded as
 // in the forward kernel (on a timeout: T3D_DEV_TIMEOUT, drain, free TMEM, return).
 #include "kernels.h"
 #include "sm100.cuh"
@@ -41,7 +41,7 @@ namespace {
 using namespace sm100;
 
 constexpr uint32_t kTileBytes = 64 * 128;  // 64 rows x 128 B: one 64-element column block
-constexpr int kBwdThreads = 256;  // warp 0 producer, warps 1 and 2 MMA issuers, warps 4..7 softmax
+constexpr int kBwdThreads = 256;  // warp 0 producer, warps 1-3 MMA issuers, warps 4..7 softmax
 constexpr int kTeardown = 1;               // named barrier of all threads before TMEM is freed
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -198,11 +198,11 @@ struct alignas(1024) DqSmem {
   uint8_t q[C::kOne];
   uint8_t dout[C::kOne];
   uint64_t kv_full[C::kStages], kv_empty[C::kStages];
-  uint64_t q_full, q_empty;    // the unit's Q and dOe tiles landed / no longer read
-  uint64_t s_full, s_empty;    // S and dP of a step in TMEM / read by the softmax
+  uint64_t q_full, q_empty;    // the unit's Q and dOe tiles landed / read by its last S and dP
+  uint64_t s_full[2], s_empty[2];  // S ([0]) and dP ([1]) of a step in TMEM / read by the softmax
   uint64_t ds_full, ds_empty;  // dS of a step in TMEM / read by its dQ MMAs
   uint64_t dq_full, dq_empty;  // a unit's dQ complete / read by the epilogue
-  uint64_t drain[2];           // every MMA of the S / dP issuer, of the dQ issuer, complete
+  uint64_t drain[3];           // every MMA of the S, the dQ, the dP issuer complete
   uint8_t vc[kMaxTiles];
   uint32_t tmem_base;
   int abort;
@@ -245,15 +245,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&s.kv_empty[t], 1);
     }
     mbar_init(&s.q_full, 1);
-    mbar_init(&s.q_empty, 1);
-    mbar_init(&s.s_full, 1);
-    mbar_init(&s.s_empty, 128);
+    mbar_init(&s.q_empty, 2);  // one commit from each of the S and dP issuers
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s.s_full[t], 1);
+      mbar_init(&s.s_empty[t], 128);
+    }
     mbar_init(&s.ds_full, 128);
     mbar_init(&s.ds_empty, 1);
     mbar_init(&s.dq_full, 1);
     mbar_init(&s.dq_empty, 128);
-    mbar_init(&s.drain[0], 1);
-    mbar_init(&s.drain[1], 1);
+    for (int t = 0; t < 3; ++t) mbar_init(&s.drain[t], 1);
     s.abort = 0;
     fence_mbar_init();
   }
@@ -322,17 +323,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (t >= 0) mbar_wait(&s.kv_full[t % C::kStages], (uint32_t)((t / C::kStages) & 1), nullptr);
       if (nq > 0) mbar_wait(&s.q_full, (uint32_t)((nq - 1) & 1), nullptr);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- S and dP issuer
-    // S / dP and dQ have one issuing thread each (as in the forward kernel): an mbarrier wait in
-    // the thread that issues MMAs lets its queued MMAs drain first, and the other thread's queued
-    // MMAs keep the pipe busy meanwhile.
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------- S issuer (warp 1), dP issuer (3)
+    // S, dP and dQ have one issuing thread each (as in the forward kernel): an mbarrier wait in
+    // the thread that issues MMAs lets its queued MMAs drain first, and the other threads' queued
+    // MMAs keep the pipe busy meanwhile. S and dP complete separately, so the softmax forms P
+    // while dP is computed, and each product's buffer is free once the softmax has read it.
     if (lane == 0) {
+      const int which = warp == 1 ? 0 : 1;  // 0: S = Q . K_pair^T, 1: dP = dOe . V_pair^T
       constexpr uint32_t idesc_s = idesc_bf16(64, 128, false, false);
-      const uint64_t dq_ = sdesc_sw128(smem_u32(s.q), 16, 1024);
-      const uint64_t ddo = sdesc_sw128(smem_u32(s.dout), 16, 1024);
-      const uint64_t dk = sdesc_sw128(smem_u32(s.k[0]), 16, 1024);
-      const uint64_t dv = sdesc_sw128(smem_u32(s.v[0]), 16, 1024);
+      const uint64_t da = sdesc_sw128(smem_u32(which ? s.dout : s.q), 16, 1024);
+      const uint64_t db = sdesc_sw128(smem_u32(which ? s.v[0] : s.k[0]), 16, 1024);
+      const uint32_t d_acc = tmem + (which ? kDqColDP : kDqColS);
       long gp = 0;
       int active = 0;
       bool ok = true;
@@ -345,29 +347,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int n = 0; n < np; ++n, ++gp) {
           const int st = (int)(gp % C::kStages);
           if (!mbar_wait(&s.kv_full[st], (uint32_t)((gp / C::kStages) & 1), abort_flag, lim) ||
-              !mbar_wait(&s.s_empty, (uint32_t)((gp & 1) ^ 1), abort_flag, lim)) {
+              !mbar_wait(&s.s_empty[which], (uint32_t)((gp & 1) ^ 1), abort_flag, lim)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t kb = dk + (uint64_t)(st * (C::kPair >> 4));
-          const uint64_t vb = dv + (uint64_t)(st * (C::kPair >> 4));
+          const uint64_t b0 = db + (uint64_t)(st * (C::kPair >> 4));
 #pragma unroll
           for (int kk = 0; kk < kD / 16; ++kk) {
             const int hh = kk >> 2, sub = kk & 3;
             const uint64_t ao = (uint64_t)((hh * kTileBytes + sub * 32) >> 4);
             const uint64_t bo = (uint64_t)((hh * 2 * kTileBytes + sub * 32) >> 4);
-            mma_bf16(tmem + kDqColS, dq_ + ao, kb + bo, idesc_s, kk ? 1u : 0u);
-            mma_bf16(tmem + kDqColDP, ddo + ao, vb + bo, idesc_s, kk ? 1u : 0u);
+            mma_bf16(d_acc, da + ao, b0 + bo, idesc_s, kk ? 1u : 0u);
           }
-          mma_commit(&s.s_full);
+          mma_commit(&s.s_full[which]);
           if (n == np - 1) mma_commit(&s.q_empty);
         }
         ++active;
       }
       if (!ok) bwd_fail(&s.abort, a.dev_status);
-      mma_commit(&s.drain[0]);
-      mbar_wait(&s.drain[0], 0, nullptr);
+      mma_commit(&s.drain[which ? 2 : 0]);
+      mbar_wait(&s.drain[which ? 2 : 0], 0, nullptr);
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------- dQ issuer
@@ -446,16 +446,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int ja = na, jb = nb;
         na = 2 * n + 2 < cnt ? list[2 * n + 2] : -1;
         nb = 2 * n + 3 < cnt ? list[2 * n + 3] : -1;
-        if (!mbar_wait(&s.s_full, (uint32_t)(gp & 1), abort_flag, lim)) give_up();
+        const int ca = (ja >= 0 && ja < g.nT) ? s.vc[ja] : 0;
+        const int cb = (jb >= 0 && jb < g.nT) ? s.vc[jb] : 0;
+        // P from S while dP is still being computed
+        if (!mbar_wait(&s.s_full[0], (uint32_t)(gp & 1), abort_flag, lim)) give_up();
         tc_fence_after();
         uint32_t sv[64], pv[64];
         tmem_ld_16x256b_x16(lane_base + kDqColS, sv);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&s.s_empty[0]);
+        float pr[64];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = 8 * j + 2 * t0 + (e & 1);
+            const bool valid = key < 64 ? key < ca : key - 64 < cb;
+            const float lse = e < 2 ? lse0 : lse1;
+            pr[4 * j + e] = valid ? ex2(fmaf(__uint_as_float(sv[4 * j + e]), sl2, -lse)) : 0.f;
+          }
+        }
+        if (!mbar_wait(&s.s_full[1], (uint32_t)(gp & 1), abort_flag, lim)) give_up();
+        tc_fence_after();
         tmem_ld_16x256b_x16(lane_base + kDqColDP, pv);
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(&s.s_empty);
-        const int ca = (ja >= 0 && ja < g.nT) ? s.vc[ja] : 0;
-        const int cb = (jb >= 0 && jb < g.nT) ? s.vc[jb] : 0;
+        mbar_arrive(&s.s_empty[1]);
         // dS = P (dP - delta) as bf16 pairs, in the layout of the forward's P: keys 8j + 2 t0 and
         // + 1 to column 4j + t0 (tcgen05.st 16x128b), two stores of 32 columns.
         uint32_t dsw[2][16];
@@ -464,11 +481,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           float d[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int key = 8 * j + 2 * t0 + (e & 1);
-            const bool valid = key < 64 ? key < ca : key - 64 < cb;
-            const float lse = e < 2 ? lse0 : lse1, dl = e < 2 ? dl0 : dl1;
-            const float p = valid ? ex2(fmaf(__uint_as_float(sv[4 * j + e]), sl2, -lse)) : 0.f;
-            d[e] = p * (__uint_as_float(pv[4 * j + e]) - dl);
+            const float dl = e < 2 ? dl0 : dl1;
+            d[e] = pr[4 * j + e] * (__uint_as_float(pv[4 * j + e]) - dl);
           }
           const __nv_bfloat162 q0 = __floats2bfloat162_rn(d[0], d[1]);
           const __nv_bfloat162 q1 = __floats2bfloat162_rn(d[2], d[3]);
