@@ -184,6 +184,38 @@ __device__ int select_topk_any(const float* row, int n, int k, int32_t* out, int
 }
 
 
+// Exact end of the value search once the bracket [lo, hi) holds c <= 32 of the row's values: the
+// candidates (value v, tile ix) sit one per lane (lanes >= c hold v = -2, below every e). They are
+// sorted by value descending, then tile ascending (a bitonic sort across the lanes), and summed in
+// that order on top of fhi = F(hi), the mass of the tiles above the bracket, until the target is
+// reached. Returns the crossing value; need_eq is how many tiles of that value are taken (the
+// lowest-indexed ones, the tie rule of the emission).
+__device__ float finish_bracket(float v, int ix, int c, float fhi, float target, int& need_eq) {
+  const int lane = threadIdx.x & 31;
+  for (int k = 2; k <= 32; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, v, j);
+      const int oi = __shfl_xor_sync(0xffffffffu, ix, j);
+      const bool first = v > ov || (v == ov && ix < oi);  // this lane's entry comes first
+      const bool lower = (lane & j) == 0, desc = (lane & k) == 0;
+      if ((lower == desc) != first) {
+        v = ov;
+        ix = oi;
+      }
+    }
+  }
+  float x = v >= 0.f ? v : 0.f;  // inclusive prefix sum in sorted order
+  for (int o = 1; o < 32; o <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const unsigned hit = __ballot_sync(0xffffffffu, lane < c && fhi + x >= target);
+  const int js = hit != 0u ? __ffs(hit) - 1 : c - 1;  // rounding: take every candidate
+  const float vs = __shfl_sync(0xffffffffu, v, js);
+  need_eq = __popc(__ballot_sync(0xffffffffu, lane <= js && v == vs));
+  return vs;
+}
+
 // Cumulative-mass selection of one row (one warp). The scores in row[0..nT) are replaced by
 // e_j = exp(scale * (S_j - max S)); tiles are ranked by e (ties: lower index) and the smallest
 // prefix whose sum reaches mass * sum(e) is kept. Writes ascending indices to out and returns the
@@ -192,7 +224,7 @@ __device__ int select_topk_any(const float* row, int n, int k, int32_t* out, int
 // mass_fix_kernel then selects from the score row (that rare path stays out of this kernel, whose
 // register count, and so its occupancy, it would otherwise set).
 __device__ int select_mass_row(float* row, int nT, float scale, float mass, int min_k, int kmax,
-                               int32_t* out, int32_t* dev_status) {
+                               int32_t* out, int32_t* dev_status, float* cv, int* ci) {
   const int lane = threadIdx.x & 31;
   if (mass >= 1.f) {
     // Every probability of a softmax is positive, so the running sum reaches 1 only with the last
@@ -208,37 +240,53 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
   float mx = -INFINITY;
   for (int j = lane; j < nT; j += 32) mx = fmaxf(mx, row[j]);
   mx = warp_max(mx);
-  float tot = 0.f;
+  float tot = 0.f, mn = INFINITY;
   for (int j = lane; j < nT; j += 32) {
     const float e = expf(scale * (row[j] - mx));
     row[j] = e;
     tot += e;
+    mn = fminf(mn, e);
   }
   __syncwarp();
   tot = warp_sum(tot);
+  mn = -warp_max(-mn);
   const float target = mass * tot;
   // Largest key thr with sum_{key >= thr} e >= target: the key of the tile at which the running
   // sum (descending order) first reaches the target. First a search on the values: a bracket
-  // [lo, hi) with F(lo) >= target > F(hi), F(t) = sum of the e >= t, narrowed by interpolating F
-  // linearly (Illinois rule against a stalling end) until exactly one value lies in it — that
-  // value is the crossing tile's, and F(lo) is then the sum of the same tiles in the same order as
-  // the emission below recomputes. Rows where that does not happen within the step budget (ties
+  // [lo, hi) with F(lo) >= target > F(hi), F(t) = sum of the e >= t, starting from the row's
+  // smallest value and just above its largest (1), narrowed by interpolating F linearly (Illinois
+  // rule against a stalling end) until at most 32 values lie in it; those are then ranked and
+  // summed exactly (finish_bracket). Rows where that does not happen within the step budget (ties
   // at the crossing value) take the bit-by-bit key search.
   uint32_t prefix = 0;
   bool found = false;
+  int need_fin = -1;  // need_eq from finish_bracket, when it ran
   {
-    float lo = 0.f, hi = 2.f;  // every e lies in [0, 1]
+    float lo = mn, hi = __int_as_float(0x3f800001);  // every e lies in [mn, 1]
     float Flo = tot, Fhi = 0.f;
     int clo = nT, chi = 0;
     float wlo = 1.f, whi = 1.f;
     int side = 0;
     for (int step = 0; step < 24; ++step) {
-      if (clo - chi == 1) {
-        float v = -1.f;
-        for (int j = lane; j < nT; j += 32)
-          if (row[j] >= lo && row[j] < hi) v = row[j];
-        v = warp_max(v);
-        prefix = float_key(v);
+      if (clo - chi <= 32) {
+        const unsigned lt = lanemask_lt();
+        int base = 0;
+        for (int j0 = 0; j0 < nT; j0 += 32) {
+          const int j = j0 + lane;
+          const bool inb = j < nT && row[j] >= lo && row[j] < hi;
+          const unsigned bb = __ballot_sync(0xffffffffu, inb);
+          if (inb) {
+            cv[base + __popc(bb & lt)] = row[j];
+            ci[base + __popc(bb & lt)] = j;
+          }
+          base += __popc(bb);
+        }
+        __syncwarp();
+        const int c = clo - chi;
+        const float v = lane < c ? cv[lane] : -2.f;
+        const int ix = lane < c ? ci[lane] : 0x7fffffff;
+        __syncwarp();
+        prefix = float_key(finish_bracket(v, ix, c, Fhi, target, need_fin));
         found = true;
         break;
       }
@@ -292,8 +340,8 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
   above = warp_sum(above);
   n_above = warp_sum_int(n_above);
   // Tiles tied at the threshold are taken in ascending index until the target is reached.
-  int need_eq = 0;
-  {
+  int need_eq = need_fin > 0 ? need_fin : 0;
+  if (need_fin < 0) {
     float acc = above;
     bool done = false;
     for (int j0 = 0; j0 < nT && !done; j0 += 32) {
@@ -325,10 +373,12 @@ __device__ int select_mass_row(float* row, int nT, float scale, float mass, int 
 
 // select_mass_row with the row in registers (lane l holds entries l + 32 i, i < KPL): the same
 // operations in the same order, so the same sums and the same selection, without the shared-memory
-// traffic and address arithmetic of every pass. Pads hold -1, below every e.
+// traffic and address arithmetic of every pass. Pads hold -1, below every e. cv / ci: the warp's
+// 32-entry scratch for finish_bracket.
 template <int KPL>
 __device__ int select_mass_row_reg(const float* __restrict__ srow, int nT, float scale, float mass,
-                                   int min_k, int kmax, int32_t* out, int32_t* dev_status) {
+                                   int min_k, int kmax, int32_t* out, int32_t* dev_status,
+                                   float* cv, int* ci) {
   const int lane = threadIdx.x & 31;
   const unsigned lt = lanemask_lt();
   float e[KPL];
@@ -349,34 +399,48 @@ __device__ int select_mass_row_reg(const float* __restrict__ srow, int nT, float
 #pragma unroll
   for (int i = 0; i < KPL; ++i) mx = fmaxf(mx, e[i]);
   mx = warp_max(mx);
-  float tot = 0.f;
+  float tot = 0.f, mn = INFINITY;
 #pragma unroll
   for (int i = 0; i < KPL; ++i) {
     if (lane + 32 * i < nT) {
       e[i] = expf(scale * (e[i] - mx));
       tot += e[i];
+      mn = fminf(mn, e[i]);
     } else {
       e[i] = -1.f;
     }
   }
   tot = warp_sum(tot);
+  mn = -warp_max(-mn);
   const float target = mass * tot;
   uint32_t prefix = 0;
   bool found = false;
+  int need_fin = -1;  // need_eq from finish_bracket, when it ran
   {
-    float lo = 0.f, hi = 2.f;
+    float lo = mn, hi = __int_as_float(0x3f800001);  // every e lies in [mn, 1]
     float Flo = tot, Fhi = 0.f;
     int clo = nT, chi = 0;
     float wlo = 1.f, whi = 1.f;
     int side = 0;
     for (int step = 0; step < 24; ++step) {
-      if (clo - chi == 1) {
-        float v = -1.f;
+      if (clo - chi <= 32) {
+        int base = 0;
 #pragma unroll
-        for (int i = 0; i < KPL; ++i)
-          if (e[i] >= lo && e[i] < hi) v = e[i];
-        v = warp_max(v);
-        prefix = float_key(v);
+        for (int i = 0; i < KPL; ++i) {
+          const bool inb = e[i] >= lo && e[i] < hi;  // pads hold -1 < lo
+          const unsigned bb = __ballot_sync(0xffffffffu, inb);
+          if (inb) {
+            cv[base + __popc(bb & lt)] = e[i];
+            ci[base + __popc(bb & lt)] = lane + 32 * i;
+          }
+          base += __popc(bb);
+        }
+        __syncwarp();
+        const int c = clo - chi;
+        const float v = lane < c ? cv[lane] : -2.f;
+        const int ix = lane < c ? ci[lane] : 0x7fffffff;
+        __syncwarp();
+        prefix = float_key(finish_bracket(v, ix, c, Fhi, target, need_fin));
         found = true;
         break;
       }
@@ -433,8 +497,8 @@ __device__ int select_mass_row_reg(const float* __restrict__ srow, int nT, float
   above = warp_sum(above);
   n_above = warp_sum_int(n_above);
   // Tiles tied at the threshold are taken in ascending index until the target is reached.
-  int need_eq = 0;
-  {
+  int need_eq = need_fin > 0 ? need_fin : 0;
+  if (need_fin < 0) {
     float acc = above;
     bool done = false;
 #pragma unroll
@@ -789,6 +853,8 @@ __global__ void __launch_bounds__(kSelThreads) mass_rows_kernel(Geo g, const flo
                                                                 int32_t* __restrict__ kv_cnt,
                                                                 int32_t* dev_status) {
   extern __shared__ float rowbuf[];  // KPL == 0: [8 warps][nT]
+  __shared__ float cv[kSelThreads / 32][32];  // finish_bracket's candidates, per warp
+  __shared__ int ci[kSelThreads / 32][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nT = g.nT;
   const long rows = (long)g.B * g.heads * nT;
@@ -800,10 +866,11 @@ __global__ void __launch_bounds__(kSelThreads) mass_rows_kernel(Geo g, const flo
       float* row = rowbuf + (long)w * nT;
       for (int j = lane; j < nT; j += 32) row[j] = src[j];
       __syncwarp();
-      count = select_mass_row(row, nT, scale, mass, min_k, kmax, kv_idx + r * kmax, dev_status);
+      count = select_mass_row(row, nT, scale, mass, min_k, kmax, kv_idx + r * kmax, dev_status,
+                              cv[w], ci[w]);
     } else {
       count = select_mass_row_reg<KPL>(src, nT, scale, mass, min_k, kmax, kv_idx + r * kmax,
-                                       dev_status);
+                                       dev_status, cv[w], ci[w]);
     }
     if (lane == 0) kv_cnt[r] = count;  // -1 - k: mass_fix_kernel keeps the top k instead
     __syncwarp();

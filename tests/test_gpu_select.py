@@ -95,6 +95,28 @@ def test_mass_matches_oracle(grid, D, scale, tau, min_k):
         assert n >= 0.3 * B * heads * nT
 
 
+@pytest.mark.parametrize("grid", [(12, 20, 40), (16, 32, 56), (16, 40, 88), (20, 40, 88)])
+@pytest.mark.parametrize("scale,ties", [(0.088388, False), (0.088388, True), (1.0, True)])
+def test_mass_long_rows(grid, scale, ties):
+    """Rows of 150, 448, 880 and 1,100 tiles: every register width of the row search (8, 16 and 32
+    values per lane) and the shared-memory one, on near-uniform rows (scale 1/sqrt(128): the
+    bracket search ends with a ranked handful of candidates) and with exact ties among the keys."""
+    T, H, W = grid
+    nT = len(tiling.variable_block_sizes(T, H, W))
+    B, heads, D, tau = 1, 2, 128, 0.9
+    pq, pk = _pooled(B, heads, nT, D, seed=nT + int(10 * scale) + ties, ties=ties)
+    kv_idx, kv_cnt = tile_select_mass(pq.cuda(), pk.cuda(), T, H, W, scale, tau, 1)
+    S = select.tile_scores(f64(pq), f64(pk))
+    n = _check_mass(gpu_sets(kv_idx, kv_cnt), S, scale, tau, 1)
+    # Share of rows whose cut is decided by more than the gap rule (oracle, these seeds): 88-90% at
+    # scale 1; at scale 1/sqrt(128) 33-36% of the 150-tile rows and under 4% of the longer ones,
+    # whose other rows are checked as valid prefixes of the ranking with mass ~ tau.
+    if scale == 1.0:
+        assert n >= 0.8 * B * heads * nT
+    elif nT <= 256:
+        assert n >= 0.3 * B * heads * nT
+
+
 def test_mass_overflow_truncates_to_most_probable():
     T, H, W, D = 9, 10, 13, 64
     nT = 36
