@@ -12,12 +12,14 @@ import pytest
 import oracle.attention
 import oracle.attention_bwd
 import oracle.bsa
+import oracle.packed
 import oracle.pool
 import oracle.select
 import oracle.tiling
 from tests import test_oracle_attention as ta
 from tests import test_oracle_attention_bwd as tb
 from tests import test_oracle_bsa_ratio as tr
+from tests import test_oracle_packed as tk
 from tests import test_oracle_pool_select as tp
 from tests import test_oracle_tiling as tt
 
@@ -118,6 +120,94 @@ def _bwd_pruned_keep_own_grad(qt, kt, vt, vc, sets, scale, do, keep=None, src=No
     return dq, dk, dv
 
 
+_orig_packed_geometry = oracle.packed.packed_geometry
+
+
+def _geometry_partial_run_first(segs, tile_shape):
+    """Dense segments cut with their partial run first instead of last."""
+    geo = _orig_packed_geometry(segs, tile_shape)
+    E = geo["E"]
+    sr, vc = geo["slot_row"].copy(), geo["vc"].copy()
+    t, off = 0, 0
+    for s in segs:
+        if isinstance(s, int):
+            n = -(-s // E)
+            sizes = [s - E * (n - 1)] + [E] * (n - 1)
+            for sz in sizes:
+                sr[E * t:E * (t + 1)] = -1
+                sr[E * t:E * t + sz] = np.arange(off, off + sz)
+                vc[t] = sz
+                off += sz
+                t += 1
+        else:
+            off += s[0] * s[1] * s[2]
+    return dict(geo, slot_row=sr, vc=vc)
+
+
+def _geometry_regions_in_64_shape(segs, tile_shape):
+    """Every region tiled with the 64-token shape whatever the tile size."""
+    E = int(np.prod(tile_shape))
+    geo = _orig_packed_geometry(segs, (4, 4, 4))
+    if E == 64:
+        return geo
+    n = len(geo["vc"])
+    sr = np.full(n * E, -1, dtype=np.int64)
+    for t in range(n):
+        sr[E * t:E * t + 64] = geo["slot_row"][64 * t:64 * (t + 1)]
+    return dict(geo, slot_row=sr, E=E)
+
+
+def _select_ceil(S, geo, keep_rates, exempt=True, dense=False):
+    """Per-region keep count rounded up instead of truncated."""
+    nT = S.shape[-1]
+
+    def top(row, lo, hi, rate):
+        order = sorted(range(lo, hi), key=lambda j: (-row[j], j))
+        return order[:min(hi - lo, math.ceil(rate * (hi - lo)))]
+
+    def row_sets(row, i):
+        if dense or (exempt and i < geo["n_prefix"]):
+            return np.arange(nT)
+        if not exempt:
+            return np.asarray(sorted(top(row, 0, nT, keep_rates[-1])))
+        kept = list(range(geo["n_prefix"]))
+        for (lo, hi), r in zip(geo["spans"], keep_rates):
+            kept += top(row, lo, hi, r)
+        return np.asarray(sorted(kept))
+
+    return [[[row_sets(S[b, h, i], i) for i in range(nT)] for h in range(S.shape[1])]
+            for b in range(S.shape[0])]
+
+
+_orig_select = oracle.packed.select
+
+
+def _select_prefix_queries_not_exempt(S, geo, keep_rates, exempt=True, dense=False):
+    """Prefix query tiles select like video query tiles."""
+    return _orig_select(S, dict(geo, n_prefix=0, spans=[(0, geo["n_prefix"])] + list(geo["spans"])),
+                        [1.0] + list(keep_rates), exempt, dense)
+
+
+def _select_rates_reversed(S, geo, keep_rates, exempt=True, dense=False):
+    return _orig_select(S, geo, list(keep_rates)[::-1], exempt, dense)
+
+
+def _rates_generated_first(n_regions, sparsity, ref_keep_rate, exempt):
+    r = _orig_rates(n_regions, sparsity, ref_keep_rate, exempt)
+    return r[-1:] + r[:-1]
+
+
+_orig_rates = oracle.packed.span_keep_rates
+
+
+def _scatter_pads_one(x, geo):
+    y = np.ones((x.shape[0], geo["slot_row"].shape[0]) + x.shape[2:], dtype=x.dtype)
+    for slot, r in enumerate(geo["slot_row"]):
+        if r >= 0:
+            y[:, slot] = x[:, r]
+    return y
+
+
 @pytest.mark.parametrize("patch,pin", [
     ((oracle.tiling, "tile_partition_indices", _swapped_partition),
      lambda: tt.test_partition_matches_sort_by_tile_key((5, 9, 9))),
@@ -136,6 +226,16 @@ def _bwd_pruned_keep_own_grad(qt, kt, vt, vc, sets, scale, do, keep=None, src=No
     ((oracle.attention_bwd, "attend_rows_bwd", _bwd_dk_unscaled), tb.test_finite_differences_tiny),
     ((oracle.attention_bwd, "block_sparse_attention_bwd", _bwd_pruned_keep_own_grad),
      tb.test_pruned_rows_route_their_gradient_to_the_source_row),
+    ((oracle.packed, "packed_geometry", _geometry_partial_run_first),
+     tk.test_geometry_mixed_tile64_fixture),
+    ((oracle.packed, "packed_geometry", _geometry_regions_in_64_shape),
+     tk.test_geometry_tile128_fixture),
+    ((oracle.packed, "select", _select_ceil), tk.test_select_hand_worked_row),
+    ((oracle.packed, "select", _select_prefix_queries_not_exempt), tk.test_select_hand_worked_row),
+    ((oracle.packed, "select", _select_rates_reversed), tk.test_select_hand_worked_row),
+    ((oracle.packed, "span_keep_rates", _rates_generated_first),
+     tk.test_token_segments_and_keep_rates_contract),
+    ((oracle.packed, "scatter", _scatter_pads_one), tk.test_scatter_gather_round_trip_and_zero_pads),
 ])
 def test_planted_mistake_is_caught(monkeypatch, patch, pin):
     mod, name, fn = patch
