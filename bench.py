@@ -291,6 +291,7 @@ STATIC_KERNELS = {
     "attention": 1,
     "attention_packed": 2,  # packed: list rewrite into 64-row halves, attention
     "gather": 1,
+    "backward": 5,      # dOe / delta, kept-pair map, key-to-query lists, dQ, dK / dV
 }
 
 
@@ -592,6 +593,7 @@ def run_backward(args, w):
     e1.record()
     torch.cuda.synchronize()
     clocks = sampler.stop()
+    launches, launch_src = count_launches([("backward", call)])
     ms = e0.elapsed_time(e1) / args.steps
     pairs = int(model.kv_cnt.sum().item())
     flops = pairs * 10 * 64 * 64 * w.D
@@ -608,6 +610,8 @@ def run_backward(args, w):
                          "unit": "TFLOP/s", "frac": tflops / peaks["bf16_tflops"],
                          "traffic": None, "kernel": "block_sparse_attn_bwd (all launches)",
                          "peak_source": f"{peaks['source']} bf16 dense (burst)"},
+            "gpu_launches": args.steps * launches["backward"],
+            "gpu_launches_per_step": {"by_stage": launches, "source": launch_src},
             "device_status": int(status.item()), "clocks": clocks}
     print(json.dumps(line), flush=True)
     return 0
