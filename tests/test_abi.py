@@ -9,6 +9,8 @@ import re
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from block_sparse_video_tile3d_b200 import _lib
 from block_sparse_video_tile3d_b200._lib import Geom, lib
@@ -42,6 +44,17 @@ def test_geometry_matches_oracle(grid):
     from block_sparse_video_tile3d_b200 import geometry
     nT, Lp, vc = geometry(*grid)
     want = tiling.variable_block_sizes(*grid)
+    assert nT == len(want) and Lp == 64 * nT
+    np.testing.assert_array_equal(np.asarray(vc), want)
+
+
+@settings(max_examples=60, deadline=None, derandomize=True)
+@given(T=st.integers(1, 40), H=st.integers(1, 40), W=st.integers(1, 70))
+def test_geometry_matches_oracle_on_random_grids(T, H, W):
+    """Random grids, ragged in every dimension: tile count, padded length and valid counts."""
+    from block_sparse_video_tile3d_b200 import geometry
+    nT, Lp, vc = geometry(T, H, W)
+    want = tiling.variable_block_sizes(T, H, W)
     assert nT == len(want) and Lp == 64 * nT
     np.testing.assert_array_equal(np.asarray(vc), want)
 

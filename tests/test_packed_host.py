@@ -7,6 +7,8 @@ import math
 
 import numpy as np
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 from block_sparse_video_tile3d_b200 import _lib
 from block_sparse_video_tile3d_b200._lib import lib
@@ -25,6 +27,24 @@ SEQS = [
 @pytest.mark.parametrize("E", [64, 128])
 @pytest.mark.parametrize("seq", SEQS)
 def test_geometry_matches_oracle(seq, E):
+    geo = PackedGeometry(seq, tile_size=E, device="cpu")
+    ref = opacked.packed_geometry(opacked.token_segments(seq, (1, 1, 1)), TILE_SHAPES[E])
+    assert geo.rows == ref["rows"] and geo.n_prefix == ref["n_prefix"]
+    assert geo.spans == [tuple(s) for s in ref["spans"]]
+    assert geo.vc == ref["vc"].tolist()
+    assert geo.slot_row_host == ref["slot_row"].tolist()
+
+
+_segment = st.one_of(st.integers(1, 300),
+                     st.tuples(st.integers(1, 12), st.integers(1, 12), st.integers(1, 12)))
+
+
+@settings(max_examples=40, deadline=None, derandomize=True)
+@given(seq=st.lists(_segment, min_size=1, max_size=6).filter(
+    lambda q: any(isinstance(x, tuple) for x in q)), E=st.sampled_from([64, 128]))
+def test_geometry_matches_oracle_on_random_sequences(seq, E):
+    """Random mixes of dense runs and regions (ragged every way): the library's host geometry is
+    the oracle's, slot for slot."""
     geo = PackedGeometry(seq, tile_size=E, device="cpu")
     ref = opacked.packed_geometry(opacked.token_segments(seq, (1, 1, 1)), TILE_SHAPES[E])
     assert geo.rows == ref["rows"] and geo.n_prefix == ref["n_prefix"]
