@@ -3,7 +3,6 @@ rows per 64-row block (the rows least cosine-similar to the block mean), then th
 kept-query pooling, mass selection and attention as the threshold mode."""
 import numpy as np
 import pytest
-import torch
 
 from block_sparse_video_tile3d_b200 import (TileSparseAttention, tile3d_scatter,
                                             tile_prune_queries_ratio, workloads)

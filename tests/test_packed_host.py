@@ -5,7 +5,6 @@ selection reading, and bad arguments are rejected on the host (no GPU: nothing h
 import ctypes
 import math
 
-import numpy as np
 import pytest
 from hypothesis import given, settings
 from hypothesis import strategies as st
