@@ -269,13 +269,16 @@ def _stage_bytes(w, name, pairs, kmax):
     return 0
 
 
+ATTN_SOURCES = ("attn_sm100.cu", "common.cuh", "kernels.h", "sm100.cuh")  # the forward kernel's
+
+
 def _source_sha() -> str:
+    """Hash of the sources the forward attention kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "block_sparse_video_tile3d_b200", "csrc")
-    for n in sorted(os.listdir(csrc)):
-        if n.startswith("attn") or n in ("common.cuh", "kernels.h", "sm100.cuh"):
-            with open(os.path.join(csrc, n), "rb") as f:
-                h.update(n.encode() + f.read())
+    for n in sorted(ATTN_SOURCES):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(n.encode() + f.read())
     return h.hexdigest()[:16]
 
 
